@@ -1,0 +1,149 @@
+"""Seeded synthetic inputs for the KDA decode step.
+
+This module draws random numbers and nothing else: it holds none of the
+decode step's arithmetic, so both the CUDA path and the fp64 oracle can take
+their inputs from it without sharing any computation.  All tensors are made on
+the CPU with ``torch.Generator`` (seeded) and may then be copied to a device.
+
+Input recipe (every configuration, unless stated otherwise):
+  * state pool fp32 ``[num_slots, HV, K, V]`` ~ N(0, 0.02^2) (0.02 is the std);
+  * q, k, v drawn fp32 ~ N(0, 1); q and k are L2-normalised over K per
+    (n, t, h) in fp32 and then all three are rounded to bf16;
+  * g fp32 ``[N, T, HV, K]`` = -softplus(N(0, 1)) per key channel (log-decay);
+  * beta fp32 ``[N, T, HV]`` = sigmoid(N(0, 1));
+  * slot_idx int32 ``[N]``: distinct slots drawn by a random permutation;
+  * gated variant: gate z bf16 ``[N, T, HV, V]`` ~ N(0, 1), RMS-norm weight
+    bf16 ``[V]`` ~ N(1, 0.1^2), eps = 1e-6;
+  * scale = 1/sqrt(K).
+
+The shapes follow the serving shapes of the pages: K = V = 128 and 8 local
+value heads with N = 32 sequences dominating decode graphs (vLLM #57585,
+"Retained baseline trace attribution"), T = 4 for speculative decode
+(vLLM #57585, "Microbenchmark and earlier serving limits"), a gated RMS norm
+after the decode kernel (b12x #249, sequence diagram).  No public dataset is
+involved; these draws stand in for the activations of a KDA layer.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    N: int
+    T: int
+    HV: int
+    K: int
+    V: int
+    num_slots: int
+    gated: bool
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    g: torch.Tensor
+    beta: torch.Tensor
+    state: torch.Tensor
+    slot_idx: torch.Tensor
+    scale: float
+    gate: torch.Tensor | None = None
+    norm_weight: torch.Tensor | None = None
+    eps: float = 1e-6
+
+    def tensors(self):
+        """Dict of the call's tensors (gate/norm_weight only when gated)."""
+        d = dict(q=self.q, k=self.k, v=self.v, g=self.g, beta=self.beta,
+                 state=self.state, slot_idx=self.slot_idx)
+        if self.gated:
+            d.update(gate=self.gate, norm_weight=self.norm_weight)
+        return d
+
+    def to(self, device, state_too: bool = True) -> "Workload":
+        """Copy of the workload with its tensors on ``device``."""
+        upd = {}
+        for key, t in self.tensors().items():
+            if key == "state" and not state_too:
+                continue
+            upd[key] = t.to(device)
+        return dataclasses.replace(self, **upd)
+
+    def io_bytes(self) -> int:
+        """Bytes of per-call inputs and outputs other than the state pool."""
+        n = (self.q.numel() + self.k.numel() + self.v.numel()) * 2 + self.g.numel() * 4
+        n += self.beta.numel() * 4 + self.slot_idx.numel() * 4 + self.N * self.T * self.HV * self.V * 2
+        if self.gated:
+            n += self.gate.numel() * 2 + self.norm_weight.numel() * 2
+        return n
+
+    def state_bytes_touched(self) -> int:
+        """State bytes one call reads (it writes the same amount back)."""
+        active = int((self.slot_idx >= 0).sum())
+        return active * self.HV * self.K * self.V * 4
+
+
+def _bf16(x: torch.Tensor) -> torch.Tensor:
+    return x.to(torch.bfloat16)
+
+
+def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | None = None,
+         gated: bool = False, seed: int = 0, name: str = "custom",
+         decay: str = "softplus", inactive: int = 0, state_std: float = 0.02) -> Workload:
+    """Draw one call's inputs.
+
+    ``decay``: ``"softplus"`` (g = -softplus(N(0,1))) or ``"uniform"``
+    (exp(g) ~ U[0.5, 1)).  ``inactive``: how many rows (the last ones) get a
+    negative slot index, as CUDA-graph padding rows do.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    if num_slots is None:
+        num_slots = max(1, 2 * N)
+    if N > num_slots:
+        raise ValueError("need N <= num_slots for distinct slots")
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    q = randn(N, T, HV, K)
+    k = randn(N, T, HV, K)
+    v = randn(N, T, HV, V)
+    q = q / q.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+    k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+    if decay == "softplus":
+        g = -torch.nn.functional.softplus(randn(N, T, HV, K))
+    elif decay == "uniform":
+        g = torch.log(0.5 + 0.5 * torch.rand(N, T, HV, K, generator=gen, dtype=torch.float32))
+    else:
+        raise ValueError(decay)
+    beta = torch.sigmoid(randn(N, T, HV))
+    state = randn(num_slots, HV, K, V) * state_std
+    slot_idx = torch.randperm(num_slots, generator=gen)[:N].to(torch.int32)
+    if inactive:
+        slot_idx[N - inactive:] = -1
+    gate = norm_weight = None
+    if gated:
+        gate = _bf16(randn(N, T, HV, V))
+        norm_weight = _bf16(1.0 + 0.1 * randn(V))
+    return Workload(name=name, N=N, T=T, HV=HV, K=K, V=V, num_slots=num_slots, gated=gated,
+                    q=_bf16(q), k=_bf16(k), v=_bf16(v), g=g.contiguous(), beta=beta.contiguous(),
+                    state=state.contiguous(), slot_idx=slot_idx.contiguous(),
+                    scale=1.0 / math.sqrt(K), gate=gate, norm_weight=norm_weight)
+
+
+# The five workloads: name -> keyword arguments of ``make``.
+CONFIGS = {
+    "n1_t1_hv8": dict(N=1, T=1, HV=8, num_slots=1),
+    "n32_t1_hv8": dict(N=32, T=1, HV=8, num_slots=64),
+    "n32_t1_hv16_gated": dict(N=32, T=1, HV=16, num_slots=128, gated=True),
+    "n1_t4_hv8": dict(N=1, T=4, HV=8, num_slots=2),
+    "n8_t4_hv8": dict(N=8, T=4, HV=8, num_slots=16),
+    "n32_t4_hv8": dict(N=32, T=4, HV=8, num_slots=64),
+    "n256_t1_hv32": dict(N=256, T=1, HV=32, num_slots=1024, decay="uniform"),
+}
+
+
+def config(name: str, seed: int = 0) -> Workload:
+    """One of the named workloads (K = V = 128), drawn with ``seed``."""
+    return make(name=name, seed=seed, **CONFIGS[name])
