@@ -1,0 +1,451 @@
+#!/usr/bin/env python3
+"""Benchmark of the recurrent KDA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one ``kda_decode`` call over one batch (default workload
+``n32_t1_hv8``: N=32 sequences, T=1 token, HV=8 value heads, K=V=128, fp32
+state pool of 64 slots).  The timed region replays, from a CUDA graph, K calls
+that rotate over R independent replicas of the inputs and pool whose combined
+touched bytes exceed twice the L2 cache, so every call reads its state from
+HBM (the pages' cold-L2 graph-replay method).  Timing uses CUDA events on the
+launching stream with a device synchronize on both sides; under torchrun each
+rank runs its own batch (weak scaling, no collective on the data path) and the
+reported time is the maximum over ranks.
+
+Printed (rank 0, one JSON line): µs per call for the whole job, the achieved
+HBM bandwidth of the decode kernel against the measured copy bandwidth
+(roofline), the fp64 oracle timed on the host cores (cpu_baseline), the same
+metric end to end through the public Python API with pinned host buffers
+(e2e), SM clocks sampled during the timed region, and the kernel launch count.
+
+``--impl reference`` times the fp64 oracle instead (on rank 0, host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA decode µs/call and achieved HBM GB/s (% of B200 peak) at N32/T1/HV8"
+UNIT = "us/call"
+FALLBACK_HBM_GBS = 6650.0
+CSRC = os.path.join(ROOT, "linear_attention_recurrent_decode_b200", "csrc")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "kda_decode_n32_t1_hv8.md")
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Maximum of ``value`` over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): disjoint seed streams."""
+    return base + 100_003 * rank
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source and this workload; else None."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    fields = {}
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if line.startswith("- ") and ":" in line:
+                key, val = line[2:].split(":", 1)
+                fields[key.strip()] = val.strip().strip("`")
+    if fields.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    if fields.get("workload") != workload:
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi SM clocks and throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.text = ""
+        try:
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.cmd = ["nvidia-smi", "-i", gid, f"--query-gpu={','.join(self.FIELDS)}",
+                        "--format=csv,noheader,nounits", "-lms", "100"]
+        except Exception:
+            self.cmd = None
+
+    def __enter__(self):
+        if self.cmd:
+            try:
+                self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                             text=True)
+            except OSError:
+                self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.text, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.text, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for rec in csv.reader(io.StringIO(self.text)):
+            if len(rec) != len(self.FIELDS):
+                continue
+            try:
+                rows.append([x.strip() for x in rec])
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        smax = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+def call_fn(kda, d, out, stream):
+    if d.gated:
+        return lambda: kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx,
+                                                    d.gate, d.norm_weight, eps=d.eps, out=out,
+                                                    scale=d.scale, stream=stream)
+    return lambda: kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, out=out,
+                                  scale=d.scale, stream=stream)
+
+
+def choose_replicas(touched_bytes: int, l2_bytes: int) -> int:
+    """Enough replicas that the bytes touched between two uses of one replica
+    exceed twice the L2 size."""
+    return max(2, int(math.ceil(2 * l2_bytes / max(1, touched_bytes))) + 1)
+
+
+def time_cpu_oracle(w, budget_s: float = 8.0, max_calls: int = 200):
+    """Median wall time of the fp64 oracle on the full call, all host cores."""
+    import numpy as np
+
+    import oracle
+
+    threads = os.cpu_count() or 1
+    pool = w.state.double().numpy().copy()
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while len(times) < max_calls and (len(times) < 3 or time.perf_counter() < t_end):
+        t0 = time.perf_counter()
+        oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, None, w.slot_idx, w.scale,
+                              gate=w.gate if w.gated else None,
+                              norm_weight=w.norm_weight if w.gated else None, eps=w.eps,
+                              threads=threads, state_inplace=pool)
+        times.append(time.perf_counter() - t0)
+    return statistics.median(times), threads, len(times)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import linear_attention_recurrent_decode_b200 as kda
+    from linear_attention_recurrent_decode_b200 import workloads
+
+    rank, local_rank, world = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    kda.library()
+
+    base = workloads.config(args.config, seed=rank_seed(0, rank))
+    bytes_per_call = base.io_bytes() + 2 * base.state_bytes_touched()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = args.replicas or choose_replicas(base.state_bytes_touched() + base.io_bytes(), l2)
+    reps = [base.to(dev)] + [workloads.config(args.config, seed=rank_seed(1 + r, rank)).to(dev)
+                             for r in range(R - 1)]
+    outs = [torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=dev) for w in reps]
+    stream = torch.cuda.Stream(device=dev)
+    calls = [call_fn(kda, d, o, stream) for d, o in zip(reps, outs)]
+
+    # warm-up: W eager calls on the timing stream
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            calls[i % R]()
+    torch.cuda.synchronize()
+
+    # CUDA graphs: one of R calls (replayed) and one of the K mod R remainder
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for fn in fns:
+                    fn()
+        return g
+
+    full, rem = divmod(args.steps, R)
+    g_full = capture(calls) if full else None
+    g_rem = capture(calls[:rem]) if rem else None
+    with torch.cuda.stream(stream):  # graph upload + one more untimed pass
+        if g_full:
+            g_full.replay()
+        if g_rem:
+            g_rem.replay()
+    torch.cuda.synchronize()
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if (rank == 0 and not args.no_clocks) else None
+    if sampler:
+        sampler.__enter__()
+        time.sleep(0.25)
+    t_wall0 = time.perf_counter()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(full):
+            g_full.replay()
+        if g_rem:
+            g_rem.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    if sampler:
+        sampler.__exit__(None, None, None)
+    if world > 1:
+        dist.barrier()
+    ms_rank = e0.elapsed_time(e1)
+    ms_max = reduce_max(ms_rank, dev)
+    del g_full, g_rem
+
+    # end to end through the public API: pinned host inputs in, output back out
+    e2e = run_e2e(kda, base, dev, stream, min(args.steps, args.e2e_steps), world)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    us_per_call_job = ms_max * 1e3 / (args.steps * world)
+    launch_us = ms_max * 1e3 / args.steps
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_per_call / (launch_us * 1e-6) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        t_cpu, cores, n_calls = time_cpu_oracle(base)
+        cpu = {"value": t_cpu * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n_calls} full calls of {args.config} (fp64 C loop, threads over (n,h))"}
+    clocks = sampler.summary() if sampler else None
+    line = {
+        "metric": METRIC, "value": round(us_per_call_job, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; bf16 q/k/v, fp32 g/beta/state)",
+        "config": {"workload": args.config, "N": base.N, "T": base.T, "HV": base.HV, "K": base.K,
+                   "V": base.V, "num_slots": base.num_slots, "gated": base.gated,
+                   "replicas": R, "l2": f"inputs larger than L2: {R} rotating replicas touch "
+                   f"{R * (base.state_bytes_touched() + base.io_bytes()) / 1e6:.0f} MB > 2 x "
+                   f"{l2 / 1e6:.0f} MB L2", "timing": "CUDA graph replay, CUDA events",
+                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "gbs": round(achieved, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": bytes_per_call,
+                     "traffic": profiled_traffic(args.config)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": args.steps,
+        "wall_s_timed": round(t_wall, 3),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(kda, w, dev, stream, steps, world):
+    """µs per call with each step's inputs copied from pinned host memory and its
+    output read back, through the public Python API, eager launches."""
+    import torch
+
+    host = {k: t.pin_memory() for k, t in w.tensors().items() if k != "state"}
+    devbuf = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
+    pool = w.state.to(dev)
+    out_d = torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty(out_d.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for k in host:
+            devbuf[k].copy_(host[k], non_blocking=True)
+        if w.gated:
+            kda.kda_decode_gated_rmsnorm(devbuf["q"], devbuf["k"], devbuf["v"], devbuf["g"], devbuf["beta"],
+                                         pool, devbuf["slot_idx"], devbuf["gate"], devbuf["norm_weight"],
+                                         eps=w.eps, scale=w.scale, out=out_d, stream=stream)
+        else:
+            kda.kda_decode(devbuf["q"], devbuf["k"], devbuf["v"], devbuf["g"], devbuf["beta"], pool,
+                           devbuf["slot_idx"], scale=w.scale, out=out_d, stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1), dev)
+    return {"value": round(ms * 1e3 / (steps * world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "how": "eager public-API calls; pinned host inputs copied in and the output copied out "
+                   "every step; the state pool stays resident on the GPU"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """fp64 oracle on the host cores, same workload/metric; rank 0 only."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    from linear_attention_recurrent_decode_b200 import workloads
+    import oracle
+
+    w = workloads.config(args.config)
+    units = w.N * w.HV
+    threads = os.cpu_count() or 1
+    pool = w.state.double().numpy().copy()
+    kw = dict(gate=w.gate, norm_weight=w.norm_weight, eps=w.eps) if w.gated else dict(eps=w.eps)
+
+    def one(lo, hi, thr):
+        t0 = time.perf_counter()
+        oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, None, w.slot_idx, w.scale, threads=thr,
+                              units=(lo, hi), state_inplace=pool, **kw)
+        return time.perf_counter() - t0
+
+    t_full = min(one(0, units, threads) for _ in range(2))
+    budget = args.reference_budget_s
+    total = args.steps + args.warmup
+    if total * t_full <= budget:
+        per_step, thr = units, threads
+    else:
+        per_step = max(1, min(units, int(units * budget / (total * t_full))))
+        thr = max(1, min(threads, per_step))
+    times = []
+    lo = 0
+    for i in range(total):
+        hi = min(units, lo + per_step)
+        dt = one(lo, hi, thr)
+        if i >= args.warmup:
+            times.append(dt * units / (hi - lo))
+        lo = 0 if hi >= units else hi
+    us = statistics.mean(times) * 1e6
+    sample = (f"each step: units [{per_step} of {units}] (n,h) of {args.config}, scaled to a full call"
+              if per_step < units else f"each step: one full call of {args.config}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; bf16 q/k/v, fp32 g/beta/state)",
+        "config": {"workload": args.config, "N": w.N, "T": w.T, "HV": w.HV, "K": w.K, "V": w.V,
+                   "num_slots": w.num_slots, "gated": w.gated},
+        "cpu_baseline": {"value": round(us, 3), "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(us, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200_000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--config", default="n32_t1_hv8")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--replicas", type=int, default=0, help="0 = enough to exceed 2x L2")
+    ap.add_argument("--e2e-steps", type=int, default=5000)
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-budget-s", type=float, default=90.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.steps < 1:
+        raise SystemExit("--steps must be >= 1")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

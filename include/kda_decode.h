@@ -1,0 +1,135 @@
+/*
+ * kda_decode.h -- C ABI of the B200 (sm_100a) recurrent Kimi Delta Attention
+ * (KDA) decode step.
+ *
+ * The operation.  For every sequence n in [0, N), value head h in [0, HV) and
+ * token t in [0, T), applied in token order to the fp32 state S[K][V] that the
+ * sequence keeps in slot slot_idx[n] of a caller-owned state pool:
+ *
+ *     S   <- Diag(exp(g[n,t,h,:])) S                 per-key-channel decay
+ *     u   <- beta[n,t,h] * (v[n,t,h,:] - S^T k[n,t,h,:])   delta-rule correction
+ *     S   <- S + k[n,t,h,:] u^T                       rank-1 write
+ *     o   <- scale * S^T q[n,t,h,:]                   readout of the updated state
+ *     out[n,t,h,:] <- bf16(o)                          (kda_decode)
+ *     out[n,t,h,:] <- bf16(o / sqrt(mean(o^2) + eps) * w * sigmoid(z[n,t,h,:]))
+ *                                                     (kda_decode_gated_rmsnorm)
+ *
+ * Where it comes from (pages by title):
+ *   - vLLM #57585 "Tune recurrent KDA launch configuration on SM90",
+ *     "Microbenchmark and earlier serving limits": BF16 q/k/v, FP32 recurrent
+ *     state, K = V = 128; "Retained baseline trace attribution": one recurrent
+ *     KDA call per KDA layer per decode step, 8 local heads, head dim 128.
+ *   - FlashInfer #4562 "feat(cake_kda): add optimized H12 packed decode across
+ *     SM100 family": the kernel updates the state and writes the output
+ *     (sequence diagram); the slot table `state_indices` and the scale
+ *     0.08838834764831845 = 1/sqrt(128) are kernel arguments (binding launch);
+ *     caller-stream execution, caller-owned output, indexed recurrent state,
+ *     inactive graph-padding rows, CUDA graph replay (PR description).
+ *   - b12x #249 "feat(gdn): add direct single-token KDA decode": decode, then
+ *     a gated RMS norm of the decoded output with z (sequence diagram);
+ *     output must not overlap the read-only inputs (review of `_overlaps`).
+ *   None of the pages prints the recurrence as a formula: the step order
+ *   above (decay, correction on the decayed state, write, readout after the
+ *   write) is the plainest reading that all of them support.
+ *
+ * Layouts.  Every tensor is dense, row-major (last index fastest), in device
+ * memory of the current CUDA device:
+ *     q, k        bf16  [N, T, HV, K]     (one q/k head per value head)
+ *     v           bf16  [N, T, HV, V]
+ *     g           fp32  [N, T, HV, K]     log-decay, decay = exp(g)
+ *     beta        fp32  [N, T, HV]
+ *     state_pool  fp32  [num_slots, HV, K, V], read and written in place
+ *     slot_idx    int32 [N]               slot of each row; < 0 = inactive row
+ *     out         bf16  [N, T, HV, V]
+ *     gate (z)    bf16  [N, T, HV, V]     gated variant only
+ *     norm_weight bf16  [V]               gated variant only, shared by heads
+ *
+ * Supported sizes: K in {64, 128, 256}; V a multiple of 32; V <= 256 for the
+ * gated variant (its V tiles form one thread-block cluster); HV >= 1;
+ * N, T >= 0 (N == 0 or T == 0 is a no-op that touches no pointer).
+ * Alignment: q, k, v, g, state_pool, out, gate, norm_weight on 16 bytes;
+ * beta and slot_idx on 4 bytes.
+ *
+ * Ownership and execution.  The caller owns every buffer.  A call allocates
+ * nothing, never synchronises the host, and enqueues exactly one kernel on
+ * `stream` (NULL = the legacy default stream); it can be captured in a CUDA
+ * graph.  The first call on a device reads that device's compute capability
+ * once and caches it.
+ *
+ * Caller contract (checked only where noted):
+ *   - active slots in slot_idx are distinct and < num_slots (the pool size is
+ *     not an argument, so the library cannot check the upper bound);
+ *   - rows with slot_idx[n] < 0 get an all-zero output and do not touch the
+ *     pool (CUDA-graph padding rows);
+ *   - out overlaps no input and no part of the pool; the library rejects an
+ *     out/input overlap, and any buffer that starts inside the pool's slot-0
+ *     block or that contains the pool base (KDA_ERR_ALIAS).
+ *
+ * Errors.  Every entry point validates on the host and returns a status; it
+ * never aborts, throws or prints.  Nothing is enqueued unless it returns
+ * KDA_OK.  KDA_ERR_CUDA reports a failed launch (cudaGetLastError is not
+ * consumed for unrelated earlier errors).
+ */
+#ifndef KDA_DECODE_H
+#define KDA_DECODE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+struct CUstream_st;
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null pointer with work to do, negative size, bad eps */
+    KDA_ERR_UNSUPPORTED = 2, /* K, V or HV outside the supported set */
+    KDA_ERR_ALIAS = 3,       /* out overlaps an input or the pool */
+    KDA_ERR_MISALIGNED = 4,  /* a pointer breaks the alignment rule above */
+    KDA_ERR_DEVICE = 5,      /* current device is not compute capability 10.0 */
+    KDA_ERR_CUDA = 6         /* the CUDA runtime refused the launch */
+} kda_status;
+
+/*
+ * Plain decode step (see the top of this file).  Writes bf16(o) to out and the
+ * updated state back to each active row's slot.  scale is usually 1/sqrt(K).
+ */
+KDA_API kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, float *state_pool, const int32_t *slot_idx,
+                      void *out, int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
+                      float scale, kda_stream_t stream);
+
+/*
+ * Decode step followed, in the same kernel, by the gated RMS norm over V of
+ * each (n, t, h) output row: y = o / sqrt(mean_V(o^2) + eps) * norm_weight *
+ * sigmoid(gate), computed in fp32 from the unrounded o, then rounded to bf16
+ * into out.  eps must be finite and >= 0.  The state update is identical to
+ * kda_decode's.
+ */
+KDA_API kda_status kda_decode_gated_rmsnorm(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, float *state_pool,
+                                    const int32_t *slot_idx, const void *gate,
+                                    const void *norm_weight, float eps, void *out, int64_t N,
+                                    int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
+                                    kda_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+KDA_API const char *kda_status_string(kda_status status);
+
+/* Library ABI version: (major << 16) | minor. */
+KDA_API int32_t kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_DECODE_H */

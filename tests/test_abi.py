@@ -1,0 +1,133 @@
+"""The C-ABI library builds, loads and exports every symbol its header declares;
+host-side validation answers without touching a GPU.
+
+The validation tests pass fabricated addresses that the library must reject
+before any launch; they only run where no CUDA device is present, so a
+validation bug can never launch a kernel on them.  The GPU tests repeat the
+rejections with real buffers.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import linear_attention_recurrent_decode_b200 as kda
+from linear_attention_recurrent_decode_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda_decode.h")
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fabricated pointers: CPU-only check")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return kda.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return {re.findall(r"\w+", m)[-1] for m in re.findall(r"^KDA_API([^(;]*)\(", text, re.M)}
+
+
+def test_header_declares_the_documented_entry_points():
+    assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_status_string",
+                                    "kda_abi_version"}
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(kda.EXPORTED_SYMBOLS) == declared_functions()
+
+
+def test_library_exports_nothing_else(lib):
+    out = os.popen(f"nm -D --defined-only {kda.LIBRARY_PATH}").read()
+    syms = {line.split()[-1] for line in out.splitlines() if line.split()[1] in ("T", "t")}
+    assert {s for s in syms if s.startswith("kda_")} == declared_functions()
+
+
+def test_status_strings_and_version(lib):
+    assert kda.status_string(kda.KDA_OK) == "ok"
+    for s in range(1, 7):
+        assert kda.status_string(s) and kda.status_string(s) != "unknown status"
+    assert kda.status_string(99) == "unknown status"
+    assert lib.kda_abi_version() == (1 << 16)
+
+
+# ----------------------------------------------------------------- validation
+BASE = 1 << 40  # never dereferenced: every call below is rejected on the host
+
+
+def call(lib, N=2, T=1, HV=2, K=128, V=128, q=None, k=None, v=None, g=None, beta=None,
+         state=None, slot=None, out=None, gate=None, w=None, eps=1e-6, gated=False):
+    step = 1 << 30
+    ptr = dict(q=BASE, k=BASE + step, v=BASE + 2 * step, g=BASE + 3 * step, beta=BASE + 4 * step,
+               state=BASE + 5 * step, slot=BASE + 8 * step, out=BASE + 9 * step,
+               gate=BASE + 10 * step, w=BASE + 11 * step)
+    for key, val in dict(q=q, k=k, v=v, g=g, beta=beta, state=state, slot=slot, out=out, gate=gate,
+                         w=w).items():
+        if val is not None:
+            ptr[key] = val
+    if gated:
+        return lib.kda_decode_gated_rmsnorm(ptr["q"], ptr["k"], ptr["v"], ptr["g"], ptr["beta"],
+                                            ptr["state"], ptr["slot"], ptr["gate"], ptr["w"], eps,
+                                            ptr["out"], N, T, HV, K, V, 0.1, None)
+    return lib.kda_decode(ptr["q"], ptr["k"], ptr["v"], ptr["g"], ptr["beta"], ptr["state"],
+                          ptr["slot"], ptr["out"], N, T, HV, K, V, 0.1, None)
+
+
+@no_gpu
+@pytest.mark.parametrize("gated", [False, True])
+def test_empty_batches_are_noops_without_pointers(lib, gated):
+    assert call(lib, N=0, q=0, k=0, v=0, g=0, beta=0, state=0, slot=0, out=0, gate=0, w=0,
+                gated=gated) == kda.KDA_OK
+    assert call(lib, T=0, q=0, k=0, v=0, g=0, beta=0, state=0, slot=0, out=0, gate=0, w=0,
+                gated=gated) == kda.KDA_OK
+
+
+@no_gpu
+@pytest.mark.parametrize("gated", [False, True])
+def test_rejections(lib, gated):
+    E = kda
+    assert call(lib, N=-1, gated=gated) == E.KDA_ERR_INVALID_ARG
+    assert call(lib, T=-2, gated=gated) == E.KDA_ERR_INVALID_ARG
+    assert call(lib, HV=0, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, K=96, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, K=512, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, V=100, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, V=0, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, q=0, gated=gated) == E.KDA_ERR_INVALID_ARG
+    assert call(lib, slot=0, gated=gated) == E.KDA_ERR_INVALID_ARG
+    assert call(lib, q=BASE + 8, gated=gated) == E.KDA_ERR_MISALIGNED
+    assert call(lib, state=BASE + 5 * (1 << 30) + 4, gated=gated) == E.KDA_ERR_MISALIGNED
+    assert call(lib, beta=BASE + 4 * (1 << 30) + 2, gated=gated) == E.KDA_ERR_MISALIGNED
+    # out overlapping an input, or the pool
+    assert call(lib, out=BASE + 64, gated=gated) == E.KDA_ERR_ALIAS
+    assert call(lib, out=BASE + 5 * (1 << 30), gated=gated) == E.KDA_ERR_ALIAS
+    # an input starting inside the pool's slot 0
+    assert call(lib, g=BASE + 5 * (1 << 30) + 4096, gated=gated) == E.KDA_ERR_ALIAS
+    if gated:
+        assert call(lib, V=288, gated=True) == E.KDA_ERR_UNSUPPORTED  # 9 tiles > one cluster
+        assert call(lib, gate=0, gated=True) == E.KDA_ERR_INVALID_ARG
+        assert call(lib, w=BASE + 11 * (1 << 30) + 2, gated=True) == E.KDA_ERR_MISALIGNED
+        assert call(lib, eps=-1.0, gated=True) == E.KDA_ERR_INVALID_ARG
+        assert call(lib, eps=float("nan"), gated=True) == E.KDA_ERR_INVALID_ARG
+        assert call(lib, eps=float("inf"), gated=True) == E.KDA_ERR_INVALID_ARG
+        assert call(lib, out=BASE + 10 * (1 << 30), gated=True) == E.KDA_ERR_ALIAS
+
+
+@no_gpu
+def test_valid_call_without_a_device_reports_device_error(lib):
+    assert call(lib) == kda.KDA_ERR_DEVICE
+    assert call(lib, gated=True) == kda.KDA_ERR_DEVICE
+
+
+def test_binding_refuses_cpu_tensors():
+    from linear_attention_recurrent_decode_b200 import workloads
+
+    w = workloads.make(N=1, T=1, HV=1, K=64, V=32, num_slots=1)
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.kda_decode(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx)

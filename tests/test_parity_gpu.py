@@ -1,0 +1,242 @@
+"""Parity of the CUDA path with the fp64 oracle, through the C ABI.
+
+Every test draws seeded inputs from ``workloads`` (shared with the oracle),
+runs the library on the GPU, runs the oracle on the CPU on the same inputs and
+compares element by element with the tolerances of ``tests/parity.py``:
+outputs within 1 bf16 ulp (and 2e-3 normwise), state within 1e-5 relative,
+untouched slots bit-identical.
+"""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_recurrent_decode_b200 as kda
+import oracle
+from linear_attention_recurrent_decode_b200 import workloads
+from tests.parity import check_out, check_state
+
+pytestmark = pytest.mark.gpu
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+def run_gpu(w, dev, out=None, stream=None):
+    """Run one call on ``dev``; returns (out_fp64, pool_after_gpu, pool_before_gpu)."""
+    d = w.to(dev)
+    before = d.state.clone()
+    if w.gated:
+        o = kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, d.gate,
+                                         d.norm_weight, eps=w.eps, scale=w.scale, out=out, stream=stream)
+    else:
+        o = kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, scale=w.scale, out=out,
+                           stream=stream)
+    torch.cuda.synchronize()
+    return o, d.state, before
+
+
+def run_oracle(w, rows=None):
+    """Oracle on all rows, or on the listed rows only (with a compact pool of their slots)."""
+    if rows is None:
+        kw = dict(gate=w.gate, norm_weight=w.norm_weight, eps=w.eps) if w.gated else {}
+        return oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx, w.scale,
+                                     threads=THREADS, **kw)
+    rows = torch.as_tensor(rows)
+    slots = w.slot_idx[rows]
+    compact = w.state[slots.clamp_min(0).long()]
+    local = torch.where(slots >= 0, torch.arange(len(rows), dtype=torch.int32), slots)
+    kw = dict(gate=w.gate[rows], norm_weight=w.norm_weight, eps=w.eps) if w.gated else {}
+    return oracle.kda_decode_ref(w.q[rows], w.k[rows], w.v[rows], w.g[rows], w.beta[rows], compact,
+                                 local, w.scale, threads=THREADS, **kw)
+
+
+def assert_parity(w, o_gpu, pool_gpu, pool_before, rows=None):
+    out_ref, st_ref = run_oracle(w, rows)
+    sel = slice(None) if rows is None else torch.as_tensor(rows)
+    check_out(o_gpu[sel].float().cpu().numpy(), out_ref)
+    slots = w.slot_idx if rows is None else w.slot_idx[torch.as_tensor(rows)]
+    for i, s in enumerate(slots.tolist()):
+        if s < 0:
+            continue
+        ref = st_ref[s] if rows is None else st_ref[i]
+        check_state(pool_gpu[s].cpu().numpy(), ref, what=f"state slot {s}")
+    # every slot that no active row names is bit-identical
+    touched = torch.zeros(w.num_slots, dtype=torch.bool, device=pool_gpu.device)
+    act = w.slot_idx[w.slot_idx >= 0].long().to(pool_gpu.device)
+    touched[act] = True
+    assert torch.equal(pool_gpu[~touched], pool_before[~touched]), "an untouched slot changed"
+    if len(act):
+        changed = (pool_gpu[act] != pool_before[act]).flatten(1).any(dim=1)
+        assert bool(changed.all()), "an active slot was not written"
+
+
+SMALL_CONFIGS = ["n1_t1_hv8", "n32_t1_hv8", "n32_t1_hv16_gated", "n1_t4_hv8", "n8_t4_hv8", "n32_t4_hv8"]
+
+
+@pytest.mark.parametrize("name", SMALL_CONFIGS)
+def test_named_workload_parity(name, cuda_device):
+    w = workloads.config(name)
+    o, pool, before = run_gpu(w, cuda_device)
+    assert_parity(w, o, pool, before)
+
+
+def test_large_batch_parity_sampled(cuda_device):
+    """N=256, T=1, HV=32, 1024-slot pool (2 GiB): sampled rows against the oracle,
+    including the rows whose slots sit furthest into the pool, every other
+    slot checked bit-exact on the GPU."""
+    w = workloads.config("n256_t1_hv32")
+    o, pool, before = run_gpu(w, cuda_device)
+    order = torch.argsort(w.slot_idx, descending=True)
+    rows = sorted(set(order[:8].tolist()) | set(range(0, 256, 9)))
+    assert int(w.slot_idx[rows].max()) >= 1000
+    assert_parity(w, o, pool, before, rows=rows)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_pool_offsets_beyond_32_bits(gated, cuda_device):
+    """Slots whose element offsets exceed 2^31 (a 8.6 GB pool): the kernel's
+    64-bit slot arithmetic lands every row in its own slot.  Only the active
+    slots hold drawn states; the rest of the pool is zero and must stay zero."""
+    HV, K, V = 2, 128, 128
+    num_slots = 66_000  # 66000 * 2 * 128 * 128 = 2.16e9 elements > 2^31
+    w = workloads.make(N=4, T=2, HV=HV, K=K, V=V, num_slots=4, gated=gated, seed=21)
+    big_slots = torch.tensor([65_999, 32_768, 65_537, 7], dtype=torch.int32)
+    assert int(big_slots.max()) * HV * K * V > 2 ** 31
+    pool = torch.zeros(num_slots, HV, K, V, dtype=torch.float32, device=cuda_device)
+    pool[big_slots.long().to(cuda_device)] = w.state[w.slot_idx.long()].to(cuda_device)
+    d = w.to(cuda_device, state_too=False)
+    big_idx = big_slots.to(cuda_device)
+    if gated:
+        o = kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, pool, big_idx, d.gate, d.norm_weight,
+                                         eps=w.eps, scale=w.scale)
+    else:
+        o = kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, pool, big_idx, scale=w.scale)
+    torch.cuda.synchronize()
+    kw = dict(gate=w.gate, norm_weight=w.norm_weight, eps=w.eps) if gated else {}
+    out_ref, st_ref = oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx, w.scale, **kw)
+    check_out(o.float().cpu().numpy(), out_ref)
+    for n in range(w.N):
+        check_state(pool[int(big_slots[n])].cpu().numpy(), st_ref[int(w.slot_idx[n])])
+    mask = torch.ones(num_slots, dtype=torch.bool, device=cuda_device)
+    mask[big_slots.long().to(cuda_device)] = False
+    assert int(torch.count_nonzero(pool[mask])) == 0
+    del pool
+
+
+CASES = [
+    # N, T, HV, K, V, gated, inactive
+    (1, 1, 1, 128, 32, False, 0),
+    (3, 1, 3, 128, 96, False, 0),       # 3 tiles: ragged V
+    (5, 2, 2, 64, 160, False, 1),
+    (4, 3, 1, 256, 64, False, 0),
+    (2, 5, 2, 128, 128, False, 0),
+    (7, 1, 5, 128, 128, False, 2),      # padding rows
+    (2, 8, 1, 64, 32, False, 0),
+    (1, 1, 1, 128, 32, True, 0),        # cluster of 1
+    (3, 1, 3, 128, 96, True, 0),
+    (2, 3, 2, 64, 256, True, 1),        # cluster of 8 (largest)
+    (4, 2, 2, 256, 128, True, 0),
+    (6, 4, 2, 128, 224, True, 2),
+]
+
+
+@pytest.mark.parametrize("N,T,HV,K,V,gated,inactive", CASES)
+def test_shapes_parity(N, T, HV, K, V, gated, inactive, cuda_device):
+    w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=2 * N + 1, gated=gated,
+                       inactive=inactive, seed=N * 1000 + T * 100 + V)
+    o, pool, before = run_gpu(w, cuda_device)
+    assert_parity(w, o, pool, before)
+    if inactive:
+        assert torch.all(o[N - inactive:] == 0)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_t_steps_equal_successive_single_steps(gated, cuda_device):
+    w = workloads.make(N=6, T=4, HV=3, K=128, V=128, num_slots=9, gated=gated, seed=11)
+    d = w.to(cuda_device)
+    pool_a = d.state.clone()
+    pool_b = d.state.clone()
+    fn = kda.kda_decode_gated_rmsnorm if gated else kda.kda_decode
+    extra = (lambda sl: (d.gate[:, sl].contiguous(), d.norm_weight)) if gated else (lambda sl: ())
+    out_a = fn(d.q, d.k, d.v, d.g, d.beta, pool_a, d.slot_idx, *extra(slice(None)))
+    outs = []
+    for t in range(w.T):
+        sl = slice(t, t + 1)
+        outs.append(fn(d.q[:, sl].contiguous(), d.k[:, sl].contiguous(), d.v[:, sl].contiguous(),
+                       d.g[:, sl].contiguous(), d.beta[:, sl].contiguous(), pool_b, d.slot_idx,
+                       *extra(sl)))
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, torch.cat(outs, dim=1))
+    assert torch.equal(pool_a, pool_b)
+
+
+def test_empty_batch_is_noop(cuda_device):
+    w = workloads.make(N=2, T=1, HV=2, K=128, V=128, num_slots=3)
+    d = w.to(cuda_device)
+    before = d.state.clone()
+    kda.kda_decode(d.q[:0], d.k[:0], d.v[:0], d.g[:0], d.beta[:0], d.state, d.slot_idx[:0])
+    kda.kda_decode(d.q[:, :0], d.k[:, :0], d.v[:, :0], d.g[:, :0], d.beta[:, :0], d.state, d.slot_idx)
+    torch.cuda.synchronize()
+    assert torch.equal(d.state, before)
+
+
+def test_all_rows_inactive(cuda_device):
+    w = workloads.make(N=3, T=2, HV=2, K=128, V=64, num_slots=4, inactive=3, gated=True)
+    o, pool, before = run_gpu(w, cuda_device, out=torch.full((3, 2, 2, 64), 7.0, dtype=torch.bfloat16,
+                                                              device=cuda_device))
+    assert torch.all(o == 0)
+    assert torch.equal(pool, before)
+
+
+def test_side_stream_and_graph_replay(cuda_device):
+    """A call captured in a CUDA graph on a side stream replays to the eager result."""
+    w = workloads.config("n32_t1_hv8")
+    d = w.to(cuda_device)
+    pool_eager = d.state.clone()
+    pool_graph = d.state.clone()
+    out_eager = kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, pool_eager, d.slot_idx)
+    out_graph = torch.empty_like(out_eager)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, pool_graph, d.slot_idx, out=out_graph, stream=s)
+    torch.cuda.synchronize()
+    assert torch.equal(pool_graph, d.state), "capture must not execute the kernel"
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out_graph, out_eager)
+    assert torch.equal(pool_graph, pool_eager)
+    graph.replay()  # a second step advances the state again, like the eager path
+    kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, pool_eager, d.slot_idx)
+    torch.cuda.synchronize()
+    assert torch.equal(pool_graph, pool_eager)
+    del graph
+
+
+def test_rejections_with_real_buffers(cuda_device):
+    w = workloads.make(N=2, T=1, HV=2, K=128, V=128, num_slots=3)
+    d = w.to(cuda_device)
+    lib = kda.library()
+    s = torch.cuda.current_stream().cuda_stream
+    before = d.state.clone()
+
+    def call(q=None, out=None, state=None, K=128):
+        return lib.kda_decode(q or d.q.data_ptr(), d.k.data_ptr(), d.v.data_ptr(), d.g.data_ptr(),
+                              d.beta.data_ptr(), state or d.state.data_ptr(), d.slot_idx.data_ptr(),
+                              out or d.q.data_ptr() + 64, 2, 1, 2, K, 128, 0.1, s)
+
+    out = torch.empty(2, 1, 2, 128, dtype=torch.bfloat16, device=cuda_device)
+    assert call() == kda.KDA_ERR_ALIAS                             # out inside q
+    assert call(out=d.state.data_ptr()) == kda.KDA_ERR_ALIAS       # out = pool
+    assert call(out=out.data_ptr() + 2) == kda.KDA_ERR_MISALIGNED
+    assert call(out=out.data_ptr(), K=96) == kda.KDA_ERR_UNSUPPORTED
+    assert call(out=out.data_ptr(), q=d.q.data_ptr() + 8) == kda.KDA_ERR_MISALIGNED
+    torch.cuda.synchronize()
+    assert torch.equal(d.state, before)
+    assert call(out=out.data_ptr()) == kda.KDA_OK
+    with pytest.raises(kda.KdaError):
+        kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, out=d.v)
+    torch.cuda.synchronize()
