@@ -137,16 +137,23 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
 
   cudaError_t err = cudaErrorInvalidValue;
   const bool multi = T > 1;
-#define KDA_LAUNCH(KK, GG, MM) err = cudaLaunchKernelEx(&cfg, kda::kda_decode_kernel<KK, GG, MM>, p)
-#define KDA_LAUNCH_K(KK)                                   \
-  do {                                                     \
-    if (gated) {                                           \
-      if (multi) KDA_LAUNCH(KK, true, true);               \
-      else KDA_LAUNCH(KK, true, false);                    \
-    } else {                                               \
-      if (multi) KDA_LAUNCH(KK, false, true);              \
-      else KDA_LAUNCH(KK, false, false);                   \
-    }                                                      \
+  const bool v128 = V == 128;
+  // One instantiation per (K, V fixed at 128 or not, gated, T > 1).
+#define KDA_LAUNCH(KK, VV, GG, MM) err = cudaLaunchKernelEx(&cfg, kda::kda_decode_kernel<KK, VV, GG, MM>, p)
+#define KDA_LAUNCH_V(KK, GG, MM)               \
+  do {                                         \
+    if (v128) KDA_LAUNCH(KK, 128, GG, MM);     \
+    else KDA_LAUNCH(KK, 0, GG, MM);            \
+  } while (0)
+#define KDA_LAUNCH_K(KK)                              \
+  do {                                                \
+    if (gated) {                                      \
+      if (multi) KDA_LAUNCH_V(KK, true, true);        \
+      else KDA_LAUNCH_V(KK, true, false);             \
+    } else {                                          \
+      if (multi) KDA_LAUNCH_V(KK, false, true);       \
+      else KDA_LAUNCH_V(KK, false, false);            \
+    }                                                 \
   } while (0)
   switch (K) {
     case 64: KDA_LAUNCH_K(64); break;
@@ -155,6 +162,7 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
     default: return KDA_ERR_UNSUPPORTED;
   }
 #undef KDA_LAUNCH_K
+#undef KDA_LAUNCH_V
 #undef KDA_LAUNCH
   return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
