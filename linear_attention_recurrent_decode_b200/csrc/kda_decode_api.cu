@@ -124,15 +124,20 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
   cfg.blockDim = dim3(kda::kThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  // Programmatic stream serialization: the kernel waits for earlier work in
+  // the stream (griddepcontrol.wait) before its first global access, so the
+  // launch itself may overlap the tail of the previous kernel.
+  cudaLaunchAttribute attr[2];
   cfg.attrs = attr;
-  cfg.numAttrs = 0;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs = 1;
   if (gated) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(tiles);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(tiles);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
 
   cudaError_t err = cudaErrorInvalidValue;

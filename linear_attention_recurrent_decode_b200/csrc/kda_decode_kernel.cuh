@@ -30,6 +30,14 @@
 // memory (DSMEM) and a cluster barrier completes the RMS over V; the norm,
 // weight and sigmoid gate are applied before the bf16 store.
 //
+// Launch overlap: kernels are launched with programmatic stream
+// serialization.  Every global access of a CTA comes after griddepcontrol.wait
+// (all work earlier in the stream complete and visible), and a CTA lets the
+// next kernel in the stream start launching once it is about to write its
+// state back, so the next call's launch overlaps this call's stores.  The
+// state is written with streaming (evict-first) stores: it is not read again
+// before the next decode step.
+//
 // No tensor cores: the step is a chain of mat-vec products with O(1) flops
 // per state byte, far below any tensor-core ridge point; the roofline is HBM.
 //
@@ -154,6 +162,12 @@ __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+__device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- token staging (T > 1)
 // Shared-memory image of one token's inputs for one CTA (K key rows, the
 // CTA's 32 value columns).  Every member starts on a 16-byte boundary.
@@ -267,6 +281,7 @@ kda_decode_kernel(const Params p) {
   const int64_t col = static_cast<int64_t>(tile) * kBV + cq * 4;
   const bool writer = (warp == 0) && (rg == 0);  // 8 lanes store the tile's 32 outputs
 
+  wait_prior_grids();
   const int32_t slot = __ldg(p.slot_idx + n);
 
   // Token inputs do not depend on the slot: issue them before it lands.
@@ -450,8 +465,9 @@ kda_decode_kernel(const Params p) {
     if constexpr (!MULTI) break;  // T == 1
   }
 
+  allow_next_grid();
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) sp[i * (V / 4)] = make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y);
+  for (int i = 0; i < RPT; ++i) __stcs(sp + i * (V / 4), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
 }
 
 }  // namespace kda

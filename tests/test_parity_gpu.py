@@ -240,3 +240,30 @@ def test_rejections_with_real_buffers(cuda_device):
     with pytest.raises(kda.KdaError):
         kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, out=d.v)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_back_to_back_calls_see_prior_writes(gated, cuda_device):
+    """Calls are launched with programmatic stream serialization; each call must
+    still see everything earlier in the stream: the previous call's state write
+    and a torch kernel that rewrites the next call's inputs in place."""
+    w = workloads.make(N=8, T=1, HV=4, K=128, V=128, num_slots=16, gated=gated, seed=31)
+    d = w.to(cuda_device)
+    fn = kda.kda_decode_gated_rmsnorm if gated else kda.kda_decode
+    extra = (d.gate, d.norm_weight) if gated else ()
+    outs = []
+    for step in range(3):
+        outs.append(fn(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, *extra).clone())
+        d.v.mul_(-0.5)          # foreign kernels on the same stream between calls
+        d.g.add_(-0.25)
+    torch.cuda.synchronize()
+    state = w.state.double().numpy().copy()
+    v, g = w.v.clone(), w.g.clone()
+    kw = dict(gate=w.gate, norm_weight=w.norm_weight, eps=w.eps) if gated else {}
+    for step in range(3):
+        ref, state = oracle.kda_decode_ref(w.q, w.k, v, g, w.beta, state, w.slot_idx, w.scale, **kw)
+        check_out(outs[step].float().cpu().numpy(), ref, what=f"step {step}")
+        v = (v.float() * -0.5).to(torch.bfloat16)
+        g = g + -0.25
+    for s in w.slot_idx.tolist():
+        check_state(d.state[s].cpu().numpy(), state[s], what=f"slot {s}")
