@@ -43,7 +43,7 @@ METRIC = "KDA decode µs/call and achieved HBM GB/s (% of B200 peak) at N32/T1/H
 UNIT = "us/call"
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "linear_attention_recurrent_decode_b200", "csrc")
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "kda_decode_n32_t1_hv8.md")
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 # ------------------------------------------------------------------ helpers
@@ -79,24 +79,27 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(workload: str):
-    """dram bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source and this workload; else None."""
-    if not os.path.exists(PROFILE_SUMMARY):
+    """dram bytes (read + write) per launch from a committed ncu summary under
+    profiles/ taken on this workload with the current kernel source; else None."""
+    if not os.path.isdir(PROFILES):
         return None
-    fields = {}
-    with open(PROFILE_SUMMARY) as f:
-        for line in f:
-            if line.startswith("- ") and ":" in line:
-                key, val = line[2:].split(":", 1)
-                fields[key.strip()] = val.strip().strip("`")
-    if fields.get("kernel_source_hash") != kernel_source_hash():
-        return None
-    if fields.get("workload") != workload:
-        return None
-    try:
-        return int(fields["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    current = kernel_source_hash()
+    for name in sorted(os.listdir(PROFILES)):
+        if not name.endswith(".md"):
+            continue
+        fields = {}
+        with open(os.path.join(PROFILES, name)) as f:
+            for line in f:
+                if line.startswith("- ") and ":" in line:
+                    key, val = line[2:].split(":", 1)
+                    fields.setdefault(key.strip(), val.strip().strip("`"))
+        if fields.get("workload") != workload or fields.get("kernel_source_hash") != current:
+            continue
+        try:
+            return int(fields["dram_bytes_per_launch"])
+        except (KeyError, ValueError):
+            continue
+    return None
 
 
 def measured_peaks():
