@@ -138,6 +138,12 @@ CASES = [
     (2, 3, 2, 64, 256, True, 1),        # cluster of 8 (largest)
     (4, 2, 2, 256, 128, True, 0),
     (6, 4, 2, 128, 224, True, 2),
+    # more tokens than one shared-memory chunk: prefetch of the next chunk, ragged last chunk
+    (3, 9, 2, 128, 128, False, 0),
+    (2, 17, 3, 64, 96, False, 1),
+    (2, 20, 2, 256, 64, False, 0),
+    (3, 9, 2, 128, 128, True, 1),
+    (2, 17, 1, 64, 256, True, 0),
 ]
 
 
@@ -152,8 +158,9 @@ def test_shapes_parity(N, T, HV, K, V, gated, inactive, cuda_device):
 
 
 @pytest.mark.parametrize("gated", [False, True])
-def test_t_steps_equal_successive_single_steps(gated, cuda_device):
-    w = workloads.make(N=6, T=4, HV=3, K=128, V=128, num_slots=9, gated=gated, seed=11)
+@pytest.mark.parametrize("T", [4, 12])
+def test_t_steps_equal_successive_single_steps(gated, T, cuda_device):
+    w = workloads.make(N=6, T=T, HV=3, K=128, V=128, num_slots=9, gated=gated, seed=11)
     d = w.to(cuda_device)
     pool_a = d.state.clone()
     pool_b = d.state.clone()
