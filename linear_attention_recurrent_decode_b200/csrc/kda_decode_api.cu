@@ -143,22 +143,23 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
   cudaError_t err = cudaErrorInvalidValue;
   const bool multi = T > 1;
   const bool v128 = V == 128;
-  // One instantiation per (K, V fixed at 128 or not, gated, T > 1).
-#define KDA_LAUNCH(KK, VV, GG, MM) err = cudaLaunchKernelEx(&cfg, kda::kda_decode_kernel<KK, VV, GG, MM>, p)
-#define KDA_LAUNCH_V(KK, GG, MM)               \
-  do {                                         \
-    if (v128) KDA_LAUNCH(KK, 128, GG, MM);     \
-    else KDA_LAUNCH(KK, 0, GG, MM);            \
+  // One instantiation per (K, V fixed at 128 or not, gated); T == 1 and T > 1
+  // (chunked) kernels.
+#define KDA_LAUNCH(KERNEL, KK, VV, GG) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG>, p)
+#define KDA_LAUNCH_V(KK, GG)                                                 \
+  do {                                                                       \
+    if (multi) {                                                             \
+      if (v128) KDA_LAUNCH(kda_decode_chunked_kernel, KK, 128, GG);          \
+      else KDA_LAUNCH(kda_decode_chunked_kernel, KK, 0, GG);                 \
+    } else {                                                                 \
+      if (v128) KDA_LAUNCH(kda_decode_kernel, KK, 128, GG);                  \
+      else KDA_LAUNCH(kda_decode_kernel, KK, 0, GG);                         \
+    }                                                                        \
   } while (0)
-#define KDA_LAUNCH_K(KK)                              \
-  do {                                                \
-    if (gated) {                                      \
-      if (multi) KDA_LAUNCH_V(KK, true, true);        \
-      else KDA_LAUNCH_V(KK, true, false);             \
-    } else {                                          \
-      if (multi) KDA_LAUNCH_V(KK, false, true);       \
-      else KDA_LAUNCH_V(KK, false, false);            \
-    }                                                 \
+#define KDA_LAUNCH_K(KK)                   \
+  do {                                     \
+    if (gated) KDA_LAUNCH_V(KK, true);     \
+    else KDA_LAUNCH_V(KK, false);          \
   } while (0)
   switch (K) {
     case 64: KDA_LAUNCH_K(64); break;

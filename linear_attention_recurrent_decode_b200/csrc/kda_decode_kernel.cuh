@@ -21,9 +21,20 @@
 // CTA computes at the same moment after its loads land: instruction count is
 // on the critical path, and the packed forms halve it.
 //
-// Multi-token calls (T > 1) stage the next chunk of tokens' q, k, g, v, gate
-// and beta in shared memory with cp.async, so the state tile is the only
-// per-thread register payload.
+// Multi-token calls (T > 1) use a second kernel that takes the tokens in
+// chunks of up to four.  Within a chunk every token's reductions run against
+// the chunk-start state, with the cumulative decays folded into per-row
+// coefficients, and the tokens are coupled through small per-head scalars:
+// with d_t = exp(g_t), A_t = d_0 ... d_t and B(s->t) = d_{s+1} ... d_t,
+//   R_t = S0^T (A_t k_t),   Q_t = S0^T (A_t q_t),
+//   M[t][s] = sum_i k_s,i B(s->t)_i k_t,i  (s < t),
+//   P[t][s] = sum_i k_s,i B(s->t)_i q_t,i  (s <= t),
+//   u_t = beta_t (v_t - R_t - sum_{s<t} M[t][s] u_s),
+//   o_t = scale (Q_t + sum_{s<=t} P[t][s] u_s),
+//   S_end = A_last S0 + sum_t (B(t->last) k_t) u_t^T,
+// which is the token-by-token recurrence regrouped (equal in exact
+// arithmetic): one cross-thread exchange per chunk instead of one per token,
+// and each state element is read and written once per chunk.
 //
 // The gated variant launches the V/32 tiles of one (n, h) as a thread-block
 // cluster: each CTA pushes its partial sum of o^2 into every peer's shared
@@ -62,7 +73,7 @@ constexpr int kBV = 32;                     // value columns per CTA
 constexpr int kColQuads = kBV / 4;          // float4 column groups per row segment (8)
 constexpr int kRowGroups = 32 / kColQuads;  // row groups per warp (4)
 constexpr int kMaxClusterTiles = 8;         // portable cluster size bound
-constexpr int kTokenChunk = 8;              // tokens staged in shared memory at a time (T > 1)
+constexpr int kChunk = 4;                   // tokens per chunk in the multi-token kernel
 
 struct Params {
   const __nv_bfloat16* q;
@@ -168,7 +179,7 @@ __device__ __forceinline__ void allow_next_grid() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---------------------------------------------------------------- token staging (T > 1)
+// ---------------------------------------------------------------- token staging (T > 1 kernel)
 // Shared-memory image of one token's inputs for one CTA (K key rows, the
 // CTA's 32 value columns).  Every member starts on a 16-byte boundary.
 template <int K>
@@ -210,33 +221,7 @@ __device__ __forceinline__ void stage_tokens(TokenSmem<K>* buf, const Params& p,
   }
 }
 
-template <int RPT, int K>
-__device__ __forceinline__ void read_token(TokenIn<RPT>& in, const TokenSmem<K>& s, int r0, int cq) {
-  if constexpr (RPT % 8 == 0) {
-#pragma unroll
-    for (int i = 0; i < RPT / 8; ++i) {
-      const uint4 a = *reinterpret_cast<const uint4*>(s.q + r0 + 8 * i);
-      const uint4 b = *reinterpret_cast<const uint4*>(s.k + r0 + 8 * i);
-      in.q[4 * i] = a.x; in.q[4 * i + 1] = a.y; in.q[4 * i + 2] = a.z; in.q[4 * i + 3] = a.w;
-      in.k[4 * i] = b.x; in.k[4 * i + 1] = b.y; in.k[4 * i + 2] = b.z; in.k[4 * i + 3] = b.w;
-    }
-  } else {
-    const uint2 a = *reinterpret_cast<const uint2*>(s.q + r0);
-    const uint2 b = *reinterpret_cast<const uint2*>(s.k + r0);
-    in.q[0] = a.x; in.q[1] = a.y; in.k[0] = b.x; in.k[1] = b.y;
-  }
-#pragma unroll
-  for (int i = 0; i < RPT / 4; ++i) {
-    const float4 x = *reinterpret_cast<const float4*>(s.g + r0 + 4 * i);
-    in.g[4 * i] = x.x; in.g[4 * i + 1] = x.y; in.g[4 * i + 2] = x.z; in.g[4 * i + 3] = x.w;
-  }
-  const uint2 vv = *reinterpret_cast<const uint2*>(s.v + 4 * cq);
-  const uint2 zz = *reinterpret_cast<const uint2*>(s.z + 4 * cq);
-  in.v[0] = vv.x; in.v[1] = vv.y; in.z[0] = zz.x; in.z[1] = zz.y;
-  in.beta = s.beta[0];
-}
-
-// ---------------------------------------------------------------- kernel
+// ---------------------------------------------------------------- T == 1 kernel
 // Thread layout inside the CTA (K x 32 tile, 128 threads):
 //   warp w owns key rows [w*K/4, (w+1)*K/4); inside a warp, lane = rg*8 + cq
 //   with row group rg in [0,4) and column quad cq in [0,8); the thread holds
@@ -244,8 +229,7 @@ __device__ __forceinline__ void read_token(TokenIn<RPT>& in, const TokenSmem<K>&
 //   4cq .. 4cq+3 of the tile.  One warp-wide float4 load covers 4 rows x 128 B.
 //
 // VS: the value width when fixed at compile time (row strides become
-// immediates), 0 for a run-time V.  MULTI: T > 1 (tokens staged in shared
-// memory); MULTI = false is the T == 1 path with all inputs in registers.
+// immediates), 0 for a run-time V.
 //
 // Resident CTAs per SM the register budget is capped for: at K = 128 seven
 // CTAs (<= 72 registers a thread) hold 1036 tiles on 148 SMs, a single wave
@@ -255,16 +239,96 @@ struct MinBlocks {
   static constexpr int value = K >= 256 ? 3 : (K >= 128 ? 7 : 8);
 };
 
-template <int K, int VS, bool GATED, bool MULTI>
+// Reduce-scatter of the two column-pair partials (S'^T k, S'^T q) across the
+// 4 row groups of a warp, then across the 4 warps through shared memory.
+// Returns the full sums for this thread's 4 columns.
+struct Reduced {
+  float2 rk[2], rq[2];
+  float qk;
+};
+__device__ __forceinline__ Reduced reduce_tile(const float2 (&pk)[2], const float2 (&pq)[2], float qk,
+                                               float2 (*red)[2][kColQuads * 2], float* red_qk, int warp,
+                                               int lane, int cq) {
+  // after the xor-16 step lanes with bit 4 clear hold S'^T k sums, set hold
+  // S'^T q; after the xor-8 step each lane holds one column pair of its set
+  const bool hi16 = (lane & 16) != 0;
+  const bool hi8 = (lane & 8) != 0;
+  float2 keep[2], send[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    keep[j] = hi16 ? pq[j] : pk[j];
+    send[j] = hi16 ? pk[j] : pq[j];
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float2 r = make_float2(__shfl_xor_sync(0xffffffffu, send[j].x, 16),
+                                 __shfl_xor_sync(0xffffffffu, send[j].y, 16));
+    keep[j] = __fadd2_rn(keep[j], r);
+  }
+  float2 mine = hi8 ? keep[1] : keep[0];
+  const float2 other = hi8 ? keep[0] : keep[1];
+  mine = __fadd2_rn(mine, make_float2(__shfl_xor_sync(0xffffffffu, other.x, 8),
+                                      __shfl_xor_sync(0xffffffffu, other.y, 8)));
+  qk += __shfl_xor_sync(0xffffffffu, qk, 8);
+  qk += __shfl_xor_sync(0xffffffffu, qk, 16);
+  red[warp][hi16 ? 1 : 0][cq * 2 + (hi8 ? 1 : 0)] = mine;
+  if (lane == 0) red_qk[warp] = qk;
+  __syncthreads();
+
+  // across the 4 warps (fixed order: identical sums in every thread)
+  Reduced r;
+  r.rk[0] = r.rk[1] = r.rq[0] = r.rq[1] = f2(0.f);
+  r.qk = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float4 a = *reinterpret_cast<const float4*>(&red[w][0][cq * 2]);
+    const float4 b = *reinterpret_cast<const float4*>(&red[w][1][cq * 2]);
+    r.rk[0] = __fadd2_rn(r.rk[0], make_float2(a.x, a.y));
+    r.rk[1] = __fadd2_rn(r.rk[1], make_float2(a.z, a.w));
+    r.rq[0] = __fadd2_rn(r.rq[0], make_float2(b.x, b.y));
+    r.rq[1] = __fadd2_rn(r.rq[1], make_float2(b.z, b.w));
+    r.qk += red_qk[w];
+  }
+  return r;
+}
+
+// Gated RMS norm of one output row across the V tiles of a cluster: lanes
+// 0..7 of warp 0 (the writers) hold the tile's 32 outputs in o; nrm is this
+// CTA's [kMaxClusterTiles] receive buffer for the per-tile sums of o^2.
+// Every thread of every CTA in the cluster must call it (cluster barrier).
+__device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], const float2 (&wgt)[2],
+                                           const uint32_t (&z)[2], float* nrm, int tile, int tiles,
+                                           int64_t V, float eps, bool writer, int lane) {
+  float ss = 0.f;
+  if (writer) {
+    ss = o[0].x * o[0].x + o[0].y * o[0].y + o[1].x * o[1].x + o[1].y * o[1].y;
+#pragma unroll
+    for (int m = 1; m < kColQuads; m <<= 1) ss += __shfl_xor_sync(0x000000ffu, ss, m);
+    if (lane < tiles) cluster_store_f32(cluster_map(smem_u32(&nrm[tile]), static_cast<uint32_t>(lane)), ss);
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (writer) {
+    float tot = 0.f;
+    for (int r = 0; r < tiles; ++r) tot += nrm[r];
+    const float inv = rsqrtf(tot / static_cast<float>(V) + eps);
+    const float zz[4] = {bf16lo(z[0]), bf16hi(z[0]), bf16lo(z[1]), bf16hi(z[1])};
+    const float ov[4] = {o[0].x, o[0].y, o[1].x, o[1].y};
+    const float wv[4] = {wgt[0].x, wgt[0].y, wgt[1].x, wgt[1].y};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) y[j] = ov[j] * inv * wv[j] * (1.0f / (1.0f + __expf(-zz[j])));
+  }
+}
+
+template <int K, int VS, bool GATED>
 __global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
 kda_decode_kernel(const Params p) {
   constexpr int RPT = K / (kWarps * kRowGroups);
   static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
 
-  __shared__ __align__(16) float2 red[2][kWarps][2][kColQuads * 2];  // [buf][warp][k|q][column pairs]
-  __shared__ float red_qk[2][kWarps];
-  __shared__ float nrm[2][kMaxClusterTiles];  // gated: per-tile sum of o^2
-  __shared__ TokenSmem<K> tok[MULTI ? 2 : 1][MULTI ? kTokenChunk : 1];
+  __shared__ __align__(16) float2 red[kWarps][2][kColQuads * 2];  // [warp][k|q][column pairs]
+  __shared__ float red_qk[kWarps];
+  __shared__ float nrm[kMaxClusterTiles];  // gated: per-tile sum of o^2
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,36 +344,26 @@ kda_decode_kernel(const Params p) {
   const int64_t h = unit - n * p.HV;
   const int64_t col = static_cast<int64_t>(tile) * kBV + cq * 4;
   const bool writer = (warp == 0) && (rg == 0);  // 8 lanes store the tile's 32 outputs
+  const int64_t row = n * p.HV + h;              // (n, t = 0, h)
 
   wait_prior_grids();
   const int32_t slot = __ldg(p.slot_idx + n);
 
   // Token inputs do not depend on the slot: issue them before it lands.
   TokenIn<RPT> cur;
-  if constexpr (MULTI) {
-    stage_tokens<K, GATED>(tok[0], p, V, n, h, static_cast<int64_t>(tile) * kBV, 0,
-                           static_cast<int>(p.T < kTokenChunk ? p.T : kTokenChunk));
-    cp_async_commit();
-  } else {
-    const int64_t row = n * p.HV + h;  // T == 1
-    ld_bf16_rows<RPT>(cur.q, p.q + row * K + r0);
-    ld_bf16_rows<RPT>(cur.k, p.k + row * K + r0);
-    ld_f32_rows<RPT>(cur.g, p.g + row * K + r0);
-    const uint2 vv = __ldg(reinterpret_cast<const uint2*>(p.v + row * V + col));
-    cur.v[0] = vv.x; cur.v[1] = vv.y;
-    if constexpr (GATED) {
-      const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + row * V + col));
-      cur.z[0] = zz.x; cur.z[1] = zz.y;
-    }
-    cur.beta = __ldg(p.beta + row);
+  ld_bf16_rows<RPT>(cur.q, p.q + row * K + r0);
+  ld_bf16_rows<RPT>(cur.k, p.k + row * K + r0);
+  ld_f32_rows<RPT>(cur.g, p.g + row * K + r0);
+  const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + row * V + col));
+  cur.v[0] = vv_raw.x; cur.v[1] = vv_raw.y;
+  if constexpr (GATED) {
+    const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + row * V + col));
+    cur.z[0] = zz.x; cur.z[1] = zz.y;
   }
+  cur.beta = __ldg(p.beta + row);
 
   if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
-    if constexpr (MULTI) cp_async_wait<0>();
-    if (writer) {
-      for (int64_t t = 0; t < p.T; ++t)
-        *reinterpret_cast<uint2*>(p.out + ((n * p.T + t) * p.HV + h) * V + col) = make_uint2(0u, 0u);
-    }
+    if (writer) *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(0u, 0u);
     return;  // uniform over the cluster: every tile of this (n, h) sees the same slot
   }
 
@@ -332,137 +386,350 @@ kda_decode_kernel(const Params p) {
     wgt[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
   }
 
+  // decay and the partial reductions over this thread's rows
+  float2 pk[2] = {f2(0.f), f2(0.f)}, pq[2] = {f2(0.f), f2(0.f)};
+  float qk = 0.f;
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float qi = bf16_at(cur.q, i);
+    const float ki = bf16_at(cur.k, i);
+    const float2 d = f2(__expf(cur.g[i]));
+    const float2 k2 = f2(ki), q2 = f2(qi);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      s[i][j] = __fmul2_rn(s[i][j], d);
+      pk[j] = __ffma2_rn(s[i][j], k2, pk[j]);
+      pq[j] = __ffma2_rn(s[i][j], q2, pq[j]);
+    }
+    qk = fmaf(qi, ki, qk);
+  }
+  const Reduced r = reduce_tile(pk, pq, qk, red, red_qk, warp, lane, cq);
+
+  // correction, rank-1 write, readout
+  const float2 beta2 = f2(cur.beta);
+  const float2 qk2 = f2(r.qk);
   const float2 scale2 = f2(p.scale);
-  for (int64_t t = 0; t < p.T; ++t) {
-    const int buf = static_cast<int>(t & 1);
-    if constexpr (MULTI) {
-      const int j = static_cast<int>(t % kTokenChunk);
-      const int cb = static_cast<int>((t / kTokenChunk) & 1);
-      if (j == 0) {
-        const int64_t next0 = t + kTokenChunk;
-        if (next0 < p.T) {  // prefetch the next chunk into the other buffer
-          const int64_t left = p.T - next0;
-          stage_tokens<K, GATED>(tok[cb ^ 1], p, V, n, h, static_cast<int64_t>(tile) * kBV, next0,
-                                 static_cast<int>(left < kTokenChunk ? left : kTokenChunk));
-          cp_async_commit();
-          cp_async_wait<1>();
-        } else {
-          cp_async_wait<0>();
-        }
-        __syncthreads();
-      }
-      read_token<RPT, K>(cur, tok[cb][j], r0, cq);
-    }
-
-    // decay and the partial reductions over this thread's rows
-    float2 pk[2] = {f2(0.f), f2(0.f)}, pq[2] = {f2(0.f), f2(0.f)};
-    float qk = 0.f;
+  float2 u[2], o[2];
+  const float2 vv[2] = {make_float2(bf16lo(cur.v[0]), bf16hi(cur.v[0])),
+                        make_float2(bf16lo(cur.v[1]), bf16hi(cur.v[1]))};
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-      const float qi = bf16_at(cur.q, i);
-      const float ki = bf16_at(cur.k, i);
-      const float2 d = f2(__expf(cur.g[i]));
-      const float2 k2 = f2(ki), q2 = f2(qi);
+  for (int j = 0; j < 2; ++j) {
+    u[j] = __fmul2_rn(beta2, __fadd2_rn(vv[j], make_float2(-r.rk[j].x, -r.rk[j].y)));
+    o[j] = __fmul2_rn(scale2, __ffma2_rn(qk2, u[j], r.rq[j]));
+  }
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        s[i][j] = __fmul2_rn(s[i][j], d);
-        pk[j] = __ffma2_rn(s[i][j], k2, pk[j]);
-        pq[j] = __ffma2_rn(s[i][j], q2, pq[j]);
-      }
-      qk = fmaf(qi, ki, qk);
-    }
+  for (int i = 0; i < RPT; ++i) {
+    const float2 k2 = f2(bf16_at(cur.k, i));
+#pragma unroll
+    for (int j = 0; j < 2; ++j) s[i][j] = __ffma2_rn(k2, u[j], s[i][j]);
+  }
 
-    // Reduce-scatter across the 4 row groups of the warp: after the xor-16
-    // step lanes with bit 4 clear hold S'^T k sums, set hold S'^T q; after the
-    // xor-8 step each lane holds one column pair of its set.
-    const bool hi16 = (lane & 16) != 0;
-    const bool hi8 = (lane & 8) != 0;
-    float2 keep[2], send[2];
+  if constexpr (GATED) {
+    cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
+    float y[4];
+    gated_norm(y, o, wgt, cur.z, nrm, tile, tiles, V, p.eps, writer, lane);
+    if (writer)
+      *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+  } else if (writer) {
+    *reinterpret_cast<uint2*>(p.out + row * V + col) =
+        make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
+  }
+
+  allow_next_grid();
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) __stcs(sp + i * (V / 4), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
+}
+
+// ---------------------------------------------------------------- T > 1 kernel
+// Index of M[t][s] (s < t) and of P[t][s] (s <= t) in the per-chunk scalars.
+constexpr int kNumM = kChunk * (kChunk - 1) / 2;
+constexpr int kNumMP = kNumM + kChunk * (kChunk + 1) / 2;
+__host__ __device__ constexpr int m_index(int t, int s) { return t * (t - 1) / 2 + s; }
+__host__ __device__ constexpr int p_index(int t, int s) { return kNumM + t * (t + 1) / 2 + s; }
+
+// Per-row coefficients of one chunk (see the top of this file).
+template <int K>
+struct alignas(16) ChunkCoef {
+  float4 kt[K];  // A_t k_t            for t = 0..3 (zero past the chunk's last token)
+  float4 qt[K];  // A_t q_t
+  float4 c[K];   // B(t->last) k_t
+  float a[K];    // A_last
+};
+
+// Per-row chunk coefficients (one thread per key row) and each warp's partial
+// sums of the M/P scalars.
+template <int K>
+__device__ __forceinline__ void chunk_prep(ChunkCoef<K>& cf, float (*mp_part)[kNumMP],
+                                           const TokenSmem<K>* raw, int tc, int warp, int lane) {
+  float mp[kNumMP];
+#pragma unroll
+  for (int i = 0; i < kNumMP; ++i) mp[i] = 0.f;
+  for (int r = threadIdx.x; r < K; r += kThreads) {
+    float d[kChunk], kk[kChunk], qq[kChunk];
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) {
+      const bool live = t < tc;
+      d[t] = live ? __expf(raw[t].g[r]) : 1.f;
+      kk[t] = live ? __bfloat162float(raw[t].k[r]) : 0.f;
+      qq[t] = live ? __bfloat162float(raw[t].q[r]) : 0.f;
+    }
+    float A[kChunk];
+    A[0] = d[0];
+#pragma unroll
+    for (int t = 1; t < kChunk; ++t) A[t] = A[t - 1] * d[t];
+    float E[kChunk];  // B(t->last) = d_{t+1} ... d_{tc-1}
+    E[kChunk - 1] = 1.f;
+#pragma unroll
+    for (int t = kChunk - 2; t >= 0; --t) E[t] = (t + 1 < tc) ? E[t + 1] * d[t + 1] : 1.f;
+    cf.kt[r] = make_float4(A[0] * kk[0], A[1] * kk[1], A[2] * kk[2], A[3] * kk[3]);
+    cf.qt[r] = make_float4(A[0] * qq[0], A[1] * qq[1], A[2] * qq[2], A[3] * qq[3]);
+    cf.c[r] = make_float4(E[0] * kk[0], E[1] * kk[1], E[2] * kk[2], E[3] * kk[3]);
+    cf.a[r] = tc == 1 ? A[0] : (tc == 2 ? A[1] : (tc == 3 ? A[2] : A[3]));
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) {
+      float B = 1.f;  // B(s->t), s walking down from t
+#pragma unroll
+      for (int s = t; s >= 0; --s) {
+        const float ks = kk[s] * B;
+        if (s < t) mp[m_index(t, s)] = fmaf(ks, kk[t], mp[m_index(t, s)]);
+        mp[p_index(t, s)] = fmaf(ks, qq[t], mp[p_index(t, s)]);
+        B *= d[s];
+      }
+    }
+  }
+  // reduce-scatter the 16 scalars across the warp: lane L ends with scalar (L >> 1) & 15
+#pragma unroll
+  for (int m = 16, half = kNumMP / 2; m >= 2; m >>= 1, half >>= 1) {
+    const bool hi = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = hi ? mp[i + half] : mp[i];
+      const float send = hi ? mp[i] : mp[i + half];
+      mp[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  mp[0] += __shfl_xor_sync(0xffffffffu, mp[0], 1);
+  if ((lane & 1) == 0) mp_part[warp][(lane >> 1) & 15] = mp[0];
+}
+
+// Partial sums of S0^T w_t over this thread's rows for the 4 chunk tokens
+// (w = kt or qt), reduce-scattered across the warp's 4 row groups: lane
+// (rg, cq) stores token rg's partial for its 4 columns into red[warp][rg][cq].
+template <int RPT, int K>
+__device__ __forceinline__ void chunk_pass(const float2 (&s)[RPT][2], const float4* w, float4 (*red)[kChunk][kColQuads],
+                                           int r0, int warp, int lane, int rg, int cq) {
+  float2 acc[kChunk][2];
+#pragma unroll
+  for (int t = 0; t < kChunk; ++t) acc[t][0] = acc[t][1] = f2(0.f);
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float4 c = w[r0 + i];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      keep[j] = hi16 ? pq[j] : pk[j];
-      send[j] = hi16 ? pk[j] : pq[j];
+      acc[0][j] = __ffma2_rn(s[i][j], f2(c.x), acc[0][j]);
+      acc[1][j] = __ffma2_rn(s[i][j], f2(c.y), acc[1][j]);
+      acc[2][j] = __ffma2_rn(s[i][j], f2(c.z), acc[2][j]);
+      acc[3][j] = __ffma2_rn(s[i][j], f2(c.w), acc[3][j]);
     }
+  }
+  // xor-16: lanes with bit 4 clear keep tokens {0,1}, set keep {2,3};
+  // xor-8: lanes with bit 3 clear keep the first of their two tokens.
+  const bool hi16 = (lane & 16) != 0;
+  const bool hi8 = (lane & 8) != 0;
+  float2 keep[2][2];
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const float2 r = make_float2(__shfl_xor_sync(0xffffffffu, send[j].x, 16),
-                                   __shfl_xor_sync(0xffffffffu, send[j].y, 16));
-      keep[j] = __fadd2_rn(keep[j], r);
+      const float2 k0 = hi16 ? acc[2 + tt][j] : acc[tt][j];
+      const float2 sd = hi16 ? acc[tt][j] : acc[2 + tt][j];
+      keep[tt][j] = __fadd2_rn(k0, make_float2(__shfl_xor_sync(0xffffffffu, sd.x, 16),
+                                               __shfl_xor_sync(0xffffffffu, sd.y, 16)));
     }
-    float2 mine = hi8 ? keep[1] : keep[0];
-    const float2 other = hi8 ? keep[0] : keep[1];
-    mine = __fadd2_rn(mine, make_float2(__shfl_xor_sync(0xffffffffu, other.x, 8),
-                                        __shfl_xor_sync(0xffffffffu, other.y, 8)));
-    qk += __shfl_xor_sync(0xffffffffu, qk, 8);
-    qk += __shfl_xor_sync(0xffffffffu, qk, 16);
-    red[buf][warp][hi16 ? 1 : 0][cq * 2 + (hi8 ? 1 : 0)] = mine;
-    if (lane == 0) red_qk[buf][warp] = qk;
+  }
+  float2 mine[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float2 k0 = hi8 ? keep[1][j] : keep[0][j];
+    const float2 sd = hi8 ? keep[0][j] : keep[1][j];
+    mine[j] = __fadd2_rn(k0, make_float2(__shfl_xor_sync(0xffffffffu, sd.x, 8),
+                                         __shfl_xor_sync(0xffffffffu, sd.y, 8)));
+  }
+  red[warp][rg][cq] = make_float4(mine[0].x, mine[0].y, mine[1].x, mine[1].y);
+}
+
+template <int K, int VS, bool GATED>
+__global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
+kda_decode_chunked_kernel(const Params p) {
+  constexpr int RPT = K / (kWarps * kRowGroups);
+  static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
+  static_assert(kChunk == 4 && kRowGroups == kChunk, "one row group per chunk token in the reduce-scatter");
+
+  __shared__ TokenSmem<K> tok[2][kChunk];  // raw token inputs, double-buffered by chunk
+  __shared__ ChunkCoef<K> cf;
+  __shared__ __align__(16) float4 redR[kWarps][kChunk][kColQuads];
+  __shared__ __align__(16) float4 redQ[kWarps][kChunk][kColQuads];
+  __shared__ float mp_part[kWarps][kNumMP];
+  __shared__ float mp_tot[kNumMP];
+  __shared__ float nrm[2][kChunk][kMaxClusterTiles];  // gated: per-tile sums of o^2, by chunk parity
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cq = lane & (kColQuads - 1);
+  const int rg = lane / kColQuads;
+  const int r0 = warp * (K / kWarps) + rg * RPT;
+  const int64_t V = VS ? VS : p.V;
+  const int tiles = VS ? VS / kBV : p.tiles;
+
+  const int64_t unit = blockIdx.x / tiles;  // n * HV + h
+  const int tile = static_cast<int>(blockIdx.x - unit * tiles);
+  const int64_t n = unit / p.HV;
+  const int64_t h = unit - n * p.HV;
+  const int64_t col0 = static_cast<int64_t>(tile) * kBV;
+  const int64_t col = col0 + cq * 4;
+  const bool writer = (warp == 0) && (rg == 0);
+
+  wait_prior_grids();
+  const int32_t slot = __ldg(p.slot_idx + n);
+
+  // Token inputs do not depend on the slot: stage the first chunk before it lands.
+  stage_tokens<K, GATED>(tok[0], p, V, n, h, col0, 0, static_cast<int>(p.T < kChunk ? p.T : kChunk));
+  cp_async_commit();
+
+  if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
+    cp_async_wait<0>();
+    if (writer) {
+      for (int64_t t = 0; t < p.T; ++t)
+        *reinterpret_cast<uint2*>(p.out + ((n * p.T + t) * p.HV + h) * V + col) = make_uint2(0u, 0u);
+    }
+    return;
+  }
+
+  float4* const sp =
+      reinterpret_cast<float4*>(p.state + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col);
+  float2 s[RPT][2];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float4 x = sp[i * (V / 4)];
+    s[i][0] = make_float2(x.x, x.y);
+    s[i][1] = make_float2(x.z, x.w);
+  }
+
+  if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
+
+  float2 wgt[2] = {f2(0.f), f2(0.f)};
+  if constexpr (GATED) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(p.norm_weight + col));
+    wgt[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+    wgt[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+  }
+  const float2 scale2 = f2(p.scale);
+
+  for (int64_t c0 = 0; c0 < p.T; c0 += kChunk) {
+    const int64_t left = p.T - c0;
+    const int tc = static_cast<int>(left < kChunk ? left : kChunk);
+    const int cb = static_cast<int>((c0 / kChunk) & 1);
+    __syncthreads();  // every thread is done with the previous chunk's coefficients
+    if (c0 + kChunk < p.T) {  // prefetch the next chunk into the other buffer
+      const int64_t nl = p.T - c0 - kChunk;
+      stage_tokens<K, GATED>(tok[cb ^ 1], p, V, n, h, col0, c0 + kChunk,
+                             static_cast<int>(nl < kChunk ? nl : kChunk));
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    chunk_prep<K>(cf, mp_part, tok[cb], tc, warp, lane);
     __syncthreads();
 
-    // across the 4 warps (fixed order: identical sums in every thread)
-    float2 rk[2] = {f2(0.f), f2(0.f)}, rq[2] = {f2(0.f), f2(0.f)};
-    float qkt = 0.f;
+    chunk_pass<RPT, K>(s, cf.kt, redR, r0, warp, lane, rg, cq);
+    chunk_pass<RPT, K>(s, cf.qt, redQ, r0, warp, lane, rg, cq);
+    if (threadIdx.x < kNumMP) {
+      float tot = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float4 a = *reinterpret_cast<const float4*>(&red[buf][w][0][cq * 2]);
-      const float4 b = *reinterpret_cast<const float4*>(&red[buf][w][1][cq * 2]);
-      rk[0] = __fadd2_rn(rk[0], make_float2(a.x, a.y));
-      rk[1] = __fadd2_rn(rk[1], make_float2(a.z, a.w));
-      rq[0] = __fadd2_rn(rq[0], make_float2(b.x, b.y));
-      rq[1] = __fadd2_rn(rq[1], make_float2(b.z, b.w));
-      qkt += red_qk[buf][w];
+      for (int w = 0; w < kWarps; ++w) tot += mp_part[w][threadIdx.x];
+      mp_tot[threadIdx.x] = tot;
+    }
+    __syncthreads();
+
+    // per token: correction (all threads), readout and output (writers)
+    float2 u[kChunk][2];
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) {
+      u[t][0] = u[t][1] = f2(0.f);
+      if (t < tc) {
+        const TokenSmem<K>& raw = tok[cb][t];
+        const uint2 vr = *reinterpret_cast<const uint2*>(raw.v + 4 * cq);
+        float2 x[2] = {make_float2(bf16lo(vr.x), bf16hi(vr.x)), make_float2(bf16lo(vr.y), bf16hi(vr.y))};
+        float4 R = redR[0][t][cq];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+          const float4 a = redR[w][t][cq];
+          R = make_float4(R.x + a.x, R.y + a.y, R.z + a.z, R.w + a.w);
+        }
+        x[0] = __fadd2_rn(x[0], make_float2(-R.x, -R.y));
+        x[1] = __fadd2_rn(x[1], make_float2(-R.z, -R.w));
+#pragma unroll
+        for (int sj = 0; sj < t; ++sj) {
+          const float2 m2 = f2(-mp_tot[m_index(t, sj)]);
+          x[0] = __ffma2_rn(m2, u[sj][0], x[0]);
+          x[1] = __ffma2_rn(m2, u[sj][1], x[1]);
+        }
+        const float2 b2 = f2(raw.beta[0]);
+        u[t][0] = __fmul2_rn(b2, x[0]);
+        u[t][1] = __fmul2_rn(b2, x[1]);
+
+        float2 o[2] = {f2(0.f), f2(0.f)};
+        if (writer) {
+          float4 Q = redQ[0][t][cq];
+#pragma unroll
+          for (int w = 1; w < kWarps; ++w) {
+            const float4 a = redQ[w][t][cq];
+            Q = make_float4(Q.x + a.x, Q.y + a.y, Q.z + a.z, Q.w + a.w);
+          }
+          o[0] = make_float2(Q.x, Q.y);
+          o[1] = make_float2(Q.z, Q.w);
+#pragma unroll
+          for (int sj = 0; sj <= t; ++sj) {
+            const float2 p2 = f2(mp_tot[p_index(t, sj)]);
+            o[0] = __ffma2_rn(p2, u[sj][0], o[0]);
+            o[1] = __ffma2_rn(p2, u[sj][1], o[1]);
+          }
+          o[0] = __fmul2_rn(scale2, o[0]);
+          o[1] = __fmul2_rn(scale2, o[1]);
+        }
+        const int64_t out_row = ((n * p.T + c0 + t) * p.HV + h) * V + col;
+        if constexpr (GATED) {
+          if (c0 == 0 && t == 0) cluster_wait_acquire();  // pairs with the relaxed arrive above
+          uint32_t z[2];
+          const uint2 zr = *reinterpret_cast<const uint2*>(raw.z + 4 * cq);
+          z[0] = zr.x; z[1] = zr.y;
+          float y[4];
+          gated_norm(y, o, wgt, z, nrm[cb][t], tile, tiles, V, p.eps, writer, lane);
+          if (writer)
+            *reinterpret_cast<uint2*>(p.out + out_row) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+        } else if (writer) {
+          *reinterpret_cast<uint2*>(p.out + out_row) =
+              make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
+        }
+      }
     }
 
-    // correction, rank-1 write, readout
-    const float2 beta2 = f2(cur.beta);
-    const float2 qk2 = f2(qkt);
-    float2 u[2], o[2];
-    const float2 vv[2] = {make_float2(bf16lo(cur.v[0]), bf16hi(cur.v[0])),
-                          make_float2(bf16lo(cur.v[1]), bf16hi(cur.v[1]))};
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      u[j] = __fmul2_rn(beta2, __fadd2_rn(vv[j], make_float2(-rk[j].x, -rk[j].y)));
-      o[j] = __fmul2_rn(scale2, __ffma2_rn(qk2, u[j], rq[j]));
-    }
+    // chunk-end state: S = A_last S0 + sum_t c_t u_t^T
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-      const float2 k2 = f2(bf16_at(cur.k, i));
+      const float4 c = cf.c[r0 + i];
+      const float2 a2 = f2(cf.a[r0 + i]);
 #pragma unroll
-      for (int j = 0; j < 2; ++j) s[i][j] = __ffma2_rn(k2, u[j], s[i][j]);
+      for (int j = 0; j < 2; ++j) {
+        float2 x = __fmul2_rn(a2, s[i][j]);
+        x = __ffma2_rn(f2(c.x), u[0][j], x);
+        x = __ffma2_rn(f2(c.y), u[1][j], x);
+        x = __ffma2_rn(f2(c.z), u[2][j], x);
+        s[i][j] = __ffma2_rn(f2(c.w), u[3][j], x);
+      }
     }
-
-    const int64_t out_row = ((n * p.T + t) * p.HV + h) * V + col;
-    if constexpr (GATED) {
-      // per-tile sum of o^2 (lanes 0..7 of warp 0 hold the tile's 32 outputs)
-      float ss = 0.f;
-      if (writer) {
-        ss = o[0].x * o[0].x + o[0].y * o[0].y + o[1].x * o[1].x + o[1].y * o[1].y;
-#pragma unroll
-        for (int m = 1; m < kColQuads; m <<= 1) ss += __shfl_xor_sync(0x000000ffu, ss, m);
-      }
-      if (t == 0) cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
-      if (writer && lane < tiles) {
-        cluster_store_f32(cluster_map(smem_u32(&nrm[buf][tile]), static_cast<uint32_t>(lane)), ss);
-      }
-      cluster_arrive_release();
-      cluster_wait_acquire();
-      if (writer) {
-        float tot = 0.f;
-        for (int r = 0; r < tiles; ++r) tot += nrm[buf][r];
-        const float inv = rsqrtf(tot / static_cast<float>(V) + p.eps);
-        const float zz[4] = {bf16lo(cur.z[0]), bf16hi(cur.z[0]), bf16lo(cur.z[1]), bf16hi(cur.z[1])};
-        const float ov[4] = {o[0].x, o[0].y, o[1].x, o[1].y};
-        const float wv[4] = {wgt[0].x, wgt[0].y, wgt[1].x, wgt[1].y};
-        float y[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) y[j] = ov[j] * inv * wv[j] * (1.0f / (1.0f + __expf(-zz[j])));
-        *reinterpret_cast<uint2*>(p.out + out_row) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
-      }
-    } else if (writer) {
-      *reinterpret_cast<uint2*>(p.out + out_row) =
-          make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
-    }
-    if constexpr (!MULTI) break;  // T == 1
   }
 
   allow_next_grid();

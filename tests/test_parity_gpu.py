@@ -174,8 +174,14 @@ def test_t_steps_equal_successive_single_steps(gated, T, cuda_device):
                        d.g[:, sl].contiguous(), d.beta[:, sl].contiguous(), pool_b, d.slot_idx,
                        *extra(sl)))
     torch.cuda.synchronize()
-    assert torch.equal(out_a, torch.cat(outs, dim=1))
-    assert torch.equal(pool_a, pool_b)
+    # The multi-token kernel regroups the same arithmetic by chunks of tokens,
+    # so the two paths agree to rounding, not bit for bit.
+    check_out(out_a.float().cpu().numpy(), torch.cat(outs, dim=1).float().cpu().numpy(), what="T-call vs T calls")
+    for s_ in w.slot_idx.tolist():
+        check_state(pool_a[s_].cpu().numpy(), pool_b[s_].cpu().numpy(), what=f"slot {s_}")
+    untouched = torch.ones(w.num_slots, dtype=torch.bool, device=cuda_device)
+    untouched[w.slot_idx.long().to(cuda_device)] = False
+    assert torch.equal(pool_a[untouched], pool_b[untouched])
 
 
 def test_empty_batch_is_noop(cuda_device):
