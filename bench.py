@@ -286,6 +286,7 @@ def run_ours(args):
 
     # end to end through the public API: pinned host inputs in, output back out
     e2e = run_e2e(kda, base, dev, stream, min(args.steps, args.e2e_steps), world)
+    floor = None if args.no_floor else copy_floor(base, dev, stream, R, min(args.steps, 20_000))
 
     if world > 1:
         dist.barrier()
@@ -322,6 +323,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
+        "floor": floor,
         "gpu_launches": args.steps,
         "wall_s_timed": round(t_wall, 3),
     }
@@ -341,6 +343,42 @@ def _packed(tensors: dict, alloc):
     views = {k: buf[offs[k]:offs[k] + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
              for k, t in tensors.items()}
     return buf, views
+
+
+def copy_floor(w, dev, stream, R, steps):
+    """Per-call time of a plain in-place elementwise op (torch's x.mul_(c)) over
+    exactly the state bytes one decode call reads and writes, with the same
+    rotation over R buffers and CUDA-graph replay: the practical floor for
+    moving those bytes once each way per call on this GPU."""
+    import torch
+
+    n = w.state_bytes_touched() // 4
+    bufs = [torch.randn(n, device=dev) for _ in range(R)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for b in bufs:
+            b.mul_(0.999)
+        torch.cuda.current_stream().synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for b in bufs:
+                b.mul_(1.0001)
+    reps = max(1, steps // R)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * R)
+    del g
+    return {"what": "torch in-place x.mul_(c) over the same state bytes (read + write), same replica "
+                    "rotation and graph replay", "us_per_call": round(us, 3),
+            "bytes_per_call": 2 * n * 4, "gbs": round(2 * n * 4 / (us * 1e-6) / 1e9, 1)}
 
 
 def run_e2e(kda, w, dev, stream, steps, world):
@@ -458,6 +496,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5000)
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-floor", action="store_true", help="skip the in-place copy-floor reference")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
