@@ -238,6 +238,15 @@ template <int K>
 struct MinBlocks {
   static constexpr int value = K >= 256 ? 3 : (K >= 128 ? 7 : 8);
 };
+// The gated T == 1 kernel launches clusters of V/32 CTAs, which must fit in
+// one GPC: at seven CTAs per SM only 246 clusters of four (984 CTAs) are
+// co-resident on a B200, so 512 heads take three waves.  At K = V = 128 it
+// fits in 64 registers without spilling, giving eight CTAs per SM and two
+// waves.
+template <int K, int VS, bool GATED>
+struct MinBlocksT1 {
+  static constexpr int value = (GATED && K == 128 && VS == 128) ? 8 : MinBlocks<K>::value;
+};
 
 // Reduce-scatter of the two column-pair partials (S'^T k, S'^T q) across the
 // 4 row groups of a warp, then across the 4 warps through shared memory.
@@ -296,32 +305,38 @@ __device__ __forceinline__ Reduced reduce_tile(const float2 (&pk)[2], const floa
 // 0..7 of warp 0 (the writers) hold the tile's 32 outputs in o; nrm is this
 // CTA's [kMaxClusterTiles] receive buffer for the per-tile sums of o^2.
 // Every thread of every CTA in the cluster must call it (cluster barrier).
+// (Writers only) push this tile's sum of o^2 into slot `tile` of every peer's
+// receive buffer nrm.
+__device__ __forceinline__ void push_sumsq(const float2 (&o)[2], float* nrm, int tile, int tiles, int lane) {
+  float ss = o[0].x * o[0].x + o[0].y * o[0].y + o[1].x * o[1].x + o[1].y * o[1].y;
+#pragma unroll
+  for (int m = 1; m < kColQuads; m <<= 1) ss += __shfl_xor_sync(0x000000ffu, ss, m);
+  if (lane < tiles) cluster_store_f32(cluster_map(smem_u32(&nrm[tile]), static_cast<uint32_t>(lane)), ss);
+}
+// (Writers only, after the cluster barrier) y = o / rms(o) * w * sigmoid(z).
+__device__ __forceinline__ void apply_norm(float (&y)[4], const float2 (&o)[2], const float2 (&wgt)[2],
+                                           const uint32_t (&z)[2], const float* nrm, int tiles, int64_t V,
+                                           float eps) {
+  float tot = 0.f;
+  for (int r = 0; r < tiles; ++r) tot += nrm[r];
+  const float inv = rsqrtf(tot / static_cast<float>(V) + eps);
+  const float zz[4] = {bf16lo(z[0]), bf16hi(z[0]), bf16lo(z[1]), bf16hi(z[1])};
+  const float ov[4] = {o[0].x, o[0].y, o[1].x, o[1].y};
+  const float wv[4] = {wgt[0].x, wgt[0].y, wgt[1].x, wgt[1].y};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) y[j] = ov[j] * inv * wv[j] * (1.0f / (1.0f + __expf(-zz[j])));
+}
 __device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], const float2 (&wgt)[2],
                                            const uint32_t (&z)[2], float* nrm, int tile, int tiles,
                                            int64_t V, float eps, bool writer, int lane) {
-  float ss = 0.f;
-  if (writer) {
-    ss = o[0].x * o[0].x + o[0].y * o[0].y + o[1].x * o[1].x + o[1].y * o[1].y;
-#pragma unroll
-    for (int m = 1; m < kColQuads; m <<= 1) ss += __shfl_xor_sync(0x000000ffu, ss, m);
-    if (lane < tiles) cluster_store_f32(cluster_map(smem_u32(&nrm[tile]), static_cast<uint32_t>(lane)), ss);
-  }
+  if (writer) push_sumsq(o, nrm, tile, tiles, lane);
   cluster_arrive_release();
   cluster_wait_acquire();
-  if (writer) {
-    float tot = 0.f;
-    for (int r = 0; r < tiles; ++r) tot += nrm[r];
-    const float inv = rsqrtf(tot / static_cast<float>(V) + eps);
-    const float zz[4] = {bf16lo(z[0]), bf16hi(z[0]), bf16lo(z[1]), bf16hi(z[1])};
-    const float ov[4] = {o[0].x, o[0].y, o[1].x, o[1].y};
-    const float wv[4] = {wgt[0].x, wgt[0].y, wgt[1].x, wgt[1].y};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) y[j] = ov[j] * inv * wv[j] * (1.0f / (1.0f + __expf(-zz[j])));
-  }
+  if (writer) apply_norm(y, o, wgt, z, nrm, tiles, V, eps);
 }
 
 template <int K, int VS, bool GATED>
-__global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
+__global__ void __launch_bounds__(kThreads, (MinBlocksT1<K, VS, GATED>::value))
 kda_decode_kernel(const Params p) {
   constexpr int RPT = K / (kWarps * kRowGroups);
   static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
@@ -424,20 +439,25 @@ kda_decode_kernel(const Params p) {
     for (int j = 0; j < 2; ++j) s[i][j] = __ffma2_rn(k2, u[j], s[i][j]);
   }
 
-  if constexpr (GATED) {
-    cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
-    float y[4];
-    gated_norm(y, o, wgt, cur.z, nrm, tile, tiles, V, p.eps, writer, lane);
+  if constexpr (!GATED) {
     if (writer)
-      *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
-  } else if (writer) {
-    *reinterpret_cast<uint2*>(p.out + row * V + col) =
-        make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
+      *reinterpret_cast<uint2*>(p.out + row * V + col) =
+          make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
   }
 
   allow_next_grid();
 #pragma unroll
   for (int i = 0; i < RPT; ++i) __stcs(sp + i * (V / 4), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
+
+  if constexpr (GATED) {
+    // The norm needs the whole head's o; the state does not, so it is
+    // already on its way out before the cluster exchange.
+    cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
+    float y[4];
+    gated_norm(y, o, wgt, cur.z, nrm, tile, tiles, V, p.eps, writer, lane);
+    if (writer)
+      *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+  }
 }
 
 // ---------------------------------------------------------------- T > 1 kernel
@@ -572,6 +592,7 @@ kda_decode_chunked_kernel(const Params p) {
   __shared__ float mp_part[kWarps][kNumMP];
   __shared__ float mp_tot[kNumMP];
   __shared__ float nrm[2][kChunk][kMaxClusterTiles];  // gated: per-tile sums of o^2, by chunk parity
+  __shared__ float4 osm[GATED ? kChunk : 1][kColQuads];  // gated: the writers' o, by token
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -699,17 +720,10 @@ kda_decode_chunked_kernel(const Params p) {
           o[0] = __fmul2_rn(scale2, o[0]);
           o[1] = __fmul2_rn(scale2, o[1]);
         }
-        const int64_t out_row = ((n * p.T + c0 + t) * p.HV + h) * V + col;
         if constexpr (GATED) {
-          if (c0 == 0 && t == 0) cluster_wait_acquire();  // pairs with the relaxed arrive above
-          uint32_t z[2];
-          const uint2 zr = *reinterpret_cast<const uint2*>(raw.z + 4 * cq);
-          z[0] = zr.x; z[1] = zr.y;
-          float y[4];
-          gated_norm(y, o, wgt, z, nrm[cb][t], tile, tiles, V, p.eps, writer, lane);
-          if (writer)
-            *reinterpret_cast<uint2*>(p.out + out_row) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+          if (writer) osm[t][cq] = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);  // until the chunk's exchange
         } else if (writer) {
+          const int64_t out_row = ((n * p.T + c0 + t) * p.HV + h) * V + col;
           *reinterpret_cast<uint2*>(p.out + out_row) =
               make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
         }
@@ -728,6 +742,38 @@ kda_decode_chunked_kernel(const Params p) {
         x = __ffma2_rn(f2(c.y), u[1][j], x);
         x = __ffma2_rn(f2(c.z), u[2][j], x);
         s[i][j] = __ffma2_rn(f2(c.w), u[3][j], x);
+      }
+    }
+
+    if constexpr (GATED) {
+      // one cluster exchange for the whole chunk's per-token sums of o^2
+      if (c0 == 0) cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
+      if (writer) {
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) {
+          if (t < tc) {
+            const float4 ov = osm[t][cq];
+            const float2 o[2] = {make_float2(ov.x, ov.y), make_float2(ov.z, ov.w)};
+            push_sumsq(o, nrm[cb][t], tile, tiles, lane);
+          }
+        }
+      }
+      cluster_arrive_release();
+      cluster_wait_acquire();
+      if (writer) {
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) {
+          if (t < tc) {
+            const uint2 zr = *reinterpret_cast<const uint2*>(tok[cb][t].z + 4 * cq);
+            const uint32_t z[2] = {zr.x, zr.y};
+            const float4 ov = osm[t][cq];
+            const float2 o[2] = {make_float2(ov.x, ov.y), make_float2(ov.z, ov.w)};
+            float y[4];
+            apply_norm(y, o, wgt, z, nrm[cb][t], tiles, V, p.eps);
+            const int64_t out_row = ((n * p.T + c0 + t) * p.HV + h) * V + col;
+            *reinterpret_cast<uint2*>(p.out + out_row) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+          }
+        }
       }
     }
   }
