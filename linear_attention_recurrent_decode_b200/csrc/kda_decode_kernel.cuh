@@ -592,7 +592,7 @@ kda_decode_chunked_kernel(const Params p) {
   __shared__ float mp_part[kWarps][kNumMP];
   __shared__ float mp_tot[kNumMP];
   __shared__ float nrm[2][kChunk][kMaxClusterTiles];  // gated: per-tile sums of o^2, by chunk parity
-  __shared__ float4 osm[GATED ? kChunk : 1][kColQuads];  // gated: the writers' o, by token
+  __shared__ float osm[GATED ? kChunk : 1][kBV];  // gated: warp 0's o per token and column
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -638,14 +638,6 @@ kda_decode_chunked_kernel(const Params p) {
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
-  float2 wgt[2] = {f2(0.f), f2(0.f)};
-  if constexpr (GATED) {
-    const uint2 w = __ldg(reinterpret_cast<const uint2*>(p.norm_weight + col));
-    wgt[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
-    wgt[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
-  }
-  const float2 scale2 = f2(p.scale);
-
   for (int64_t c0 = 0; c0 < p.T; c0 += kChunk) {
     const int64_t left = p.T - c0;
     const int tc = static_cast<int>(left < kChunk ? left : kChunk);
@@ -674,60 +666,47 @@ kda_decode_chunked_kernel(const Params p) {
     }
     __syncthreads();
 
-    // per token: correction (all threads), readout and output (writers)
+    // Per token, in order: each lane solves one column of its quad (column
+    // 4cq + rg), the 32 lanes of warp 0 read out the tile's 32 columns, and
+    // the quad's four u values are then gathered by shuffles for the write.
+    const int jc = rg;
+    float uu[kChunk];
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) {
+      uu[t] = 0.f;
+      if (t < tc) {
+        const TokenSmem<K>& raw = tok[cb][t];
+        float R = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) R += reinterpret_cast<const float*>(&redR[w][t][cq])[jc];
+        float x = __bfloat162float(raw.v[4 * cq + jc]) - R;
+#pragma unroll
+        for (int sj = 0; sj < t; ++sj) x = fmaf(-mp_tot[m_index(t, sj)], uu[sj], x);
+        uu[t] = raw.beta[0] * x;
+        if (warp == 0) {
+          float o = 0.f;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) o += reinterpret_cast<const float*>(&redQ[w][t][cq])[jc];
+#pragma unroll
+          for (int sj = 0; sj <= t; ++sj) o = fmaf(mp_tot[p_index(t, sj)], uu[sj], o);
+          o *= p.scale;
+          if constexpr (GATED) {
+            osm[t][4 * cq + jc] = o;  // until the chunk's exchange
+          } else {
+            p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(o);
+          }
+        }
+      }
+    }
     float2 u[kChunk][2];
 #pragma unroll
     for (int t = 0; t < kChunk; ++t) {
-      u[t][0] = u[t][1] = f2(0.f);
-      if (t < tc) {
-        const TokenSmem<K>& raw = tok[cb][t];
-        const uint2 vr = *reinterpret_cast<const uint2*>(raw.v + 4 * cq);
-        float2 x[2] = {make_float2(bf16lo(vr.x), bf16hi(vr.x)), make_float2(bf16lo(vr.y), bf16hi(vr.y))};
-        float4 R = redR[0][t][cq];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) {
-          const float4 a = redR[w][t][cq];
-          R = make_float4(R.x + a.x, R.y + a.y, R.z + a.z, R.w + a.w);
-        }
-        x[0] = __fadd2_rn(x[0], make_float2(-R.x, -R.y));
-        x[1] = __fadd2_rn(x[1], make_float2(-R.z, -R.w));
-#pragma unroll
-        for (int sj = 0; sj < t; ++sj) {
-          const float2 m2 = f2(-mp_tot[m_index(t, sj)]);
-          x[0] = __ffma2_rn(m2, u[sj][0], x[0]);
-          x[1] = __ffma2_rn(m2, u[sj][1], x[1]);
-        }
-        const float2 b2 = f2(raw.beta[0]);
-        u[t][0] = __fmul2_rn(b2, x[0]);
-        u[t][1] = __fmul2_rn(b2, x[1]);
-
-        float2 o[2] = {f2(0.f), f2(0.f)};
-        if (writer) {
-          float4 Q = redQ[0][t][cq];
-#pragma unroll
-          for (int w = 1; w < kWarps; ++w) {
-            const float4 a = redQ[w][t][cq];
-            Q = make_float4(Q.x + a.x, Q.y + a.y, Q.z + a.z, Q.w + a.w);
-          }
-          o[0] = make_float2(Q.x, Q.y);
-          o[1] = make_float2(Q.z, Q.w);
-#pragma unroll
-          for (int sj = 0; sj <= t; ++sj) {
-            const float2 p2 = f2(mp_tot[p_index(t, sj)]);
-            o[0] = __ffma2_rn(p2, u[sj][0], o[0]);
-            o[1] = __ffma2_rn(p2, u[sj][1], o[1]);
-          }
-          o[0] = __fmul2_rn(scale2, o[0]);
-          o[1] = __fmul2_rn(scale2, o[1]);
-        }
-        if constexpr (GATED) {
-          if (writer) osm[t][cq] = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);  // until the chunk's exchange
-        } else if (writer) {
-          const int64_t out_row = ((n * p.T + c0 + t) * p.HV + h) * V + col;
-          *reinterpret_cast<uint2*>(p.out + out_row) =
-              make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
-        }
-      }
+      const float a0 = __shfl_sync(0xffffffffu, uu[t], cq);
+      const float a1 = __shfl_sync(0xffffffffu, uu[t], kColQuads + cq);
+      const float a2 = __shfl_sync(0xffffffffu, uu[t], 2 * kColQuads + cq);
+      const float a3 = __shfl_sync(0xffffffffu, uu[t], 3 * kColQuads + cq);
+      u[t][0] = make_float2(a0, a1);
+      u[t][1] = make_float2(a2, a3);
     }
 
     // chunk-end state: S = A_last S0 + sum_t c_t u_t^T
@@ -748,30 +727,32 @@ kda_decode_chunked_kernel(const Params p) {
     if constexpr (GATED) {
       // one cluster exchange for the whole chunk's per-token sums of o^2
       if (c0 == 0) cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
-      if (writer) {
+      if (warp == 0) {
 #pragma unroll
         for (int t = 0; t < kChunk; ++t) {
           if (t < tc) {
-            const float4 ov = osm[t][cq];
-            const float2 o[2] = {make_float2(ov.x, ov.y), make_float2(ov.z, ov.w)};
-            push_sumsq(o, nrm[cb][t], tile, tiles, lane);
+            const float o = osm[t][4 * cq + jc];
+            float ss = o * o;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+            if (lane < tiles)
+              cluster_store_f32(cluster_map(smem_u32(&nrm[cb][t][tile]), static_cast<uint32_t>(lane)), ss);
           }
         }
       }
       cluster_arrive_release();
       cluster_wait_acquire();
-      if (writer) {
+      if (warp == 0) {
+        const float wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + jc]);
 #pragma unroll
         for (int t = 0; t < kChunk; ++t) {
           if (t < tc) {
-            const uint2 zr = *reinterpret_cast<const uint2*>(tok[cb][t].z + 4 * cq);
-            const uint32_t z[2] = {zr.x, zr.y};
-            const float4 ov = osm[t][cq];
-            const float2 o[2] = {make_float2(ov.x, ov.y), make_float2(ov.z, ov.w)};
-            float y[4];
-            apply_norm(y, o, wgt, z, nrm[cb][t], tiles, V, p.eps);
-            const int64_t out_row = ((n * p.T + c0 + t) * p.HV + h) * V + col;
-            *reinterpret_cast<uint2*>(p.out + out_row) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+            float tot = 0.f;
+            for (int r = 0; r < tiles; ++r) tot += nrm[cb][t][r];
+            const float inv = rsqrtf(tot / static_cast<float>(V) + p.eps);
+            const float z = __bfloat162float(tok[cb][t].z[4 * cq + jc]);
+            const float y = osm[t][4 * cq + jc] * inv * wj * (1.0f / (1.0f + __expf(-z)));
+            p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(y);
           }
         }
       }
