@@ -131,3 +131,11 @@ def test_binding_refuses_cpu_tensors():
     w = workloads.make(N=1, T=1, HV=1, K=64, V=32, num_slots=1)
     with pytest.raises(ValueError, match="CUDA"):
         kda.kda_decode(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx)
+
+
+@no_gpu
+def test_size_limits_are_rejected_on_the_host(lib):
+    # grid = N * HV * V/32 CTAs must fit in 2^31 - 1
+    assert call(lib, N=1 << 28, HV=2, V=128) == kda.KDA_ERR_UNSUPPORTED
+    # element counts that overflow int64
+    assert call(lib, N=1 << 40, T=1 << 20, HV=1 << 10) == kda.KDA_ERR_UNSUPPORTED

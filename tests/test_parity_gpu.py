@@ -144,6 +144,12 @@ CASES = [
     (2, 20, 2, 256, 64, False, 0),
     (3, 9, 2, 128, 128, True, 1),
     (2, 17, 1, 64, 256, True, 0),
+    # widest supported shapes: 8 value tiles with K = 256 (plain and one cluster of 8), many heads
+    (2, 1, 2, 256, 256, False, 0),
+    (2, 2, 2, 256, 256, True, 0),
+    (1, 1, 64, 128, 128, False, 0),
+    (1, 5, 48, 128, 128, True, 0),
+    (3, 1, 1, 128, 512, False, 0),
 ]
 
 
@@ -280,3 +286,26 @@ def test_back_to_back_calls_see_prior_writes(gated, cuda_device):
         g = g + -0.25
     for s in w.slot_idx.tolist():
         check_state(d.state[s].cpu().numpy(), state[s], what=f"slot {s}")
+
+
+def test_random_shapes_against_oracle(cuda_device):
+    """Seeded sweep of small random shapes (all K, V multiples of 32 up to 256,
+    T up to 11, random padding rows, plain and gated) against the oracle."""
+    rng = np.random.default_rng(20261202)
+    for case in range(24):
+        K = int(rng.choice([64, 128, 256]))
+        gated = bool(rng.integers(0, 2))
+        V = 32 * int(rng.integers(1, 9))
+        N = int(rng.integers(1, 6))
+        T = int(rng.integers(1, 12))
+        HV = int(rng.integers(1, 5))
+        inactive = int(rng.integers(0, N))
+        w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + int(rng.integers(0, 4)), gated=gated,
+                           inactive=inactive, seed=1000 + case,
+                           decay=str(rng.choice(["softplus", "uniform"])))
+        o, pool, before = run_gpu(w, cuda_device)
+        try:
+            assert_parity(w, o, pool, before)
+        except AssertionError as e:
+            raise AssertionError(f"case {case}: N={N} T={T} HV={HV} K={K} V={V} gated={gated} "
+                                 f"inactive={inactive}: {e}") from e
