@@ -39,6 +39,7 @@
  *     g           fp32  [N, T, HV, K]     log-decay, decay = exp(g)
  *     beta        fp32  [N, T, HV]
  *     state_pool  fp32  [num_slots, HV, K, V], read and written in place
+ *                 (bf16 for the *_bf16_state entry points)
  *     slot_idx    int32 [N]               slot of each row; < 0 = inactive row
  *     out         bf16  [N, T, HV, V]
  *     gate (z)    bf16  [N, T, HV, V]     gated variant only
@@ -121,6 +122,30 @@ KDA_API kda_status kda_decode_gated_rmsnorm(const void *q, const void *k, const 
                                     const void *norm_weight, float eps, void *out, int64_t N,
                                     int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
                                     kda_stream_t stream);
+
+/*
+ * The same two operations on a bf16 state pool (state_pool: bf16 bits,
+ * [num_slots, HV, K, V]).  The state is widened exactly, every step runs in
+ * fp32 exactly as in the fp32-pool entry points, and the state is rounded to
+ * the nearest bf16 (ties to even) once, when it is written back after the
+ * call's last token.  The pool's traffic halves.  Source: FlashInfer #4562
+ * "feat(cake_kda): add optimized H12 packed decode across SM100 family"
+ * keeps the recurrent state in bf16 (the binding's kernel launch passes the
+ * state as `__nv_bfloat16*`).  Arguments, layouts, alignment, errors and the
+ * caller contract are those of kda_decode / kda_decode_gated_rmsnorm.
+ */
+KDA_API kda_status kda_decode_bf16_state(const void *q, const void *k, const void *v, const float *g,
+                                         const float *beta, void *state_pool, const int32_t *slot_idx,
+                                         void *out, int64_t N, int64_t T, int64_t HV, int64_t K,
+                                         int64_t V, float scale, kda_stream_t stream);
+
+KDA_API kda_status kda_decode_gated_rmsnorm_bf16_state(const void *q, const void *k, const void *v,
+                                                       const float *g, const float *beta,
+                                                       void *state_pool, const int32_t *slot_idx,
+                                                       const void *gate, const void *norm_weight,
+                                                       float eps, void *out, int64_t N, int64_t T,
+                                                       int64_t HV, int64_t K, int64_t V, float scale,
+                                                       kda_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);

@@ -11,7 +11,7 @@ missing or the device is not sm_100a, the call raises.
 
 Tensor layouts (contiguous, on the current CUDA device):
     q, k bf16 [N,T,HV,K]; v bf16 [N,T,HV,V]; g fp32 [N,T,HV,K] (log-decay);
-    beta fp32 [N,T,HV]; state_pool fp32 [num_slots,HV,K,V]; slot_idx int32 [N]
+    beta fp32 [N,T,HV]; state_pool fp32 or bf16 [num_slots,HV,K,V]; slot_idx int32 [N]
     (negative = inactive row); out bf16 [N,T,HV,V]; gate bf16 [N,T,HV,V];
     norm_weight bf16 [V].
 """
@@ -41,6 +41,8 @@ _P, _I, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
 EXPORTED_SYMBOLS = {
     "kda_decode": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_gated_rmsnorm": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
+    "kda_decode_bf16_state": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
+    "kda_decode_gated_rmsnorm_bf16_state": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_abi_version": ([], ctypes.c_int32),
 }
@@ -115,7 +117,9 @@ def _common(q, k, v, g, beta, state_pool, slot_idx, out):
     _check(g, "g", torch.float32, (N, T, HV, K))
     _check(beta, "beta", torch.float32, (N, T, HV))
     _check(slot_idx, "slot_idx", torch.int32, (N,))
-    _check(state_pool, "state_pool", torch.float32)
+    if state_pool.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"state_pool must be float32 or bfloat16, got {state_pool.dtype}")
+    _check(state_pool, "state_pool", state_pool.dtype)
     if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (HV, K, V):
         raise ValueError(f"state_pool must be [num_slots, {HV}, {K}, {V}]")
     if out is None:
@@ -128,15 +132,19 @@ def kda_decode(q, k, v, g, beta, state_pool, slot_idx, out=None, scale: float | 
                stream=None):
     """Recurrent KDA decode step on the caller's stream; updates ``state_pool`` in
     place and returns ``out`` (allocated if not given).  ``scale`` defaults to
-    1/sqrt(K)."""
+    1/sqrt(K).  A bf16 ``state_pool`` runs the bf16-state entry point (fp32
+    math, state rounded to bf16 once per call)."""
+    import torch
+
     N, T, HV, K, V, out = _common(q, k, v, g, beta, state_pool, slot_idx, out)
     if scale is None:
         scale = 1.0 / math.sqrt(K)
-    st = library().kda_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
-                              state_pool.data_ptr(), slot_idx.data_ptr(), out.data_ptr(),
-                              N, T, HV, K, V, float(scale), _stream_handle(stream))
+    name = "kda_decode_bf16_state" if state_pool.dtype == torch.bfloat16 else "kda_decode"
+    st = getattr(library(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+                                  state_pool.data_ptr(), slot_idx.data_ptr(), out.data_ptr(),
+                                  N, T, HV, K, V, float(scale), _stream_handle(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_decode")
+        raise KdaError(st, name)
     return out
 
 
@@ -151,10 +159,12 @@ def kda_decode_gated_rmsnorm(q, k, v, g, beta, state_pool, slot_idx, gate, norm_
     _check(norm_weight, "norm_weight", torch.bfloat16, (V,))
     if scale is None:
         scale = 1.0 / math.sqrt(K)
-    st = library().kda_decode_gated_rmsnorm(
+    name = ("kda_decode_gated_rmsnorm_bf16_state" if state_pool.dtype == torch.bfloat16
+            else "kda_decode_gated_rmsnorm")
+    st = getattr(library(), name)(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(), state_pool.data_ptr(),
         slot_idx.data_ptr(), gate.data_ptr(), norm_weight.data_ptr(), float(eps), out.data_ptr(),
         N, T, HV, K, V, float(scale), _stream_handle(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_decode_gated_rmsnorm")
+        raise KdaError(st, name)
     return out

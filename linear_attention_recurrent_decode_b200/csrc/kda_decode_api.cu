@@ -49,9 +49,9 @@ bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
 bool mul_ok(int64_t a, int64_t b, int64_t* r) { return !__builtin_mul_overflow(a, b, r); }
 
 kda_status launch(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                  float* state_pool, const int32_t* slot_idx, const void* gate,
+                  void* state_pool, const int32_t* slot_idx, const void* gate,
                   const void* norm_weight, float eps, void* out, int64_t N, int64_t T, int64_t HV,
-                  int64_t K, int64_t V, float scale, kda_stream_t stream, bool gated) {
+                  int64_t K, int64_t V, float scale, kda_stream_t stream, bool gated, bool bf16_state) {
   // ---- sizes
   if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0) return KDA_ERR_INVALID_ARG;
   if (gated && !(eps >= 0.0f && eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
@@ -86,7 +86,7 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
       range_of(gated ? norm_weight : nullptr, gated ? V * 2 : 0)};
   // The pool's extent depends on slot values held on the device; the visible
   // part is slot 0 plus the base address itself.
-  const Range r_slot0 = range_of(state_pool, HV * K * V * 4);
+  const Range r_slot0 = range_of(state_pool, HV * K * V * (bf16_state ? 2 : 4));
   const uintptr_t pool_base = reinterpret_cast<uintptr_t>(state_pool);
   auto touches_pool = [&](Range r) {
     return overlaps(r, r_slot0) || (r.lo <= pool_base && pool_base < r.hi);
@@ -143,9 +143,13 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
   cudaError_t err = cudaErrorInvalidValue;
   const bool multi = T > 1;
   const bool v128 = V == 128;
-  // One instantiation per (K, V fixed at 128 or not, gated); T == 1 and T > 1
-  // (chunked) kernels.
-#define KDA_LAUNCH(KERNEL, KK, VV, GG) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG>, p)
+  // One instantiation per (K, V fixed at 128 or not, gated, state type); T == 1
+  // and T > 1 (chunked) kernels.
+#define KDA_LAUNCH(KERNEL, KK, VV, GG)                                                      \
+  do {                                                                                      \
+    if (bf16_state) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, __nv_bfloat16>, p); \
+    else err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, float>, p);                  \
+  } while (0)
 #define KDA_LAUNCH_V(KK, GG)                                                 \
   do {                                                                       \
     if (multi) {                                                             \
@@ -181,7 +185,7 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
                       float* state_pool, const int32_t* slot_idx, void* out, int64_t N, int64_t T,
                       int64_t HV, int64_t K, int64_t V, float scale, kda_stream_t stream) {
   return launch(q, k, v, g, beta, state_pool, slot_idx, nullptr, nullptr, 0.0f, out, N, T, HV, K, V,
-                scale, stream, /*gated=*/false);
+                scale, stream, /*gated=*/false, /*bf16_state=*/false);
 }
 
 kda_status kda_decode_gated_rmsnorm(const void* q, const void* k, const void* v, const float* g,
@@ -190,7 +194,25 @@ kda_status kda_decode_gated_rmsnorm(const void* q, const void* k, const void* v,
                                     int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
                                     float scale, kda_stream_t stream) {
   return launch(q, k, v, g, beta, state_pool, slot_idx, gate, norm_weight, eps, out, N, T, HV, K, V,
-                scale, stream, /*gated=*/true);
+                scale, stream, /*gated=*/true, /*bf16_state=*/false);
+}
+
+kda_status kda_decode_bf16_state(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, void* state_pool, const int32_t* slot_idx, void* out,
+                                 int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
+                                 kda_stream_t stream) {
+  return launch(q, k, v, g, beta, state_pool, slot_idx, nullptr, nullptr, 0.0f, out, N, T, HV, K, V,
+                scale, stream, /*gated=*/false, /*bf16_state=*/true);
+}
+
+kda_status kda_decode_gated_rmsnorm_bf16_state(const void* q, const void* k, const void* v,
+                                               const float* g, const float* beta, void* state_pool,
+                                               const int32_t* slot_idx, const void* gate,
+                                               const void* norm_weight, float eps, void* out, int64_t N,
+                                               int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
+                                               kda_stream_t stream) {
+  return launch(q, k, v, g, beta, state_pool, slot_idx, gate, norm_weight, eps, out, N, T, HV, K, V,
+                scale, stream, /*gated=*/true, /*bf16_state=*/true);
 }
 
 const char* kda_status_string(kda_status status) {
@@ -207,6 +229,6 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 0; }
+int32_t kda_abi_version(void) { return (1 << 16) | 1; }
 
 }  // extern "C"

@@ -41,6 +41,10 @@
 // memory (DSMEM) and a cluster barrier completes the RMS over V; the norm,
 // weight and sigmoid gate are applied before the bf16 store.
 //
+// The state pool is fp32 or bf16 (template parameter ST).  A bf16 pool is
+// widened exactly on load, all arithmetic is fp32, and the state is rounded
+// to nearest even once, when it is written back at the end of the call.
+//
 // Launch overlap: kernels are launched with programmatic stream
 // serialization.  Every global access of a CTA comes after griddepcontrol.wait
 // (all work earlier in the stream complete and visible), and a CTA lets the
@@ -81,7 +85,7 @@ struct Params {
   const __nv_bfloat16* v;
   const float* g;
   const float* beta;
-  float* state;
+  void* state;  // fp32 or bf16 [num_slots, HV, K, V] (the kernel's ST)
   const int32_t* slot_idx;
   __nv_bfloat16* out;
   const __nv_bfloat16* gate;         // gated variant only
@@ -105,6 +109,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// Four consecutive state values of one key row, in the pool's element type
+// ST: fp32 (128-bit accesses) or bf16 (64-bit accesses; widened exactly on
+// load, rounded to nearest even on store).  Stores stream (evict-first): the
+// state is not read again before the next decode step.
+template <typename ST>
+struct StateIO;
+template <>
+struct StateIO<float> {
+  static __device__ __forceinline__ void load(float2 (&s)[2], const float* p) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    s[0] = make_float2(x.x, x.y);
+    s[1] = make_float2(x.z, x.w);
+  }
+  static __device__ __forceinline__ void store(float* p, const float2 (&s)[2]) {
+    __stcs(reinterpret_cast<float4*>(p), make_float4(s[0].x, s[0].y, s[1].x, s[1].y));
+  }
+};
+template <>
+struct StateIO<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(float2 (&s)[2], const __nv_bfloat16* p) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    s[0] = make_float2(bf16lo(x.x), bf16hi(x.x));
+    s[1] = make_float2(bf16lo(x.y), bf16hi(x.y));
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float2 (&s)[2]) {
+    __stcs(reinterpret_cast<uint2*>(p), make_uint2(pack_bf16x2(s[0].x, s[0].y), pack_bf16x2(s[1].x, s[1].y)));
+  }
+};
 
 // RPT consecutive bf16 values (RPT = 4: 8 bytes; RPT % 8 == 0: 16-byte chunks).
 template <int RPT>
@@ -335,7 +368,7 @@ __device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], 
   if (writer) apply_norm(y, o, wgt, z, nrm, tiles, V, eps);
 }
 
-template <int K, int VS, bool GATED>
+template <int K, int VS, bool GATED, typename ST>
 __global__ void __launch_bounds__(kThreads, (MinBlocksT1<K, VS, GATED>::value))
 kda_decode_kernel(const Params p) {
   constexpr int RPT = K / (kWarps * kRowGroups);
@@ -382,15 +415,10 @@ kda_decode_kernel(const Params p) {
     return;  // uniform over the cluster: every tile of this (n, h) sees the same slot
   }
 
-  float4* const sp =
-      reinterpret_cast<float4*>(p.state + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col);
+  ST* const sp = static_cast<ST*>(p.state) + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col;
   float2 s[RPT][2];
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const float4 x = sp[i * (V / 4)];
-    s[i][0] = make_float2(x.x, x.y);
-    s[i][1] = make_float2(x.z, x.w);
-  }
+  for (int i = 0; i < RPT; ++i) StateIO<ST>::load(s[i], sp + i * V);
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
@@ -447,7 +475,7 @@ kda_decode_kernel(const Params p) {
 
   allow_next_grid();
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) __stcs(sp + i * (V / 4), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
+  for (int i = 0; i < RPT; ++i) StateIO<ST>::store(sp + i * V, s[i]);
 
   if constexpr (GATED) {
     // The norm needs the whole head's o; the state does not, so it is
@@ -578,7 +606,7 @@ __device__ __forceinline__ void chunk_pass(const float2 (&s)[RPT][2], const floa
   red[warp][rg][cq] = make_float4(mine[0].x, mine[0].y, mine[1].x, mine[1].y);
 }
 
-template <int K, int VS, bool GATED>
+template <int K, int VS, bool GATED, typename ST>
 __global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
 kda_decode_chunked_kernel(const Params p) {
   constexpr int RPT = K / (kWarps * kRowGroups);
@@ -626,15 +654,10 @@ kda_decode_chunked_kernel(const Params p) {
     return;
   }
 
-  float4* const sp =
-      reinterpret_cast<float4*>(p.state + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col);
+  ST* const sp = static_cast<ST*>(p.state) + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col;
   float2 s[RPT][2];
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const float4 x = sp[i * (V / 4)];
-    s[i][0] = make_float2(x.x, x.y);
-    s[i][1] = make_float2(x.z, x.w);
-  }
+  for (int i = 0; i < RPT; ++i) StateIO<ST>::load(s[i], sp + i * V);
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
@@ -761,7 +784,7 @@ kda_decode_chunked_kernel(const Params p) {
 
   allow_next_grid();
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) __stcs(sp + i * (V / 4), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
+  for (int i = 0; i < RPT; ++i) StateIO<ST>::store(sp + i * V, s[i]);
 }
 
 }  // namespace kda

@@ -7,6 +7,7 @@ the CPU with ``torch.Generator`` (seeded) and may then be copied to a device.
 
 Input recipe (every configuration, unless stated otherwise):
   * state pool fp32 ``[num_slots, HV, K, V]`` ~ N(0, 0.02^2) (0.02 is the std);
+    for a bf16 pool the same draw is rounded to bf16;
   * q, k, v drawn fp32 ~ N(0, 1); q and k are L2-normalised over K per
     (n, t, h) in fp32 and then all three are rounded to bf16;
   * g fp32 ``[N, T, HV, K]`` = -softplus(N(0, 1)) per key channel (log-decay);
@@ -81,7 +82,7 @@ class Workload:
     def state_bytes_touched(self) -> int:
         """State bytes one call reads (it writes the same amount back)."""
         active = int((self.slot_idx >= 0).sum())
-        return active * self.HV * self.K * self.V * 4
+        return active * self.HV * self.K * self.V * self.state.element_size()
 
 
 def _bf16(x: torch.Tensor) -> torch.Tensor:
@@ -90,7 +91,8 @@ def _bf16(x: torch.Tensor) -> torch.Tensor:
 
 def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | None = None,
          gated: bool = False, seed: int = 0, name: str = "custom",
-         decay: str = "softplus", inactive: int = 0, state_std: float = 0.02) -> Workload:
+         decay: str = "softplus", inactive: int = 0, state_std: float = 0.02,
+         state_dtype: str = "fp32") -> Workload:
     """Draw one call's inputs.
 
     ``decay``: ``"softplus"`` (g = -softplus(N(0,1))) or ``"uniform"``
@@ -119,6 +121,10 @@ def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | N
         raise ValueError(decay)
     beta = torch.sigmoid(randn(N, T, HV))
     state = randn(num_slots, HV, K, V) * state_std
+    if state_dtype == "bf16":
+        state = state.to(torch.bfloat16)
+    elif state_dtype != "fp32":
+        raise ValueError(state_dtype)
     slot_idx = torch.randperm(num_slots, generator=gen)[:N].to(torch.int32)
     if inactive:
         slot_idx[N - inactive:] = -1
@@ -141,6 +147,11 @@ CONFIGS = {
     "n8_t4_hv8": dict(N=8, T=4, HV=8, num_slots=16),
     "n32_t4_hv8": dict(N=32, T=4, HV=8, num_slots=64),
     "n256_t1_hv32": dict(N=256, T=1, HV=32, num_slots=1024, decay="uniform"),
+    # bf16 state pool (the state traffic halves)
+    "n32_t1_hv8_bf16state": dict(N=32, T=1, HV=8, num_slots=64, state_dtype="bf16"),
+    "n32_t1_hv16_gated_bf16state": dict(N=32, T=1, HV=16, num_slots=128, gated=True, state_dtype="bf16"),
+    "n32_t4_hv8_bf16state": dict(N=32, T=4, HV=8, num_slots=64, state_dtype="bf16"),
+    "n256_t1_hv32_bf16state": dict(N=256, T=1, HV=32, num_slots=1024, decay="uniform", state_dtype="bf16"),
 }
 
 

@@ -55,6 +55,9 @@ def load_library(path: str):
     D = ctypes.c_double
     f.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, D, D, I, I, P, P]
     f.restype = ctypes.c_int
+    r = lib.kda_oracle_round_bf16
+    r.argtypes = [P, P, I]
+    r.restype = None
     return lib
 
 
@@ -87,6 +90,15 @@ def _ptr(a: np.ndarray | None):
     return None if a is None else a.ctypes.data
 
 
+def round_bf16(x) -> np.ndarray:
+    """Doubles rounded to bf16 (nearest, ties to even) by the oracle's own C
+    routine; returned as float64 values."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    bits = np.empty(a.shape, dtype=np.uint16)
+    _load().kda_oracle_round_bf16(_ptr(a), _ptr(bits), a.size)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def kda_decode_ref(q, k, v, g, beta, state_pool, slot_idx, scale: float,
                    gate=None, norm_weight=None, eps: float = 1e-6,
                    threads: int = 1, units: tuple[int, int] | None = None,
@@ -117,9 +129,14 @@ def kda_decode_ref(q, k, v, g, beta, state_pool, slot_idx, scale: float,
         raise ValueError("gate and norm_weight go together")
     zb = None if gate is None else _as_bf16_bits(gate).reshape(N, T, HV, V)
     wb = None if norm_weight is None else _as_bf16_bits(norm_weight).reshape(V)
+    bf16_state = False
     if state_inplace is not None:
         st = state_inplace
         assert st.dtype == np.float64 and st.flags.c_contiguous
+    elif isinstance(state_pool, np.ndarray) and state_pool.dtype == np.uint16 or (
+            not isinstance(state_pool, np.ndarray) and str(state_pool.dtype) == "torch.bfloat16"):
+        bf16_state = True
+        st = (_as_bf16_bits(state_pool).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     else:
         st = _as_np(state_pool, np.float64).copy()
     num_slots = st.shape[0]
@@ -149,4 +166,6 @@ def kda_decode_ref(q, k, v, g, beta, state_pool, slot_idx, scale: float,
         bounds = sorted(set(int(b) for b in np.linspace(b0, b1, threads + 1)))
         with ThreadPoolExecutor(max_workers=threads) as ex:
             list(ex.map(lambda ab: run(*ab), zip(bounds[:-1], bounds[1:])))
+    if bf16_state:
+        st = round_bf16(st)
     return out, st

@@ -41,7 +41,11 @@
  *  - a negative slot index marks an inactive (graph-padding) row: its output
  *    is zero and the pool is not read or written;
  *  - bf16 inputs are widened exactly (bits << 16) and every step runs in
- *    double; outputs are left unrounded.
+ *    double; outputs are left unrounded;
+ *  - a bf16 state pool (FlashInfer #4562 keeps the recurrent state in bf16)
+ *    is widened exactly on entry, the steps run in double as above, and the
+ *    state is rounded to bf16 (nearest, ties to even) once, when the call
+ *    writes it back.
  *
  * The oracle is written as loops in the order of the steps above.  It uses
  * no blocking, no fusion and no algebraic shortcut (in particular it computes
@@ -171,4 +175,35 @@ int kda_oracle_decode_units(const uint16_t *q, const uint16_t *k, const uint16_t
                         rk_scratch, u_scratch);
     }
     return 0;
+}
+
+/*
+ * Round doubles to bf16 (round to nearest, ties to even), as the bf16-state
+ * variant does when it writes the state back at the end of a call.  Returns
+ * the bf16 bit patterns.  Written from the format's definition: 8 significant
+ * bits, exponent range of binary32 (normal down to 2^-126, subnormal steps of
+ * 2^-133), overflow to infinity past the largest finite value.
+ */
+static uint16_t double_to_bf16_rne(double x)
+{
+    if (isnan(x)) return 0x7fc0;
+    const uint16_t sign = signbit(x) ? 0x8000 : 0;
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    int e;
+    const double m = frexp(a, &e); /* a = m 2^e, m in [0.5, 1): leading bit has weight 2^(e-1) */
+    int lsb = (e - 1) - 7;         /* weight of the last kept bit for a normal bf16 */
+    if (lsb < -133) lsb = -133;    /* subnormal spacing */
+    const double q = nearbyint(ldexp(a, -lsb)); /* current rounding mode: to nearest, ties to even */
+    const double y = ldexp(q, lsb);
+    if (y > 3.38953138925153547590470800371487866880e38) return sign | 0x7f80; /* overflow */
+    const float f = (float)y; /* exact: at most 8 significant bits inside the binary32 range */
+    uint32_t w;
+    memcpy(&w, &f, sizeof w);
+    return sign | (uint16_t)(w >> 16);
+}
+
+void kda_oracle_round_bf16(const double *in, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16_rne(in[i]);
 }

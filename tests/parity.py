@@ -62,3 +62,22 @@ def check_state(got, ref, what="state"):
     mx = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
     assert rel <= STATE_REL, f"{what}: normwise relative error {rel:.3e} > {STATE_REL}"
     assert mx <= STATE_REL, f"{what}: max abs error / max|ref| = {mx:.3e} > {STATE_REL}"
+
+
+def check_state_bf16(got, ref, what="bf16 state"):
+    """A bf16 pool: the kernel rounds its fp32 state once, the oracle rounds its
+    fp64 state once, so each element agrees to one bf16 ulp (fp32 error can
+    move a value across a rounding boundary), plus 1e-6 max|ref| for values so
+    small that fp32 cancellation error exceeds their ulp."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    bound = bf16_ulp(ref) + 1e-6 * np.max(np.abs(ref))
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {err.size} elements off by more than 1 bf16 ulp; "
+                             f"worst at {i}: got {got[i]!r} ref {ref[i]!r}")
+    assert np.mean(got != ref) < 0.01, f"{what}: more than 1% of elements differ from the oracle"

@@ -33,7 +33,8 @@ def declared_functions():
 
 
 def test_header_declares_the_documented_entry_points():
-    assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_status_string",
+    assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
+                                    "kda_decode_gated_rmsnorm_bf16_state", "kda_status_string",
                                     "kda_abi_version"}
 
 
@@ -54,7 +55,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16)
+    assert lib.kda_abi_version() == (1 << 16) | 1
 
 
 # ----------------------------------------------------------------- validation

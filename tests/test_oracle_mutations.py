@@ -44,6 +44,9 @@ MUTANTS = {
     "eps_outside_sqrt": ("1.0 / sqrt(ss / (double)V + eps)", "1.0 / (sqrt(ss / (double)V) + eps)"),
     "sum_not_mean": ("ss / (double)V + eps", "ss + eps"),
     "no_norm_weight": (" * bf16_to_double(w[j]) * gate", " * gate"),
+    "bf16_truncates": ("const double q = nearbyint(ldexp(a, -lsb));", "const double q = floor(ldexp(a, -lsb));"),
+    "bf16_ties_away": ("const double q = nearbyint(ldexp(a, -lsb));", "const double q = round(ldexp(a, -lsb));"),
+    "bf16_no_subnormal": ("if (lsb < -133) lsb = -133;", "if (lsb < -200) lsb = -200;"),
 }
 
 

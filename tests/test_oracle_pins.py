@@ -309,3 +309,64 @@ def test_gated_unit_gate_gives_unit_rms():
     ratio = y / o
     np.testing.assert_allclose(ratio, ratio[..., :1] * np.ones_like(ratio), rtol=1e-12)
     assert np.all(ratio > 0)
+
+
+# ---------------------------------------------------------------------------
+# bf16 state: the oracle's own rounding, and the state closed forms through it
+# ---------------------------------------------------------------------------
+def _bits_to_f64(bits):
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_round_bf16_round_trip_and_ties():
+    rng = np.random.default_rng(7)
+    bits = rng.integers(0, 1 << 16, size=200_000, dtype=np.uint32).astype(np.uint16)
+    finite = (bits & 0x7F80) != 0x7F80
+    vals = _bits_to_f64(bits[finite])
+    np.testing.assert_array_equal(oracle.round_bf16(vals), vals)  # exact values are kept
+    # midpoints between neighbours round to the even neighbour, nudges go to the nearer one
+    b = bits[finite & ((bits & 0x7FFF) < 0x7F7F) & ((bits & 0x7FFF) > 0)]
+    lo, hi = _bits_to_f64(b), _bits_to_f64(b + 1)
+    mid = (lo + hi) / 2
+    even = np.where((b & 1) == 0, lo, hi)
+    np.testing.assert_array_equal(oracle.round_bf16(mid), even)
+    step = np.abs(hi - lo)
+    np.testing.assert_array_equal(oracle.round_bf16(mid - step / 8 * np.sign(hi - lo)), lo)
+    np.testing.assert_array_equal(oracle.round_bf16(mid + step / 8 * np.sign(hi - lo)), hi)
+
+
+def test_round_bf16_matches_library_conversion():
+    """torch's float64 -> bfloat16 conversion is an independent implementation
+    of the same rounding, subnormals and overflow included.  It goes through
+    float32, which double-rounds inputs whose float32 image is exactly a bf16
+    midpoint; those (about 1 in 50,000) are left to the midpoint test above."""
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal(300_000) * np.exp2(rng.uniform(-140, 130, 300_000))
+    x = np.concatenate([x, [0.0, -0.0, 3.3895313892515355e38, 3.3896e38, -3.5e38, 1e-45, 9.2e-41]])
+    f32_bits = x.astype(np.float32).view(np.uint32)
+    single_rounding = (f32_bits & 0xFFFF) != 0x8000
+    assert single_rounding.mean() > 0.999
+    x = x[single_rounding]
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x), ref)
+
+
+def test_bf16_state_closed_forms():
+    """bf16 pool: beta=0, g=0 leaves it bit-identical; from S=0 one step stores
+    round(beta k v^T)."""
+    w = workloads.make(N=2, T=1, HV=2, K=8, V=8, num_slots=3, seed=9, state_dtype="bf16")
+    w.beta.zero_()
+    w.g.zero_()
+    _, st = run(w)
+    np.testing.assert_array_equal(st, w.state.double().numpy())
+    w = workloads.make(N=2, T=1, HV=2, K=8, V=8, num_slots=3, seed=10, state_dtype="bf16")
+    w.state.zero_()
+    _, st = run(w)
+    k, v = bf16_vals(w.k), bf16_vals(w.v)
+    b = w.beta.double().numpy()
+    for n in range(w.N):
+        slot = int(w.slot_idx[n])
+        for h in range(w.HV):
+            exact = b[n, 0, h] * np.outer(k[n, 0, h], v[n, 0, h])
+            ref = torch.from_numpy(exact).to(torch.bfloat16).double().numpy()
+            np.testing.assert_array_equal(st[slot, h], ref)

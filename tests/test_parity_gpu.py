@@ -16,7 +16,7 @@ import torch
 import linear_attention_recurrent_decode_b200 as kda
 import oracle
 from linear_attention_recurrent_decode_b200 import workloads
-from tests.parity import check_out, check_state
+from tests.parity import check_out, check_state, check_state_bf16
 
 pytestmark = pytest.mark.gpu
 THREADS = max(1, min(32, os.cpu_count() or 1))
@@ -60,7 +60,10 @@ def assert_parity(w, o_gpu, pool_gpu, pool_before, rows=None):
         if s < 0:
             continue
         ref = st_ref[s] if rows is None else st_ref[i]
-        check_state(pool_gpu[s].cpu().numpy(), ref, what=f"state slot {s}")
+        if pool_gpu.dtype == torch.bfloat16:
+            check_state_bf16(pool_gpu[s].float().cpu().numpy(), ref, what=f"bf16 state slot {s}")
+        else:
+            check_state(pool_gpu[s].cpu().numpy(), ref, what=f"state slot {s}")
     # every slot that no active row names is bit-identical
     touched = torch.zeros(w.num_slots, dtype=torch.bool, device=pool_gpu.device)
     act = w.slot_idx[w.slot_idx >= 0].long().to(pool_gpu.device)
@@ -71,7 +74,8 @@ def assert_parity(w, o_gpu, pool_gpu, pool_before, rows=None):
         assert bool(changed.all()), "an active slot was not written"
 
 
-SMALL_CONFIGS = ["n1_t1_hv8", "n32_t1_hv8", "n32_t1_hv16_gated", "n1_t4_hv8", "n8_t4_hv8", "n32_t4_hv8"]
+SMALL_CONFIGS = ["n1_t1_hv8", "n32_t1_hv8", "n32_t1_hv16_gated", "n1_t4_hv8", "n8_t4_hv8", "n32_t4_hv8",
+                 "n32_t1_hv8_bf16state", "n32_t1_hv16_gated_bf16state", "n32_t4_hv8_bf16state"]
 
 
 @pytest.mark.parametrize("name", SMALL_CONFIGS)
@@ -81,11 +85,12 @@ def test_named_workload_parity(name, cuda_device):
     assert_parity(w, o, pool, before)
 
 
-def test_large_batch_parity_sampled(cuda_device):
-    """N=256, T=1, HV=32, 1024-slot pool (2 GiB): sampled rows against the oracle,
-    including the rows whose slots sit furthest into the pool, every other
-    slot checked bit-exact on the GPU."""
-    w = workloads.config("n256_t1_hv32")
+@pytest.mark.parametrize("name", ["n256_t1_hv32", "n256_t1_hv32_bf16state"])
+def test_large_batch_parity_sampled(name, cuda_device):
+    """N=256, T=1, HV=32, 1024-slot pool (2 GiB fp32 / 1 GiB bf16): sampled rows
+    against the oracle, including the rows whose slots sit furthest into the
+    pool, every other slot checked bit-exact on the GPU."""
+    w = workloads.config(name)
     o, pool, before = run_gpu(w, cuda_device)
     order = torch.argsort(w.slot_idx, descending=True)
     rows = sorted(set(order[:8].tolist()) | set(range(0, 256, 9)))
@@ -309,3 +314,32 @@ def test_random_shapes_against_oracle(cuda_device):
         except AssertionError as e:
             raise AssertionError(f"case {case}: N={N} T={T} HV={HV} K={K} V={V} gated={gated} "
                                  f"inactive={inactive}: {e}") from e
+
+
+BF16_CASES = [
+    # N, T, HV, K, V, gated, inactive
+    (3, 1, 3, 128, 96, False, 0),
+    (5, 2, 2, 64, 160, False, 1),
+    (2, 9, 2, 128, 128, False, 0),
+    (4, 1, 2, 256, 128, True, 1),
+    (2, 6, 2, 128, 256, True, 0),
+]
+
+
+@pytest.mark.parametrize("N,T,HV,K,V,gated,inactive", BF16_CASES)
+def test_bf16_state_shapes_parity(N, T, HV, K, V, gated, inactive, cuda_device):
+    """bf16 state pool: fp32 math, state rounded to bf16 once per call."""
+    w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=2 * N + 1, gated=gated, inactive=inactive,
+                       seed=7000 + N * 100 + T, state_dtype="bf16")
+    o, pool, before = run_gpu(w, cuda_device)
+    assert pool.dtype == torch.bfloat16
+    assert_parity(w, o, pool, before)
+
+
+def test_bf16_state_beta0_g0_is_bit_identical(cuda_device):
+    """beta = 0 and g = 0 leave a bf16 pool bit for bit (widening and rounding are exact)."""
+    w = workloads.make(N=4, T=3, HV=2, K=128, V=128, num_slots=6, seed=77, state_dtype="bf16")
+    w.beta.zero_()
+    w.g.zero_()
+    o, pool, before = run_gpu(w, cuda_device)
+    assert torch.equal(pool, before)
