@@ -15,6 +15,12 @@ Parity status of each entry point (what pins it, see ``tests/test_oracle_pins.py
   * ``kda_decode_ref`` with ``gate``/``norm_weight`` (gated RMS norm) -- pinned by
                                              closed forms (rank-1 readout, unit
                                              gate limit).
+  * ``round_bf16`` (bf16 state write-back) -- pinned by the format's definition
+                                             and torch's conversion.
+  * ``activate`` (raw gate / raw beta)  -- PARITY UNPINNED by the sources: no page
+                                             prints the activation; the code is pinned
+                                             only against library routines for the
+                                             formula it takes as its reading.
 """
 from __future__ import annotations
 
@@ -58,6 +64,9 @@ def load_library(path: str):
     r = lib.kda_oracle_round_bf16
     r.argtypes = [P, P, I]
     r.restype = None
+    a = lib.kda_oracle_activate
+    a.argtypes = [P, P, P, P, P, P, I, I, I]
+    a.restype = None
     return lib
 
 
@@ -86,6 +95,10 @@ def _as_np(x, dtype) -> np.ndarray:
     return np.ascontiguousarray(x, dtype=dtype)
 
 
+def _is_f64(x) -> bool:
+    return str(x.dtype) in ("float64", "torch.float64")
+
+
 def _ptr(a: np.ndarray | None):
     return None if a is None else a.ctypes.data
 
@@ -99,14 +112,30 @@ def round_bf16(x) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def activate(raw_gate, A_log, dt_bias, raw_beta):
+    """Gate and beta of the serving input form, in double (see
+    ``kda_oracle_activate`` in kda_oracle.c; the formula is a reading, not fixed
+    by the sources).  raw_gate bf16 [N,T,HV,K], A_log fp32 [HV], dt_bias fp32
+    [HV,K], raw_beta bf16 [N,T,HV] -> (g fp64 [N,T,HV,K], beta fp64 [N,T,HV])."""
+    rg = _as_bf16_bits(raw_gate)
+    N, T, HV, K = rg.shape
+    rb = _as_bf16_bits(raw_beta).reshape(N, T, HV)
+    al = _as_np(A_log, np.float32).reshape(HV)
+    db = _as_np(dt_bias, np.float32).reshape(HV, K)
+    g = np.empty((N, T, HV, K), np.float64)
+    beta = np.empty((N, T, HV), np.float64)
+    _load().kda_oracle_activate(_ptr(rg), _ptr(al), _ptr(db), _ptr(rb), _ptr(g), _ptr(beta), N * T, HV, K)
+    return g, beta
+
+
 def kda_decode_ref(q, k, v, g, beta, state_pool, slot_idx, scale: float,
                    gate=None, norm_weight=None, eps: float = 1e-6,
                    threads: int = 1, units: tuple[int, int] | None = None,
                    state_inplace: np.ndarray | None = None):
     """Run the oracle on one call.
 
-    q, k: bf16 [N,T,HV,K]; v: bf16 [N,T,HV,V]; g: fp32 [N,T,HV,K];
-    beta: fp32 [N,T,HV]; state_pool: fp32 or fp64 [num_slots,HV,K,V];
+    q, k: bf16 [N,T,HV,K]; v: bf16 [N,T,HV,V]; g: fp32 or fp64 [N,T,HV,K];
+    beta: fp32 or fp64 [N,T,HV]; state_pool: fp32 or fp64 [num_slots,HV,K,V];
     slot_idx: int32 [N] (negative = inactive row); gate: bf16 [N,T,HV,V] and
     norm_weight: bf16 [V] for the gated RMS-norm variant (both or neither).
 
@@ -122,8 +151,9 @@ def kda_decode_ref(q, k, v, g, beta, state_pool, slot_idx, scale: float,
     N, T, HV, K = qb.shape
     V = vb.shape[-1]
     assert kb.shape == (N, T, HV, K) and vb.shape == (N, T, HV, V)
-    gn = _as_np(g, np.float32).reshape(N, T, HV, K)
-    bn = _as_np(beta, np.float32).reshape(N, T, HV)
+    # g and beta are widened exactly to double (fp32 inputs) or taken as given (fp64)
+    gn = _as_np(g, np.float64 if _is_f64(g) else np.float32).astype(np.float64).reshape(N, T, HV, K)
+    bn = _as_np(beta, np.float64 if _is_f64(beta) else np.float32).astype(np.float64).reshape(N, T, HV)
     sn = _as_np(slot_idx, np.int32).reshape(N)
     if (gate is None) != (norm_weight is None):
         raise ValueError("gate and norm_weight go together")

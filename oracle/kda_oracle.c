@@ -68,15 +68,15 @@ static double bf16_to_double(uint16_t bits)
  * One (n, h) unit.  Arguments point at the unit's data:
  *   q, k   : bf16 rows for token t at q + t*q_tstride (K entries each)
  *   v      : bf16 rows at v + t*v_tstride (V entries)
- *   g      : fp32 log-decay rows at g + t*g_tstride (K entries)
- *   beta   : fp32 scalars at beta + t*beta_tstride
+ *   g      : log-decay rows at g + t*g_tstride (K entries)
+ *   beta   : scalars at beta + t*beta_tstride
  *   z      : bf16 gate rows (gated variant only, else NULL)
  *   w      : bf16 norm weight [V] (gated variant only, else NULL)
  *   S      : double state [K][V], row-major, updated in place (NULL = inactive)
  *   out    : double rows at out + t*out_tstride (V entries)
  */
 static void kda_oracle_unit(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                            const float *g, const float *beta, const uint16_t *z,
+                            const double *g, const double *beta, const uint16_t *z,
                             const uint16_t *w, double *S, double *out,
                             int64_t T, int64_t K, int64_t V,
                             int64_t q_tstride, int64_t v_tstride, int64_t g_tstride,
@@ -87,8 +87,8 @@ static void kda_oracle_unit(const uint16_t *q, const uint16_t *k, const uint16_t
         const uint16_t *qt = q + t * q_tstride;
         const uint16_t *kt = k + t * q_tstride;
         const uint16_t *vt = v + t * v_tstride;
-        const float *gt = g + t * g_tstride;
-        const double bt = (double)beta[t * beta_tstride];
+        const double *gt = g + t * g_tstride;
+        const double bt = beta[t * beta_tstride];
         double *ot = out + t * out_tstride;
 
         if (S == NULL) { /* inactive row */
@@ -98,7 +98,7 @@ static void kda_oracle_unit(const uint16_t *q, const uint16_t *k, const uint16_t
 
         /* 1. decay: S[i][j] *= exp(g[i]) */
         for (int64_t i = 0; i < K; ++i) {
-            const double d = exp((double)gt[i]);
+            const double d = exp(gt[i]);
             for (int64_t j = 0; j < V; ++j) S[i * V + j] *= d;
         }
         /* 2. rk = S^T k */
@@ -139,7 +139,7 @@ static void kda_oracle_unit(const uint16_t *q, const uint16_t *k, const uint16_t
  *
  * Layouts (all contiguous, row-major):
  *   q, k  bf16 bits [N, T, HV, K]      v, z  bf16 bits [N, T, HV, V]
- *   g     fp32      [N, T, HV, K]      beta  fp32      [N, T, HV]
+ *   g     double    [N, T, HV, K]      beta  double    [N, T, HV]
  *   state double    [num_slots, HV, K, V] (updated in place)
  *   slot_idx int32  [N]               out   double    [N, T, HV, V]
  *   w     bf16 bits [V]
@@ -150,7 +150,7 @@ static void kda_oracle_unit(const uint16_t *q, const uint16_t *k, const uint16_t
  * is negative.  Units of rows whose slot is negative get zero output.
  */
 int kda_oracle_decode_units(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                            const float *g, const float *beta, const uint16_t *z,
+                            const double *g, const double *beta, const uint16_t *z,
                             const uint16_t *w, double *state, int64_t num_slots,
                             const int32_t *slot_idx, double *out,
                             int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
@@ -206,4 +206,35 @@ static uint16_t double_to_bf16_rne(double x)
 void kda_oracle_round_bf16(const double *in, uint16_t *out, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16_rne(in[i]);
+}
+
+/*
+ * Gate and beta activations of the serving input form (raw bf16 gate and
+ * beta, per-head A_log, per-head per-key-channel dt_bias):
+ *   g[n,t,h,i]  = -exp(A_log[h]) * softplus(raw_gate[n,t,h,i] + dt_bias[h,i])
+ *   beta[n,t,h] = sigmoid(raw_beta[n,t,h])
+ * FlashInfer #4562's kernel launch takes raw_gate, raw_beta, A_log and
+ * dt_bias and b12x #249 takes raw_g and raw_beta, but neither page prints the
+ * activation: this formula is a reading (the usual one for KDA's gate), not
+ * something the pages fix.  softplus(x) = log(1 + e^x), evaluated as
+ * x + log1p(e^-x) for x > 0 so that it neither overflows nor cancels.
+ * Layouts: raw_gate bf16 [N*T, HV*K], raw_beta bf16 [N*T, HV] (dense),
+ * A_log [HV], dt_bias [HV*K]; outputs g [N*T, HV*K], beta [N*T, HV].
+ */
+static double softplus(double x) { return x > 0.0 ? x + log1p(exp(-x)) : log1p(exp(x)); }
+
+void kda_oracle_activate(const uint16_t *raw_gate, const float *A_log, const float *dt_bias,
+                         const uint16_t *raw_beta, double *g, double *beta, int64_t rows,
+                         int64_t HV, int64_t K)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t h = 0; h < HV; ++h) {
+            const double a = exp((double)A_log[h]);
+            for (int64_t i = 0; i < K; ++i) {
+                const int64_t e = (r * HV + h) * K + i;
+                g[e] = -a * softplus(bf16_to_double(raw_gate[e]) + (double)dt_bias[h * K + i]);
+            }
+            beta[r * HV + h] = 1.0 / (1.0 + exp(-bf16_to_double(raw_beta[r * HV + h])));
+        }
+    }
 }

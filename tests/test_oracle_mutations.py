@@ -37,7 +37,7 @@ MUTANTS = {
     "no_scale": ("ot[j] = scale * acc;", "ot[j] = acc;"),
     "readout_before_update": _swap_steps_4_and_5,
     "token_stride_q": ("const uint16_t *qt = q + t * q_tstride;", "const uint16_t *qt = q;"),
-    "token_stride_g": ("const float *gt = g + t * g_tstride;", "const float *gt = g;"),
+    "token_stride_g": ("const double *gt = g + t * g_tstride;", "const double *gt = g;"),
     "head_stride_beta": ("beta + (n * T * HV + h)", "beta + (n * T * HV)"),
     "slot_ignores_head": ("(((int64_t)slot * HV + h) * K * V)", "(((int64_t)slot * HV) * K * V)"),
     "gate_sign": ("exp(-bf16_to_double(zt[j]))", "exp(bf16_to_double(zt[j]))"),
@@ -47,6 +47,12 @@ MUTANTS = {
     "bf16_truncates": ("const double q = nearbyint(ldexp(a, -lsb));", "const double q = floor(ldexp(a, -lsb));"),
     "bf16_ties_away": ("const double q = nearbyint(ldexp(a, -lsb));", "const double q = round(ldexp(a, -lsb));"),
     "bf16_no_subnormal": ("if (lsb < -133) lsb = -133;", "if (lsb < -200) lsb = -200;"),
+    "gate_no_dt_bias": ("+ (double)dt_bias[h * K + i]", "+ 0.0 * dt_bias[h * K + i]"),
+    "gate_sign_flip": ("g[e] = -a * softplus(", "g[e] = a * softplus("),
+    "gate_exp_not_softplus": ("static double softplus(double x) { return x > 0.0 ? x + log1p(exp(-x)) : log1p(exp(x)); }",
+                              "static double softplus(double x) { return exp(x); }"),
+    "gate_a_not_exp": ("const double a = exp((double)A_log[h]);", "const double a = (double)A_log[h];"),
+    "beta_sign": ("beta[r * HV + h] = 1.0 / (1.0 + exp(-bf16_to_double(", "beta[r * HV + h] = 1.0 / (1.0 + exp(bf16_to_double("),
 }
 
 

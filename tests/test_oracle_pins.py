@@ -371,3 +371,41 @@ def test_bf16_state_closed_forms():
             exact = b[n, 0, h] * np.outer(k[n, 0, h], v[n, 0, h])
             ref = torch.from_numpy(exact).to(torch.bfloat16).double().numpy()
             np.testing.assert_array_equal(st[slot, h], ref)
+
+
+# ---------------------------------------------------------------------------
+# raw gate / raw beta activation (a reading: the sources name the inputs but
+# print no formula; pinned here only against library routines for that formula)
+# ---------------------------------------------------------------------------
+def test_activation_matches_library_routines():
+    rng = np.random.default_rng(11)
+    N, T, HV, K = 2, 3, 4, 8
+    raw_gate = bf16(rng.standard_normal((N, T, HV, K)) * 4)
+    raw_gate[0, 0, 0, :4] = bf16([80.0, -80.0, 0.0, 30.0])
+    raw_beta = bf16(rng.standard_normal((N, T, HV)) * 3)
+    A_log = torch.as_tensor(rng.standard_normal(HV), dtype=torch.float32)
+    dt_bias = torch.as_tensor(rng.standard_normal((HV, K)), dtype=torch.float32)
+    g, beta = oracle.activate(raw_gate, A_log, dt_bias, raw_beta)
+    x = bf16_vals(raw_gate) + dt_bias.double().numpy()[None, None]
+    g_ref = -np.exp(A_log.double().numpy())[None, None, :, None] * np.logaddexp(0.0, x)
+    np.testing.assert_allclose(g, g_ref, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(beta, expit(bf16_vals(raw_beta)), rtol=1e-14, atol=0)
+    assert np.all(g <= 0) and np.all(np.isfinite(g))
+
+
+def test_activation_feeds_the_recurrence():
+    """The decode from raw inputs equals the decode from the activated g, beta."""
+    w = workloads.make(N=2, T=2, HV=2, K=8, V=8, num_slots=3, seed=12)
+    rng = np.random.default_rng(12)
+    raw_gate = bf16(rng.standard_normal((2, 2, 2, 8)))
+    raw_beta = bf16(rng.standard_normal((2, 2, 2)))
+    A_log = torch.as_tensor(rng.standard_normal(2) - 1, dtype=torch.float32)
+    dt_bias = torch.as_tensor(rng.standard_normal((2, 8)), dtype=torch.float32)
+    g, beta = oracle.activate(raw_gate, A_log, dt_bias, raw_beta)
+    o1, s1 = oracle.kda_decode_ref(w.q, w.k, w.v, g, beta, w.state, w.slot_idx, w.scale)
+    # beta = 0 and g = 0 reached through the activation: raw_beta = -inf-ish, A_log -> -inf
+    g0, b0 = oracle.activate(raw_gate, torch.full((2,), -200.0), dt_bias, bf16(np.full((2, 2, 2), -200.0)))
+    assert np.all(np.abs(g0) < 1e-80) and np.all(b0 < 1e-80)
+    o0, s0 = oracle.kda_decode_ref(w.q, w.k, w.v, g0, b0, w.state, w.slot_idx, w.scale)
+    np.testing.assert_allclose(s0, w.state.double().numpy(), rtol=1e-12, atol=0)
+    assert np.all(np.isfinite(o1)) and np.all(np.isfinite(s1))
