@@ -147,6 +147,66 @@ KDA_API kda_status kda_decode_gated_rmsnorm_bf16_state(const void *q, const void
                                                        int64_t HV, int64_t K, int64_t V, float scale,
                                                        kda_stream_t stream);
 
+/* Element type of the state pool (kda_decode_args.state_dtype). */
+enum { KDA_STATE_FP32 = 0, KDA_STATE_BF16 = 1 };
+
+/*
+ * Arguments of kda_decode_ex: every operation above in one call, with row
+ * strides and the serving input form.
+ *
+ * Row strides.  Each input is a sequence of N*T rows, row (n, t) starting
+ * (n*T + t) * <x>_row_stride elements after the pointer; inside a row, head h
+ * of q, k, g and raw_gate occupies elements [h*K, (h+1)*K), of v and gate
+ * [h*V, (h+1)*V), of beta and raw_beta element h.  A stride must be at least
+ * the row's width; q, k, v, gate strides must be multiples of 8 elements, the
+ * g stride of 4, the raw_gate stride of 8.  This lets q, k and v be slices of
+ * one packed row [q | k | v] ("mixed_qkv", FlashInfer #4562's launch passes
+ * mixed_qkv.stride(0) for all three) and beta a strided column.  The
+ * dense layouts of the fixed entry points are the strides HV*K, HV*V and HV.
+ * out is always dense [N, T, HV, V].
+ *
+ * Decay and beta.  Either g (fp32 log-decay) and beta (fp32), or the serving
+ * form raw_gate (bf16) with A_log (fp32 [HV]) and dt_bias (fp32 [HV, K]), and
+ * raw_beta (bf16), activated in the kernel as
+ *     g = -exp(A_log[h]) * softplus(raw_gate + dt_bias[h, :]),  beta = sigmoid(raw_beta).
+ * FlashInfer #4562 (kernel launch) and b12x #249 (run_kda_single_token) take
+ * these raw inputs, but neither prints the activation: this formula is the
+ * usual KDA gate, taken as a reading.  g/beta and the raw inputs are
+ * exclusive (KDA_ERR_INVALID_ARG otherwise).
+ *
+ * gate and norm_weight both NULL selects the plain step, both set the gated
+ * RMS norm.  state_dtype selects an fp32 or bf16 pool.  Pointers without a
+ * use in the selected form must be NULL.  Alignment: q, k, v, g, raw_gate,
+ * dt_bias, state_pool, out, gate, norm_weight 16 bytes; beta, A_log,
+ * slot_idx 4 bytes; raw_beta 2 bytes.
+ */
+typedef struct {
+    const void *q;        int64_t q_row_stride;
+    const void *k;        int64_t k_row_stride;
+    const void *v;        int64_t v_row_stride;
+    const float *g;       int64_t g_row_stride;       /* also the raw_gate row stride */
+    const float *beta;    int64_t beta_row_stride;    /* also the raw_beta row stride */
+    const void *raw_gate;
+    const float *A_log;
+    const float *dt_bias;
+    const void *raw_beta;
+    void *state_pool;     int32_t state_dtype;
+    const int32_t *slot_idx;
+    const void *gate;     int64_t gate_row_stride;
+    const void *norm_weight;
+    float eps;
+    void *out;
+    int64_t N, T, HV, K, V;
+    float scale;
+} kda_decode_args;
+
+/*
+ * The general entry point (see kda_decode_args).  The operation, the caller
+ * contract, ownership and errors are those of kda_decode and
+ * kda_decode_gated_rmsnorm.  args is read during the call only.
+ */
+KDA_API kda_status kda_decode_ex(const kda_decode_args *args, kda_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 

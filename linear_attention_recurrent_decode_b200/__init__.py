@@ -22,7 +22,7 @@ import math
 import os
 import threading
 
-__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "KdaError", "library", "status_string",
+__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "LIBRARY_PATH", "EXPORTED_SYMBOLS"]
 
@@ -36,13 +36,39 @@ KDA_ERR_MISALIGNED = 4
 KDA_ERR_DEVICE = 5
 KDA_ERR_CUDA = 6
 
-# Every symbol include/kda_decode.h declares, with its ctypes signature.
 _P, _I, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+
+
+class DecodeArgs(ctypes.Structure):
+    """ctypes mirror of ``kda_decode_args`` (include/kda_decode.h)."""
+    _fields_ = [
+        ("q", _P), ("q_row_stride", _I),
+        ("k", _P), ("k_row_stride", _I),
+        ("v", _P), ("v_row_stride", _I),
+        ("g", _P), ("g_row_stride", _I),
+        ("beta", _P), ("beta_row_stride", _I),
+        ("raw_gate", _P), ("A_log", _P), ("dt_bias", _P), ("raw_beta", _P),
+        ("state_pool", _P), ("state_dtype", ctypes.c_int32),
+        ("slot_idx", _P),
+        ("gate", _P), ("gate_row_stride", _I),
+        ("norm_weight", _P),
+        ("eps", _F),
+        ("out", _P),
+        ("N", _I), ("T", _I), ("HV", _I), ("K", _I), ("V", _I),
+        ("scale", _F),
+    ]
+
+
+KDA_STATE_FP32 = 0
+KDA_STATE_BF16 = 1
+
+# Every symbol include/kda_decode.h declares, with its ctypes signature.
 EXPORTED_SYMBOLS = {
     "kda_decode": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_gated_rmsnorm": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_bf16_state": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_gated_rmsnorm_bf16_state": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
+    "kda_decode_ex": ([ctypes.POINTER(DecodeArgs), _P], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_abi_version": ([], ctypes.c_int32),
 }
@@ -167,4 +193,84 @@ def kda_decode_gated_rmsnorm(q, k, v, g, beta, state_pool, slot_idx, gate, norm_
         N, T, HV, K, V, float(scale), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, name)
+    return out
+
+
+def _rows(t, name, dtype, N, T, inner):
+    """Validate a [N, T, ...inner] view whose (n, t) rows are uniformly strided and
+    whose per-row part is dense; return its row stride in elements (0 for None)."""
+    import torch
+
+    if t is None:
+        return 0
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise TypeError(f"{name} must be a {dtype} tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if tuple(t.shape) != (N, T, *inner):
+        raise ValueError(f"{name} must have shape {(N, T, *inner)}, got {tuple(t.shape)}")
+    want = 1
+    for d in range(t.dim() - 1, 1, -1):  # the per-row part must be dense
+        if t.shape[d] > 1 and t.stride(d) != want:
+            raise ValueError(f"{name}: each (n, t) row must be contiguous")
+        want *= t.shape[d]
+    rs = t.stride(1) if T > 1 else t.stride(0)
+    if N > 1 and T > 1 and t.stride(0) != T * t.stride(1):
+        raise ValueError(f"{name}: (n, t) rows must be evenly strided (stride(0) == T * stride(1))")
+    return rs if (N * T) > 1 else max(rs, want)
+
+
+def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
+                  dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
+                  scale: float | None = None, stream=None):
+    """General decode step (``kda_decode_ex`` of the C ABI).
+
+    q, k [N,T,HV,K], v [N,T,HV,V] (bf16) may be strided views, e.g. slices of
+    one packed ``mixed_qkv`` row buffer; so may g / raw_gate [N,T,HV,K] and
+    beta / raw_beta [N,T,HV] and gate [N,T,HV,V].  Give either ``g`` and
+    ``beta`` (fp32) or the serving form ``raw_gate``, ``A_log`` [HV],
+    ``dt_bias`` [HV,K] (fp32) and ``raw_beta`` (bf16).  ``gate`` with
+    ``norm_weight`` selects the fused gated RMS norm.  The pool may be fp32 or
+    bf16.  Returns ``out`` (dense bf16 [N,T,HV,V])."""
+    import torch
+
+    N, T, HV, K = q.shape
+    V = v.shape[-1]
+    bf, f32 = torch.bfloat16, torch.float32
+    a = DecodeArgs()
+    a.q, a.q_row_stride = q.data_ptr(), _rows(q, "q", bf, N, T, (HV, K))
+    a.k, a.k_row_stride = k.data_ptr(), _rows(k, "k", bf, N, T, (HV, K))
+    a.v, a.v_row_stride = v.data_ptr(), _rows(v, "v", bf, N, T, (HV, V))
+    if raw_gate is not None:
+        a.raw_gate, a.g_row_stride = raw_gate.data_ptr(), _rows(raw_gate, "raw_gate", bf, N, T, (HV, K))
+        a.raw_beta, a.beta_row_stride = raw_beta.data_ptr(), _rows(raw_beta, "raw_beta", bf, N, T, (HV,))
+        _check(A_log, "A_log", f32, (HV,))
+        _check(dt_bias, "dt_bias", f32, (HV, K))
+        a.A_log, a.dt_bias = A_log.data_ptr(), dt_bias.data_ptr()
+    else:
+        a.g, a.g_row_stride = g.data_ptr(), _rows(g, "g", f32, N, T, (HV, K))
+        a.beta, a.beta_row_stride = beta.data_ptr(), _rows(beta, "beta", f32, N, T, (HV,))
+    if state_pool.dtype not in (f32, bf):
+        raise TypeError("state_pool must be float32 or bfloat16")
+    _check(state_pool, "state_pool", state_pool.dtype)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (HV, K, V):
+        raise ValueError(f"state_pool must be [num_slots, {HV}, {K}, {V}]")
+    a.state_pool = state_pool.data_ptr()
+    a.state_dtype = KDA_STATE_BF16 if state_pool.dtype == bf else KDA_STATE_FP32
+    _check(slot_idx, "slot_idx", torch.int32, (N,))
+    a.slot_idx = slot_idx.data_ptr()
+    if gate is not None:
+        a.gate, a.gate_row_stride = gate.data_ptr(), _rows(gate, "gate", bf, N, T, (HV, V))
+        _check(norm_weight, "norm_weight", bf, (V,))
+        a.norm_weight = norm_weight.data_ptr()
+    a.eps = float(eps)
+    if out is None:
+        out = torch.empty((N, T, HV, V), dtype=bf, device=q.device)
+    _check(out, "out", bf, (N, T, HV, V))
+    a.out = out.data_ptr()
+    a.N, a.T, a.HV, a.K, a.V = N, T, HV, K, V
+    a.scale = float(1.0 / math.sqrt(K) if scale is None else scale)
+    st = library().kda_decode_ex(ctypes.byref(a), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_ex")
     return out

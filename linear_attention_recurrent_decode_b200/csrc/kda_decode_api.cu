@@ -48,13 +48,19 @@ bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
 // Multiply non-negative sizes, flagging overflow of int64.
 bool mul_ok(int64_t a, int64_t b, int64_t* r) { return !__builtin_mul_overflow(a, b, r); }
 
-kda_status launch(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                  void* state_pool, const int32_t* slot_idx, const void* gate,
-                  const void* norm_weight, float eps, void* out, int64_t N, int64_t T, int64_t HV,
-                  int64_t K, int64_t V, float scale, kda_stream_t stream, bool gated, bool bf16_state) {
+// Bytes spanned by `rows` rows of `width` elements, `stride` elements apart.
+bool span_bytes(int64_t rows, int64_t stride, int64_t width, int64_t elem, int64_t* bytes) {
+  int64_t a;
+  if (!mul_ok(rows - 1, stride, &a) || __builtin_add_overflow(a, width, &a)) return false;
+  return mul_ok(a, elem, bytes);
+}
+
+kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
+  const int64_t N = a.N, T = a.T, HV = a.HV, K = a.K, V = a.V;
   // ---- sizes
   if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0) return KDA_ERR_INVALID_ARG;
-  if (gated && !(eps >= 0.0f && eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
+  if (gated && !(a.eps >= 0.0f && a.eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
+  if (a.state_dtype != KDA_STATE_FP32 && a.state_dtype != KDA_STATE_BF16) return KDA_ERR_INVALID_ARG;
   if (HV < 1) return KDA_ERR_UNSUPPORTED;
   if (K != 64 && K != 128 && K != 256) return KDA_ERR_UNSUPPORTED;
   if (V < kda::kBV || V % kda::kBV != 0) return KDA_ERR_UNSUPPORTED;
@@ -62,32 +68,62 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
   if (gated && tiles > kda::kMaxClusterTiles) return KDA_ERR_UNSUPPORTED;
   if (N == 0 || T == 0) return KDA_OK;  // nothing to do; no pointer is touched
 
-  int64_t rows, qk_elems, v_elems, grid;
-  if (!mul_ok(N, T, &rows) || !mul_ok(rows, HV, &rows) || !mul_ok(rows, K, &qk_elems) ||
-      !mul_ok(rows, V, &v_elems) || qk_elems > (INT64_MAX / 4) || v_elems > (INT64_MAX / 4))
+  int64_t rows, hk, hvv, grid, out_elems;
+  if (!mul_ok(N, T, &rows) || !mul_ok(HV, K, &hk) || !mul_ok(HV, V, &hvv) ||
+      !mul_ok(rows, hvv, &out_elems) || out_elems > (INT64_MAX / 4))
     return KDA_ERR_UNSUPPORTED;
   if (!mul_ok(N, HV, &grid) || !mul_ok(grid, tiles, &grid) || grid > 0x7fffffffLL)
     return KDA_ERR_UNSUPPORTED;
 
+  // ---- which decay and beta inputs: (g, beta) or the raw serving form
+  const bool raw = a.raw_gate != nullptr || a.raw_beta != nullptr;
+  if (raw) {
+    if (!a.raw_gate || !a.raw_beta || !a.A_log || !a.dt_bias || a.g || a.beta) return KDA_ERR_INVALID_ARG;
+  } else if (!a.g || !a.beta) {
+    return KDA_ERR_INVALID_ARG;
+  }
+
   // ---- pointers
-  if (!q || !k || !v || !g || !beta || !state_pool || !slot_idx || !out) return KDA_ERR_INVALID_ARG;
-  if (gated && (!gate || !norm_weight)) return KDA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
-      !aligned(state_pool, 16) || !aligned(out, 16) || !aligned(beta, 4) || !aligned(slot_idx, 4))
+  if (!a.q || !a.k || !a.v || !a.state_pool || !a.slot_idx || !a.out) return KDA_ERR_INVALID_ARG;
+  if (gated && (!a.gate || !a.norm_weight)) return KDA_ERR_INVALID_ARG;
+  const void* gsrc = raw ? a.raw_gate : static_cast<const void*>(a.g);
+  const void* bsrc = raw ? a.raw_beta : static_cast<const void*>(a.beta);
+  if (!aligned(a.q, 16) || !aligned(a.k, 16) || !aligned(a.v, 16) || !aligned(gsrc, 16) ||
+      !aligned(a.state_pool, 16) || !aligned(a.out, 16) || !aligned(bsrc, raw ? 2 : 4) ||
+      !aligned(a.slot_idx, 4))
     return KDA_ERR_MISALIGNED;
-  if (gated && (!aligned(gate, 16) || !aligned(norm_weight, 16))) return KDA_ERR_MISALIGNED;
+  if (raw && (!aligned(a.dt_bias, 16) || !aligned(a.A_log, 4))) return KDA_ERR_MISALIGNED;
+  if (gated && (!aligned(a.gate, 16) || !aligned(a.norm_weight, 16))) return KDA_ERR_MISALIGNED;
+
+  // ---- row strides: at least one row, and 16-byte aligned rows for the vector loads
+  const int64_t g_elem = raw ? 2 : 4;
+  if (a.q_row_stride < hk || a.k_row_stride < hk || a.v_row_stride < hvv || a.g_row_stride < hk ||
+      a.beta_row_stride < HV || (gated && a.gate_row_stride < hvv))
+    return KDA_ERR_INVALID_ARG;
+  if (a.q_row_stride % 8 || a.k_row_stride % 8 || a.v_row_stride % 8 ||
+      (a.g_row_stride * g_elem) % 16 || (gated && a.gate_row_stride % 8))
+    return KDA_ERR_MISALIGNED;
 
   // ---- aliasing: out must not overlap any input or the pool
-  const Range r_out = range_of(out, v_elems * 2);
+  int64_t bq, bk, bv, bg, bb, bz = 0;
+  if (!span_bytes(rows, a.q_row_stride, hk, 2, &bq) || !span_bytes(rows, a.k_row_stride, hk, 2, &bk) ||
+      !span_bytes(rows, a.v_row_stride, hvv, 2, &bv) ||
+      !span_bytes(rows, a.g_row_stride, hk, g_elem, &bg) ||
+      !span_bytes(rows, a.beta_row_stride, HV, raw ? 2 : 4, &bb) ||
+      (gated && !span_bytes(rows, a.gate_row_stride, hvv, 2, &bz)))
+    return KDA_ERR_UNSUPPORTED;
+  const Range r_out = range_of(a.out, out_elems * 2);
   const Range inputs[] = {
-      range_of(q, qk_elems * 2), range_of(k, qk_elems * 2), range_of(v, v_elems * 2),
-      range_of(g, qk_elems * 4), range_of(beta, rows * 4), range_of(slot_idx, N * 4),
-      range_of(gated ? gate : nullptr, gated ? v_elems * 2 : 0),
-      range_of(gated ? norm_weight : nullptr, gated ? V * 2 : 0)};
+      range_of(a.q, bq), range_of(a.k, bk), range_of(a.v, bv), range_of(gsrc, bg), range_of(bsrc, bb),
+      range_of(a.slot_idx, N * 4), range_of(gated ? a.gate : nullptr, gated ? bz : 0),
+      range_of(gated ? a.norm_weight : nullptr, gated ? V * 2 : 0),
+      range_of(raw ? a.A_log : nullptr, raw ? HV * 4 : 0),
+      range_of(raw ? a.dt_bias : nullptr, raw ? hk * 4 : 0)};
   // The pool's extent depends on slot values held on the device; the visible
   // part is slot 0 plus the base address itself.
-  const Range r_slot0 = range_of(state_pool, HV * K * V * (bf16_state ? 2 : 4));
-  const uintptr_t pool_base = reinterpret_cast<uintptr_t>(state_pool);
+  const bool bf16_state = a.state_dtype == KDA_STATE_BF16;
+  const Range r_slot0 = range_of(a.state_pool, hk * V * (bf16_state ? 2 : 4));
+  const uintptr_t pool_base = reinterpret_cast<uintptr_t>(a.state_pool);
   auto touches_pool = [&](Range r) {
     return overlaps(r, r_slot0) || (r.lo <= pool_base && pool_base < r.hi);
   };
@@ -102,22 +138,32 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
   if (dev != KDA_OK) return dev;
 
   kda::Params p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
-  p.g = g;
-  p.beta = beta;
-  p.state = state_pool;
-  p.slot_idx = slot_idx;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.gate = static_cast<const __nv_bfloat16*>(gate);
-  p.norm_weight = static_cast<const __nv_bfloat16*>(norm_weight);
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.k = static_cast<const __nv_bfloat16*>(a.k);
+  p.v = static_cast<const __nv_bfloat16*>(a.v);
+  p.g = a.g;
+  p.beta = a.beta;
+  p.state = a.state_pool;
+  p.slot_idx = a.slot_idx;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.gate = static_cast<const __nv_bfloat16*>(a.gate);
+  p.norm_weight = static_cast<const __nv_bfloat16*>(a.norm_weight);
+  p.raw_gate = static_cast<const __nv_bfloat16*>(a.raw_gate);
+  p.A_log = a.A_log;
+  p.dt_bias = a.dt_bias;
+  p.raw_beta = static_cast<const __nv_bfloat16*>(a.raw_beta);
+  p.q_rs = a.q_row_stride;
+  p.k_rs = a.k_row_stride;
+  p.v_rs = a.v_row_stride;
+  p.g_rs = a.g_row_stride;
+  p.b_rs = a.beta_row_stride;
+  p.z_rs = gated ? a.gate_row_stride : 0;
   p.T = T;
   p.HV = HV;
   p.V = V;
   p.tiles = static_cast<int32_t>(tiles);
-  p.scale = scale;
-  p.eps = eps;
+  p.scale = a.scale;
+  p.eps = a.eps;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -143,12 +189,17 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
   cudaError_t err = cudaErrorInvalidValue;
   const bool multi = T > 1;
   const bool v128 = V == 128;
-  // One instantiation per (K, V fixed at 128 or not, gated, state type); T == 1
-  // and T > 1 (chunked) kernels.
-#define KDA_LAUNCH(KERNEL, KK, VV, GG)                                                      \
-  do {                                                                                      \
-    if (bf16_state) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, __nv_bfloat16>, p); \
-    else err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, float>, p);                  \
+  // One instantiation per (K, V fixed at 128 or not, gated, state type, raw
+  // inputs); T == 1 and T > 1 (chunked) kernels.
+#define KDA_LAUNCH_ST(KERNEL, KK, VV, GG, RR)                                                         \
+  do {                                                                                                \
+    if (bf16_state) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, __nv_bfloat16, RR>, p);    \
+    else err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, float, RR>, p);                       \
+  } while (0)
+#define KDA_LAUNCH(KERNEL, KK, VV, GG)                 \
+  do {                                                 \
+    if (raw) KDA_LAUNCH_ST(KERNEL, KK, VV, GG, true);  \
+    else KDA_LAUNCH_ST(KERNEL, KK, VV, GG, false);     \
   } while (0)
 #define KDA_LAUNCH_V(KK, GG)                                                 \
   do {                                                                       \
@@ -174,7 +225,41 @@ kda_status launch(const void* q, const void* k, const void* v, const float* g, c
 #undef KDA_LAUNCH_K
 #undef KDA_LAUNCH_V
 #undef KDA_LAUNCH
+#undef KDA_LAUNCH_ST
   return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+// Dense (contiguous) arguments of the four fixed-layout entry points.
+kda_decode_args dense_args(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           void* state_pool, int32_t state_dtype, const int32_t* slot_idx, const void* gate,
+                           const void* norm_weight, float eps, void* out, int64_t N, int64_t T, int64_t HV,
+                           int64_t K, int64_t V, float scale) {
+  kda_decode_args a = {};
+  a.q = q;
+  a.q_row_stride = HV * K;
+  a.k = k;
+  a.k_row_stride = HV * K;
+  a.v = v;
+  a.v_row_stride = HV * V;
+  a.g = g;
+  a.g_row_stride = HV * K;
+  a.beta = beta;
+  a.beta_row_stride = HV;
+  a.state_pool = state_pool;
+  a.state_dtype = state_dtype;
+  a.slot_idx = slot_idx;
+  a.gate = gate;
+  a.gate_row_stride = HV * V;
+  a.norm_weight = norm_weight;
+  a.eps = eps;
+  a.out = out;
+  a.N = N;
+  a.T = T;
+  a.HV = HV;
+  a.K = K;
+  a.V = V;
+  a.scale = scale;
+  return a;
 }
 
 }  // namespace
@@ -184,8 +269,9 @@ extern "C" {
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                       float* state_pool, const int32_t* slot_idx, void* out, int64_t N, int64_t T,
                       int64_t HV, int64_t K, int64_t V, float scale, kda_stream_t stream) {
-  return launch(q, k, v, g, beta, state_pool, slot_idx, nullptr, nullptr, 0.0f, out, N, T, HV, K, V,
-                scale, stream, /*gated=*/false, /*bf16_state=*/false);
+  return launch(dense_args(q, k, v, g, beta, state_pool, KDA_STATE_FP32, slot_idx, nullptr, nullptr, 0.0f,
+                           out, N, T, HV, K, V, scale),
+                /*gated=*/false, stream);
 }
 
 kda_status kda_decode_gated_rmsnorm(const void* q, const void* k, const void* v, const float* g,
@@ -193,16 +279,18 @@ kda_status kda_decode_gated_rmsnorm(const void* q, const void* k, const void* v,
                                     const void* gate, const void* norm_weight, float eps, void* out,
                                     int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
                                     float scale, kda_stream_t stream) {
-  return launch(q, k, v, g, beta, state_pool, slot_idx, gate, norm_weight, eps, out, N, T, HV, K, V,
-                scale, stream, /*gated=*/true, /*bf16_state=*/false);
+  return launch(dense_args(q, k, v, g, beta, state_pool, KDA_STATE_FP32, slot_idx, gate, norm_weight, eps,
+                           out, N, T, HV, K, V, scale),
+                /*gated=*/true, stream);
 }
 
 kda_status kda_decode_bf16_state(const void* q, const void* k, const void* v, const float* g,
                                  const float* beta, void* state_pool, const int32_t* slot_idx, void* out,
                                  int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
                                  kda_stream_t stream) {
-  return launch(q, k, v, g, beta, state_pool, slot_idx, nullptr, nullptr, 0.0f, out, N, T, HV, K, V,
-                scale, stream, /*gated=*/false, /*bf16_state=*/true);
+  return launch(dense_args(q, k, v, g, beta, state_pool, KDA_STATE_BF16, slot_idx, nullptr, nullptr, 0.0f,
+                           out, N, T, HV, K, V, scale),
+                /*gated=*/false, stream);
 }
 
 kda_status kda_decode_gated_rmsnorm_bf16_state(const void* q, const void* k, const void* v,
@@ -211,24 +299,32 @@ kda_status kda_decode_gated_rmsnorm_bf16_state(const void* q, const void* k, con
                                                const void* norm_weight, float eps, void* out, int64_t N,
                                                int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
                                                kda_stream_t stream) {
-  return launch(q, k, v, g, beta, state_pool, slot_idx, gate, norm_weight, eps, out, N, T, HV, K, V,
-                scale, stream, /*gated=*/true, /*bf16_state=*/true);
+  return launch(dense_args(q, k, v, g, beta, state_pool, KDA_STATE_BF16, slot_idx, gate, norm_weight, eps,
+                           out, N, T, HV, K, V, scale),
+                /*gated=*/true, stream);
+}
+
+kda_status kda_decode_ex(const kda_decode_args* args, kda_stream_t stream) {
+  if (args == nullptr) return KDA_ERR_INVALID_ARG;
+  if ((args->gate == nullptr) != (args->norm_weight == nullptr)) return KDA_ERR_INVALID_ARG;
+  return launch(*args, /*gated=*/args->gate != nullptr, stream);
 }
 
 const char* kda_status_string(kda_status status) {
   switch (status) {
     case KDA_OK: return "ok";
-    case KDA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad eps)";
+    case KDA_ERR_INVALID_ARG:
+      return "invalid argument (null pointer, negative size, bad eps, short row stride or mixed input forms)";
     case KDA_ERR_UNSUPPORTED: return "unsupported size (K must be 64/128/256, V a multiple of 32, "
                                      "V <= 256 when gated, HV >= 1)";
     case KDA_ERR_ALIAS: return "output overlaps an input or the state pool";
-    case KDA_ERR_MISALIGNED: return "misaligned pointer (16 bytes for tensors, 4 for beta/slot_idx)";
+    case KDA_ERR_MISALIGNED: return "misaligned pointer or row stride";
     case KDA_ERR_DEVICE: return "current device is not compute capability 10.0 (sm_100a)";
     case KDA_ERR_CUDA: return "CUDA launch failed";
   }
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 1; }
+int32_t kda_abi_version(void) { return (1 << 16) | 2; }
 
 }  // extern "C"

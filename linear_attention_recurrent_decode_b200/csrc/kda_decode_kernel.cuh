@@ -41,6 +41,12 @@
 // memory (DSMEM) and a cluster barrier completes the RMS over V; the norm,
 // weight and sigmoid gate are applied before the bf16 store.
 //
+// Inputs may be row-strided views (q, k, v as slices of one packed buffer),
+// and the serving form takes a raw bf16 gate and beta activated in the kernel
+// (template parameter RAW): g = -exp(A_log[h]) softplus(raw_gate + dt_bias[h]),
+// beta = sigmoid(raw_beta).  The sources name these inputs but print no
+// activation; this is the usual KDA gate and is documented as a reading.
+//
 // The state pool is fp32 or bf16 (template parameter ST).  A bf16 pool is
 // widened exactly on load, all arithmetic is fp32, and the state is rounded
 // to nearest even once, when it is written back at the end of the call.
@@ -90,6 +96,16 @@ struct Params {
   __nv_bfloat16* out;
   const __nv_bfloat16* gate;         // gated variant only
   const __nv_bfloat16* norm_weight;  // gated variant only
+  // Serving input form (RAW kernels): g = -exp(A_log[h]) softplus(raw_gate + dt_bias[h]),
+  // beta = sigmoid(raw_beta).
+  const __nv_bfloat16* raw_gate;
+  const float* A_log;    // [HV]
+  const float* dt_bias;  // [HV, K]
+  const __nv_bfloat16* raw_beta;
+  // Row strides, in elements, between consecutive (n, t) rows of each input;
+  // element (n, t, h, i) of q sits at (n*T + t)*q_rs + h*K + i (v and gate with
+  // V, beta with 1).  g_rs / b_rs apply to g / beta or to raw_gate / raw_beta.
+  int64_t q_rs, k_rs, v_rs, g_rs, b_rs, z_rs;
   int64_t T;
   int64_t HV;
   int64_t V;
@@ -173,6 +189,12 @@ struct TokenIn {
   float beta;
 };
 
+// ---------------------------------------------------------------- serving-form activations
+// softplus(x) = log(1 + e^x), exact to fp32 rounding for every x (for x > 15
+// the correction log1p(e^-x) is below half an ulp of x).
+__device__ __forceinline__ float softplus_f(float x) { return x > 15.f ? x : log1pf(expf(x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+
 // ---------------------------------------------------------------- cp.async
 __device__ __forceinline__ uint32_t smem_u32(const void* ptr) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
@@ -226,31 +248,35 @@ struct alignas(16) TokenSmem {
 };
 
 // Issue cp.async copies of tokens [t0, t0 + cnt) into buf (all threads share the work).
-template <int K, bool GATED>
+template <int K, bool GATED, bool RAW>
 __device__ __forceinline__ void stage_tokens(TokenSmem<K>* buf, const Params& p, int64_t V, int64_t n,
                                              int64_t h, int64_t col0, int64_t t0, int cnt) {
   constexpr int kQ = K * 2 / 16;    // 16-byte chunks of q (and of k)
-  constexpr int kG = K * 4 / 16;    // of g
+  constexpr int kG = (RAW ? K * 2 : K * 4) / 16;  // of g (fp32) or raw_gate (bf16, into the g slot)
   constexpr int kV = kBV * 2 / 16;  // of v (and of z)
-  constexpr int kPer = 2 * kQ + kG + 2 * kV + 1;
+  constexpr int kPer = 2 * kQ + kG + 2 * kV + (RAW ? 0 : 1);  // raw beta is activated in the prep
   for (int c = threadIdx.x; c < cnt * kPer; c += kThreads) {
     const int j = c / kPer;
     int r = c - j * kPer;
-    const int64_t row = (n * p.T + t0 + j) * p.HV + h;
+    const int64_t nt = n * p.T + t0 + j;  // (n, t) row
     TokenSmem<K>& s = buf[j];
-    if (r < kQ) { cp_async16(smem_u32(s.q) + 16 * r, p.q + row * K + 8 * r); continue; }
+    if (r < kQ) { cp_async16(smem_u32(s.q) + 16 * r, p.q + nt * p.q_rs + h * K + 8 * r); continue; }
     r -= kQ;
-    if (r < kQ) { cp_async16(smem_u32(s.k) + 16 * r, p.k + row * K + 8 * r); continue; }
+    if (r < kQ) { cp_async16(smem_u32(s.k) + 16 * r, p.k + nt * p.k_rs + h * K + 8 * r); continue; }
     r -= kQ;
-    if (r < kG) { cp_async16(smem_u32(s.g) + 16 * r, p.g + row * K + 4 * r); continue; }
-    r -= kG;
-    if (r < kV) { cp_async16(smem_u32(s.v) + 16 * r, p.v + row * V + col0 + 8 * r); continue; }
-    r -= kV;
-    if (r < kV) {
-      if constexpr (GATED) cp_async16(smem_u32(s.z) + 16 * r, p.gate + row * V + col0 + 8 * r);
+    if (r < kG) {
+      if constexpr (RAW) cp_async16(smem_u32(s.g) + 16 * r, p.raw_gate + nt * p.g_rs + h * K + 8 * r);
+      else cp_async16(smem_u32(s.g) + 16 * r, p.g + nt * p.g_rs + h * K + 4 * r);
       continue;
     }
-    cp_async4(smem_u32(s.beta), p.beta + row);
+    r -= kG;
+    if (r < kV) { cp_async16(smem_u32(s.v) + 16 * r, p.v + nt * p.v_rs + h * V + col0 + 8 * r); continue; }
+    r -= kV;
+    if (r < kV) {
+      if constexpr (GATED) cp_async16(smem_u32(s.z) + 16 * r, p.gate + nt * p.z_rs + h * V + col0 + 8 * r);
+      continue;
+    }
+    cp_async4(smem_u32(s.beta), p.beta + nt * p.b_rs + h);
   }
 }
 
@@ -368,7 +394,7 @@ __device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], 
   if (writer) apply_norm(y, o, wgt, z, nrm, tiles, V, eps);
 }
 
-template <int K, int VS, bool GATED, typename ST>
+template <int K, int VS, bool GATED, typename ST, bool RAW>
 __global__ void __launch_bounds__(kThreads, (MinBlocksT1<K, VS, GATED>::value))
 kda_decode_kernel(const Params p) {
   constexpr int RPT = K / (kWarps * kRowGroups);
@@ -392,23 +418,37 @@ kda_decode_kernel(const Params p) {
   const int64_t h = unit - n * p.HV;
   const int64_t col = static_cast<int64_t>(tile) * kBV + cq * 4;
   const bool writer = (warp == 0) && (rg == 0);  // 8 lanes store the tile's 32 outputs
-  const int64_t row = n * p.HV + h;              // (n, t = 0, h)
+  const int64_t row = n * p.HV + h;              // (n, t = 0, h) of the dense output
 
   wait_prior_grids();
   const int32_t slot = __ldg(p.slot_idx + n);
 
   // Token inputs do not depend on the slot: issue them before it lands.
   TokenIn<RPT> cur;
-  ld_bf16_rows<RPT>(cur.q, p.q + row * K + r0);
-  ld_bf16_rows<RPT>(cur.k, p.k + row * K + r0);
-  ld_f32_rows<RPT>(cur.g, p.g + row * K + r0);
-  const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + row * V + col));
+  ld_bf16_rows<RPT>(cur.q, p.q + n * p.q_rs + h * K + r0);
+  ld_bf16_rows<RPT>(cur.k, p.k + n * p.k_rs + h * K + r0);
+  uint32_t graw[RPT / 2];
+  float dtb[RPT];
+  if constexpr (RAW) {
+    ld_bf16_rows<RPT>(graw, p.raw_gate + n * p.g_rs + h * K + r0);
+    ld_f32_rows<RPT>(dtb, p.dt_bias + h * K + r0);
+  } else {
+    ld_f32_rows<RPT>(cur.g, p.g + n * p.g_rs + h * K + r0);
+  }
+  const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + n * p.v_rs + h * V + col));
   cur.v[0] = vv_raw.x; cur.v[1] = vv_raw.y;
   if constexpr (GATED) {
-    const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + row * V + col));
+    const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + n * p.z_rs + h * V + col));
     cur.z[0] = zz.x; cur.z[1] = zz.y;
   }
-  cur.beta = __ldg(p.beta + row);
+  if constexpr (RAW) {
+    cur.beta = sigmoid_f(__bfloat162float(p.raw_beta[n * p.b_rs + h]));
+    const float neg_a = -expf(__ldg(p.A_log + h));
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) cur.g[i] = neg_a * softplus_f(bf16_at(graw, i) + dtb[i]);
+  } else {
+    cur.beta = __ldg(p.beta + n * p.b_rs + h);
+  }
 
   if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
     if (writer) *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(0u, 0u);
@@ -506,9 +546,15 @@ struct alignas(16) ChunkCoef {
 
 // Per-row chunk coefficients (one thread per key row) and each warp's partial
 // sums of the M/P scalars.
-template <int K>
-__device__ __forceinline__ void chunk_prep(ChunkCoef<K>& cf, float (*mp_part)[kNumMP],
-                                           const TokenSmem<K>* raw, int tc, int warp, int lane) {
+template <int K, bool RAW>
+__device__ __forceinline__ void chunk_prep(ChunkCoef<K>& cf, float (*mp_part)[kNumMP], TokenSmem<K>* raw,
+                                           int tc, int warp, int lane, const Params& p, int64_t h,
+                                           int64_t nt0) {
+  if constexpr (RAW) {  // beta of each chunk token from its raw value
+    if (threadIdx.x < tc)
+      raw[threadIdx.x].beta[0] = sigmoid_f(__bfloat162float(p.raw_beta[(nt0 + threadIdx.x) * p.b_rs + h]));
+  }
+  [[maybe_unused]] const float neg_a = RAW ? -expf(__ldg(p.A_log + h)) : 0.f;
   float mp[kNumMP];
 #pragma unroll
   for (int i = 0; i < kNumMP; ++i) mp[i] = 0.f;
@@ -517,7 +563,12 @@ __device__ __forceinline__ void chunk_prep(ChunkCoef<K>& cf, float (*mp_part)[kN
 #pragma unroll
     for (int t = 0; t < kChunk; ++t) {
       const bool live = t < tc;
-      d[t] = live ? __expf(raw[t].g[r]) : 1.f;
+      if constexpr (RAW) {
+        const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(raw[t].g);
+        d[t] = live ? __expf(neg_a * softplus_f(__bfloat162float(graw[r]) + __ldg(p.dt_bias + h * K + r))) : 1.f;
+      } else {
+        d[t] = live ? __expf(raw[t].g[r]) : 1.f;
+      }
       kk[t] = live ? __bfloat162float(raw[t].k[r]) : 0.f;
       qq[t] = live ? __bfloat162float(raw[t].q[r]) : 0.f;
     }
@@ -606,7 +657,7 @@ __device__ __forceinline__ void chunk_pass(const float2 (&s)[RPT][2], const floa
   red[warp][rg][cq] = make_float4(mine[0].x, mine[0].y, mine[1].x, mine[1].y);
 }
 
-template <int K, int VS, bool GATED, typename ST>
+template <int K, int VS, bool GATED, typename ST, bool RAW>
 __global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
 kda_decode_chunked_kernel(const Params p) {
   constexpr int RPT = K / (kWarps * kRowGroups);
@@ -642,7 +693,7 @@ kda_decode_chunked_kernel(const Params p) {
   const int32_t slot = __ldg(p.slot_idx + n);
 
   // Token inputs do not depend on the slot: stage the first chunk before it lands.
-  stage_tokens<K, GATED>(tok[0], p, V, n, h, col0, 0, static_cast<int>(p.T < kChunk ? p.T : kChunk));
+  stage_tokens<K, GATED, RAW>(tok[0], p, V, n, h, col0, 0, static_cast<int>(p.T < kChunk ? p.T : kChunk));
   cp_async_commit();
 
   if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
@@ -668,7 +719,7 @@ kda_decode_chunked_kernel(const Params p) {
     __syncthreads();  // every thread is done with the previous chunk's coefficients
     if (c0 + kChunk < p.T) {  // prefetch the next chunk into the other buffer
       const int64_t nl = p.T - c0 - kChunk;
-      stage_tokens<K, GATED>(tok[cb ^ 1], p, V, n, h, col0, c0 + kChunk,
+      stage_tokens<K, GATED, RAW>(tok[cb ^ 1], p, V, n, h, col0, c0 + kChunk,
                              static_cast<int>(nl < kChunk ? nl : kChunk));
       cp_async_commit();
       cp_async_wait<1>();
@@ -676,7 +727,7 @@ kda_decode_chunked_kernel(const Params p) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    chunk_prep<K>(cf, mp_part, tok[cb], tc, warp, lane);
+    chunk_prep<K, RAW>(cf, mp_part, tok[cb], tc, warp, lane, p, h, n * p.T + c0);
     __syncthreads();
 
     chunk_pass<RPT, K>(s, cf.kt, redR, r0, warp, lane, rg, cq);

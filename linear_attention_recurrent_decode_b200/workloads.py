@@ -158,3 +158,46 @@ CONFIGS = {
 def config(name: str, seed: int = 0) -> Workload:
     """One of the named workloads (K = V = 128), drawn with ``seed``."""
     return make(name=name, seed=seed, **CONFIGS[name])
+
+
+@dataclasses.dataclass
+class RawGate:
+    """Serving-form decay and beta inputs: raw bf16 gate and beta, per-head
+    A_log, per-head per-key-channel dt_bias."""
+    raw_gate: torch.Tensor  # bf16 [N, T, HV, K]
+    A_log: torch.Tensor     # fp32 [HV]
+    dt_bias: torch.Tensor   # fp32 [HV, K]
+    raw_beta: torch.Tensor  # bf16 [N, T, HV]
+
+    def to(self, device) -> "RawGate":
+        return RawGate(*(t.to(device) for t in (self.raw_gate, self.A_log, self.dt_bias, self.raw_beta)))
+
+
+def raw_gate_inputs(N: int, T: int, HV: int, K: int, seed: int = 0) -> RawGate:
+    """Draws in the ranges a KDA layer is initialised to: raw gate and raw beta
+    ~ N(0, 1); A_log = log U[1, 16); dt_bias = softplus^-1(dt) with
+    dt ~ U[0.001, 0.1) (so the decay rates sit mostly in (0.8, 1))."""
+    gen = torch.Generator().manual_seed(seed + 999_983)
+    raw_gate = torch.randn(N, T, HV, K, generator=gen).to(torch.bfloat16)
+    raw_beta = torch.randn(N, T, HV, generator=gen).to(torch.bfloat16)
+    A_log = torch.log(1.0 + 15.0 * torch.rand(HV, generator=gen))
+    dt = 0.001 + 0.099 * torch.rand(HV, K, generator=gen)
+    dt_bias = torch.log(torch.expm1(dt))
+    return RawGate(raw_gate, A_log.float(), dt_bias.float(), raw_beta)
+
+
+def pack_rows(parts, pad: int = 8):
+    """One buffer whose (n, t) rows hold the given [N, T, ...] tensors side by
+    side (as a packed ``mixed_qkv`` row holds q, k and v), each row padded by
+    ``pad`` elements so the row stride exceeds the row width.  Returns the
+    buffer and views of it shaped like the parts."""
+    N, T = parts[0].shape[:2]
+    widths = [p[0, 0].numel() for p in parts]
+    buf = torch.zeros(N, T, sum(widths) + pad, dtype=parts[0].dtype, device=parts[0].device)
+    views, off = [], 0
+    for p, wd in zip(parts, widths):
+        view = buf[:, :, off:off + wd].unflatten(-1, tuple(p.shape[2:]))
+        view.copy_(p)
+        views.append(view)
+        off += wd
+    return buf, views

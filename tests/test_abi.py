@@ -34,8 +34,8 @@ def declared_functions():
 
 def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
-                                    "kda_decode_gated_rmsnorm_bf16_state", "kda_status_string",
-                                    "kda_abi_version"}
+                                    "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
+                                    "kda_status_string", "kda_abi_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -55,7 +55,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 1
+    assert lib.kda_abi_version() == (1 << 16) | 2
 
 
 # ----------------------------------------------------------------- validation
@@ -140,3 +140,51 @@ def test_size_limits_are_rejected_on_the_host(lib):
     assert call(lib, N=1 << 28, HV=2, V=128) == kda.KDA_ERR_UNSUPPORTED
     # element counts that overflow int64
     assert call(lib, N=1 << 40, T=1 << 20, HV=1 << 10) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_args_struct_layout_matches_the_header(tmp_path):
+    """The ctypes mirror of kda_decode_args has the C compiler's field offsets."""
+    fields = [f for f, _ in kda.DecodeArgs._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "kda_decode.h"\nint main(void) {\n'
+                   + "".join(f'  printf("%zu\\n", offsetof(kda_decode_args, {f}));\n' for f in fields)
+                   + '  printf("%zu\\n", sizeof(kda_decode_args));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    os.system(f"gcc -std=c11 -I{os.path.dirname(HEADER)} -o {exe} {src}")
+    got = [int(x) for x in os.popen(str(exe)).read().split()]
+    want = [getattr(kda.DecodeArgs, f).offset for f in fields] + [ctypes.sizeof(kda.DecodeArgs)]
+    assert got == want
+
+
+@no_gpu
+def test_ex_entry_point_validation(lib):
+    E = kda
+    step = 1 << 30
+
+    def args(**kw):
+        a = kda.DecodeArgs()
+        N, T, HV, K, V = 2, 1, 2, 128, 128
+        a.q, a.q_row_stride = BASE, HV * K
+        a.k, a.k_row_stride = BASE + step, HV * K
+        a.v, a.v_row_stride = BASE + 2 * step, HV * V
+        a.g, a.g_row_stride = BASE + 3 * step, HV * K
+        a.beta, a.beta_row_stride = BASE + 4 * step, HV
+        a.state_pool, a.slot_idx, a.out = BASE + 5 * step, BASE + 8 * step, BASE + 9 * step
+        a.N, a.T, a.HV, a.K, a.V, a.scale = N, T, HV, K, V, 0.1
+        for key, val in kw.items():
+            setattr(a, key, val)
+        return lib.kda_decode_ex(ctypes.byref(a), None)
+
+    assert lib.kda_decode_ex(None, None) == E.KDA_ERR_INVALID_ARG
+    assert args() == E.KDA_ERR_DEVICE                                  # valid, no device here
+    assert args(q_row_stride=255) == E.KDA_ERR_INVALID_ARG             # shorter than a row
+    assert args(q_row_stride=260) == E.KDA_ERR_MISALIGNED              # not a multiple of 8
+    assert args(q_row_stride=512, T=1, N=2) == E.KDA_ERR_DEVICE        # a padded packed row
+    assert args(state_dtype=2) == E.KDA_ERR_INVALID_ARG
+    assert args(raw_gate=BASE + 10 * step) == E.KDA_ERR_INVALID_ARG    # raw gate mixed with g
+    assert args(gate=BASE + 10 * step) == E.KDA_ERR_INVALID_ARG        # gate without norm_weight
+    raw = dict(g=0, beta=0, raw_gate=BASE + 3 * step, raw_beta=BASE + 4 * step + 2,
+               A_log=BASE + 11 * step, dt_bias=BASE + 12 * step)
+    assert args(**raw) == E.KDA_ERR_DEVICE                             # raw form, 2-byte raw_beta is fine
+    assert args(**{**raw, "dt_bias": BASE + 12 * step + 4}) == E.KDA_ERR_MISALIGNED
+    assert args(**{**raw, "A_log": 0}) == E.KDA_ERR_INVALID_ARG

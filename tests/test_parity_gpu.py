@@ -7,6 +7,7 @@ outputs within 1 bf16 ulp (and 2e-3 normwise), state within 1e-5 relative,
 untouched slots bit-identical.
 """
 import ctypes
+import dataclasses
 import os
 
 import numpy as np
@@ -343,3 +344,63 @@ def test_bf16_state_beta0_g0_is_bit_identical(cuda_device):
     w.g.zero_()
     o, pool, before = run_gpu(w, cuda_device)
     assert torch.equal(pool, before)
+
+
+# ---------------------------------------------------------------------------
+# kda_decode_ex: strided / packed inputs and the raw serving form
+# ---------------------------------------------------------------------------
+def test_ex_dense_equals_fixed_entry_points(cuda_device):
+    for gated in (False, True):
+        w = workloads.make(N=5, T=3, HV=2, K=128, V=96, num_slots=7, gated=gated, seed=41)
+        d = w.to(cuda_device)
+        p1, p2 = d.state.clone(), d.state.clone()
+        extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if gated else {}
+        o1 = kda.kda_decode_ex(d.q, d.k, d.v, p1, d.slot_idx, g=d.g, beta=d.beta, **extra)
+        fn = kda.kda_decode_gated_rmsnorm if gated else kda.kda_decode
+        o2 = fn(d.q, d.k, d.v, d.g, d.beta, p2, d.slot_idx, *((d.gate, d.norm_weight) if gated else ()))
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(p1, p2)
+
+
+@pytest.mark.parametrize("T,gated,state", [(1, False, "fp32"), (1, True, "fp32"), (5, False, "fp32"),
+                                           (1, False, "bf16"), (6, True, "bf16")])
+def test_ex_packed_mixed_qkv_and_strided_gate(T, gated, state, cuda_device):
+    """q, k, v as slices of one padded packed row; g and beta as strided slices too."""
+    w = workloads.make(N=4, T=T, HV=3, K=128, V=128, num_slots=6, gated=gated, seed=43, state_dtype=state)
+    d = w.to(cuda_device)
+    _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=24)
+    _, (g, beta) = workloads.pack_rows([d.g, d.beta.unsqueeze(-1)], pad=5)  # 392 floats: 16-byte rows
+    beta = beta.squeeze(-1)
+    assert not q.is_contiguous() and q.stride(0) == T * (2 * 3 * 128 + 3 * 128 + 24)
+    before = d.state.clone()
+    extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if gated else {}
+    o = kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, g=g, beta=beta, **extra)
+    torch.cuda.synchronize()
+    assert_parity(w, o, d.state, before)
+
+
+@pytest.mark.parametrize("N,T,HV,K,V,gated,state", [
+    (4, 1, 2, 128, 128, False, "fp32"),
+    (32, 1, 8, 128, 128, False, "fp32"),
+    (3, 1, 2, 128, 128, True, "fp32"),
+    (3, 4, 2, 128, 128, False, "fp32"),
+    (2, 9, 2, 64, 96, True, "fp32"),
+    (3, 1, 2, 256, 64, False, "bf16"),
+    (2, 5, 2, 128, 128, True, "bf16"),
+])
+def test_ex_raw_gate_form(N, T, HV, K, V, gated, state, cuda_device):
+    """Raw gate / beta activated in the kernel, inputs packed like mixed_qkv;
+    against the oracle's activation feeding its recurrence."""
+    w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 3, gated=gated, seed=50 + N + T,
+                       state_dtype=state, inactive=1 if N > 2 else 0)
+    rg = workloads.raw_gate_inputs(N, T, HV, K, seed=51)
+    d, r = w.to(cuda_device), rg.to(cuda_device)
+    _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
+    before = d.state.clone()
+    extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if gated else {}
+    o = kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, raw_gate=r.raw_gate, A_log=r.A_log,
+                          dt_bias=r.dt_bias, raw_beta=r.raw_beta, **extra)
+    torch.cuda.synchronize()
+    g, beta = oracle.activate(rg.raw_gate, rg.A_log, rg.dt_bias, rg.raw_beta)
+    w_ref = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
+    assert_parity(w_ref, o, d.state, before)
