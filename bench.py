@@ -170,6 +170,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 def call_fn(kda, d, out, stream):
+    if d.raw is not None:  # serving form: q, k, v packed in one row buffer, raw gate and beta
+        from linear_attention_recurrent_decode_b200 import workloads
+
+        _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
+        extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=d.eps) if d.gated else {}
+        r = d.raw
+        return lambda: kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, raw_gate=r.raw_gate, A_log=r.A_log,
+                                         dt_bias=r.dt_bias, raw_beta=r.raw_beta, out=out, scale=d.scale,
+                                         stream=stream, **extra)
     if d.gated:
         return lambda: kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx,
                                                     d.gate, d.norm_weight, eps=d.eps, out=out,
@@ -184,6 +193,14 @@ def choose_replicas(touched_bytes: int, l2_bytes: int) -> int:
     return max(2, int(math.ceil(2 * l2_bytes / max(1, touched_bytes))) + 1)
 
 
+def _oracle_gate(oracle, w):
+    """(g, beta) for the oracle: as drawn, or activated from the serving form."""
+    if w.raw is None:
+        return w.g, w.beta
+    r = w.raw
+    return oracle.activate(r.raw_gate, r.A_log, r.dt_bias, r.raw_beta)
+
+
 def time_cpu_oracle(w, budget_s: float = 8.0, max_calls: int = 200):
     """Median wall time of the fp64 oracle on the full call, all host cores."""
     import numpy as np
@@ -196,7 +213,8 @@ def time_cpu_oracle(w, budget_s: float = 8.0, max_calls: int = 200):
     t_end = time.perf_counter() + budget_s
     while len(times) < max_calls and (len(times) < 3 or time.perf_counter() < t_end):
         t0 = time.perf_counter()
-        oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, None, w.slot_idx, w.scale,
+        g, beta = _oracle_gate(oracle, w)
+        oracle.kda_decode_ref(w.q, w.k, w.v, g, beta, None, w.slot_idx, w.scale,
                               gate=w.gate if w.gated else None,
                               norm_weight=w.norm_weight if w.gated else None, eps=w.eps,
                               threads=threads, state_inplace=pool)
@@ -402,7 +420,12 @@ def run_e2e(kda, w, dev, stream, steps, world):
 
     def step():
         dev_buf.copy_(host_buf, non_blocking=True)
-        if w.gated:
+        if w.raw is not None:
+            extra = dict(gate=devv["gate"], norm_weight=devv["norm_weight"], eps=w.eps) if w.gated else {}
+            kda.kda_decode_ex(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], raw_gate=devv["raw_gate"],
+                              A_log=devv["A_log"], dt_bias=devv["dt_bias"], raw_beta=devv["raw_beta"],
+                              scale=w.scale, out=out_d, stream=stream, **extra)
+        elif w.gated:
             kda.kda_decode_gated_rmsnorm(devv["q"], devv["k"], devv["v"], devv["g"], devv["beta"], pool,
                                          devv["slot_idx"], devv["gate"], devv["norm_weight"], eps=w.eps,
                                          scale=w.scale, out=out_d, stream=stream)
@@ -447,7 +470,8 @@ def run_reference(args):
 
     def one(lo, hi, thr):
         t0 = time.perf_counter()
-        oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, None, w.slot_idx, w.scale, threads=thr,
+        g, beta = _oracle_gate(oracle, w)
+        oracle.kda_decode_ref(w.q, w.k, w.v, g, beta, None, w.slot_idx, w.scale, threads=thr,
                               units=(lo, hi), state_inplace=pool, **kw)
         return time.perf_counter() - t0
 

@@ -427,11 +427,18 @@ kda_decode_kernel(const Params p) {
   TokenIn<RPT> cur;
   ld_bf16_rows<RPT>(cur.q, p.q + n * p.q_rs + h * K + r0);
   ld_bf16_rows<RPT>(cur.k, p.k + n * p.k_rs + h * K + r0);
-  uint32_t graw[RPT / 2];
-  float dtb[RPT];
+  // Serving form: the 8 column-quad lanes of a row group share its RPT rows,
+  // so each lane activates the rows i = cq (mod 8) and the decays travel by
+  // shuffle; otherwise every thread reads its rows' log-decays.
+  constexpr int kOwn = RPT > kColQuads ? RPT / kColQuads : 1;  // rows activated per lane
+  float graw[kOwn], dtb[kOwn];
   if constexpr (RAW) {
-    ld_bf16_rows<RPT>(graw, p.raw_gate + n * p.g_rs + h * K + r0);
-    ld_f32_rows<RPT>(dtb, p.dt_bias + h * K + r0);
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j) {
+      const int i = (cq % RPT) + j * kColQuads;
+      graw[j] = __bfloat162float(p.raw_gate[n * p.g_rs + h * K + r0 + i]);
+      dtb[j] = __ldg(p.dt_bias + h * K + r0 + i);
+    }
   } else {
     ld_f32_rows<RPT>(cur.g, p.g + n * p.g_rs + h * K + r0);
   }
@@ -444,8 +451,13 @@ kda_decode_kernel(const Params p) {
   if constexpr (RAW) {
     cur.beta = sigmoid_f(__bfloat162float(p.raw_beta[n * p.b_rs + h]));
     const float neg_a = -expf(__ldg(p.A_log + h));
+    float gown[kOwn];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) cur.g[i] = neg_a * softplus_f(bf16_at(graw, i) + dtb[i]);
+    for (int j = 0; j < kOwn; ++j) gown[j] = neg_a * softplus_f(graw[j] + dtb[j]);
+    const int base = lane & ~(kColQuads - 1);  // lane of cq = 0 in this row group
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+      cur.g[i] = __shfl_sync(0xffffffffu, gown[i / kColQuads], base + (i % kColQuads) % RPT);
   } else {
     cur.beta = __ldg(p.beta + n * p.b_rs + h);
   }

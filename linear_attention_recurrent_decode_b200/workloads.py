@@ -53,11 +53,19 @@ class Workload:
     gate: torch.Tensor | None = None
     norm_weight: torch.Tensor | None = None
     eps: float = 1e-6
+    # Serving form: raw gate / beta (then g and beta are None) and q, k, v
+    # read as slices of one packed row buffer.
+    raw: "RawGate | None" = None
 
     def tensors(self):
-        """Dict of the call's tensors (gate/norm_weight only when gated)."""
-        d = dict(q=self.q, k=self.k, v=self.v, g=self.g, beta=self.beta,
-                 state=self.state, slot_idx=self.slot_idx)
+        """Dict of the call's tensors (gate/norm_weight only when gated; the raw
+        gate inputs instead of g and beta in the serving form)."""
+        d = dict(q=self.q, k=self.k, v=self.v, state=self.state, slot_idx=self.slot_idx)
+        if self.raw is None:
+            d.update(g=self.g, beta=self.beta)
+        else:
+            d.update(raw_gate=self.raw.raw_gate, A_log=self.raw.A_log, dt_bias=self.raw.dt_bias,
+                     raw_beta=self.raw.raw_beta)
         if self.gated:
             d.update(gate=self.gate, norm_weight=self.norm_weight)
         return d
@@ -69,15 +77,16 @@ class Workload:
             if key == "state" and not state_too:
                 continue
             upd[key] = t.to(device)
-        return dataclasses.replace(self, **upd)
+        raw = None
+        if self.raw is not None:
+            raw = RawGate(*(upd.pop(k) for k in ("raw_gate", "A_log", "dt_bias", "raw_beta")))
+        return dataclasses.replace(self, raw=raw, **upd)
 
     def io_bytes(self) -> int:
         """Bytes of per-call inputs and outputs other than the state pool."""
-        n = (self.q.numel() + self.k.numel() + self.v.numel()) * 2 + self.g.numel() * 4
-        n += self.beta.numel() * 4 + self.slot_idx.numel() * 4 + self.N * self.T * self.HV * self.V * 2
-        if self.gated:
-            n += self.gate.numel() * 2 + self.norm_weight.numel() * 2
-        return n
+        t = self.tensors()
+        return sum(x.numel() * x.element_size() for key, x in t.items() if key != "state") + \
+            self.N * self.T * self.HV * self.V * 2
 
     def state_bytes_touched(self) -> int:
         """State bytes one call reads (it writes the same amount back)."""
@@ -92,7 +101,7 @@ def _bf16(x: torch.Tensor) -> torch.Tensor:
 def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | None = None,
          gated: bool = False, seed: int = 0, name: str = "custom",
          decay: str = "softplus", inactive: int = 0, state_std: float = 0.02,
-         state_dtype: str = "fp32") -> Workload:
+         state_dtype: str = "fp32", serving: bool = False) -> Workload:
     """Draw one call's inputs.
 
     ``decay``: ``"softplus"`` (g = -softplus(N(0,1))) or ``"uniform"``
@@ -132,10 +141,12 @@ def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | N
     if gated:
         gate = _bf16(randn(N, T, HV, V))
         norm_weight = _bf16(1.0 + 0.1 * randn(V))
+    raw = raw_gate_inputs(N, T, HV, K, seed=seed) if serving else None
     return Workload(name=name, N=N, T=T, HV=HV, K=K, V=V, num_slots=num_slots, gated=gated,
-                    q=_bf16(q), k=_bf16(k), v=_bf16(v), g=g.contiguous(), beta=beta.contiguous(),
+                    q=_bf16(q), k=_bf16(k), v=_bf16(v),
+                    g=None if serving else g.contiguous(), beta=None if serving else beta.contiguous(),
                     state=state.contiguous(), slot_idx=slot_idx.contiguous(),
-                    scale=1.0 / math.sqrt(K), gate=gate, norm_weight=norm_weight)
+                    scale=1.0 / math.sqrt(K), gate=gate, norm_weight=norm_weight, raw=raw)
 
 
 # The five workloads: name -> keyword arguments of ``make``.
@@ -152,6 +163,10 @@ CONFIGS = {
     "n32_t1_hv16_gated_bf16state": dict(N=32, T=1, HV=16, num_slots=128, gated=True, state_dtype="bf16"),
     "n32_t4_hv8_bf16state": dict(N=32, T=4, HV=8, num_slots=64, state_dtype="bf16"),
     "n256_t1_hv32_bf16state": dict(N=256, T=1, HV=32, num_slots=1024, decay="uniform", state_dtype="bf16"),
+    # serving input form: q, k, v packed in one row buffer, raw gate and beta activated in-kernel
+    "n32_t1_hv8_raw": dict(N=32, T=1, HV=8, num_slots=64, serving=True),
+    "n32_t1_hv16_gated_raw_bf16state": dict(N=32, T=1, HV=16, num_slots=128, gated=True, serving=True,
+                                            state_dtype="bf16"),
 }
 
 
