@@ -170,14 +170,19 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 def call_fn(kda, d, out, stream):
-    if d.raw is not None:  # serving form: q, k, v packed in one row buffer, raw gate and beta
+    if d.packed or d.raw is not None:  # q, k, v packed in one row buffer; raw or activated gate and beta
         from linear_attention_recurrent_decode_b200 import workloads
 
-        _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
+        q, k, v = d.q, d.k, d.v
+        if d.packed:
+            _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
         extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=d.eps) if d.gated else {}
-        r = d.raw
-        return lambda: kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, raw_gate=r.raw_gate, A_log=r.A_log,
-                                         dt_bias=r.dt_bias, raw_beta=r.raw_beta, out=out, scale=d.scale,
+        if d.raw is not None:
+            r = d.raw
+            extra.update(raw_gate=r.raw_gate, A_log=r.A_log, dt_bias=r.dt_bias, raw_beta=r.raw_beta)
+        else:
+            extra.update(g=d.g, beta=d.beta)
+        return lambda: kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, out=out, scale=d.scale,
                                          stream=stream, **extra)
     if d.gated:
         return lambda: kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx,
@@ -420,11 +425,15 @@ def run_e2e(kda, w, dev, stream, steps, world):
 
     def step():
         dev_buf.copy_(host_buf, non_blocking=True)
-        if w.raw is not None:
+        if w.raw is not None or w.packed:
             extra = dict(gate=devv["gate"], norm_weight=devv["norm_weight"], eps=w.eps) if w.gated else {}
-            kda.kda_decode_ex(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], raw_gate=devv["raw_gate"],
-                              A_log=devv["A_log"], dt_bias=devv["dt_bias"], raw_beta=devv["raw_beta"],
-                              scale=w.scale, out=out_d, stream=stream, **extra)
+            if w.raw is not None:
+                extra.update(raw_gate=devv["raw_gate"], A_log=devv["A_log"], dt_bias=devv["dt_bias"],
+                             raw_beta=devv["raw_beta"])
+            else:
+                extra.update(g=devv["g"], beta=devv["beta"])
+            kda.kda_decode_ex(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], scale=w.scale, out=out_d,
+                              stream=stream, **extra)
         elif w.gated:
             kda.kda_decode_gated_rmsnorm(devv["q"], devv["k"], devv["v"], devv["g"], devv["beta"], pool,
                                          devv["slot_idx"], devv["gate"], devv["norm_weight"], eps=w.eps,

@@ -137,7 +137,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
   const kda_status dev = check_device();
   if (dev != KDA_OK) return dev;
 
-  kda::Params p;
+  kda::ParamsEx p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
   p.v = static_cast<const __nv_bfloat16*>(a.v);
@@ -186,20 +186,28 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
     cfg.numAttrs = 2;
   }
 
+  // Input form: raw serving inputs; dense rows (offsets from the shape alone,
+  // whatever entry point was called); any other row strides.
+  const bool dense = a.q_row_stride == hk && a.k_row_stride == hk && a.v_row_stride == hvv &&
+                     a.g_row_stride == hk && a.beta_row_stride == HV && (!gated || a.gate_row_stride == hvv);
+  const int form = raw ? kda::kInRaw : dense ? kda::kInDense : kda::kInStrided;
+
   cudaError_t err = cudaErrorInvalidValue;
   const bool multi = T > 1;
   const bool v128 = V == 128;
-  // One instantiation per (K, V fixed at 128 or not, gated, state type, raw
-  // inputs); T == 1 and T > 1 (chunked) kernels.
+  // One instantiation per (K, V fixed at 128 or not, gated, state type, input
+  // form); T == 1 and T > 1 (chunked) kernels.
 #define KDA_LAUNCH_ST(KERNEL, KK, VV, GG, RR)                                                         \
   do {                                                                                                \
-    if (bf16_state) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, __nv_bfloat16, RR>, p);    \
-    else err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, float, RR>, p);                       \
+    const kda::ParamsOf<RR>& pf = p; /* the dense form takes the smaller block */                     \
+    if (bf16_state) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, __nv_bfloat16, RR>, pf);   \
+    else err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, float, RR>, pf);                      \
   } while (0)
-#define KDA_LAUNCH(KERNEL, KK, VV, GG)                 \
-  do {                                                 \
-    if (raw) KDA_LAUNCH_ST(KERNEL, KK, VV, GG, true);  \
-    else KDA_LAUNCH_ST(KERNEL, KK, VV, GG, false);     \
+#define KDA_LAUNCH(KERNEL, KK, VV, GG)                                             \
+  do {                                                                             \
+    if (form == kda::kInRaw) KDA_LAUNCH_ST(KERNEL, KK, VV, GG, kda::kInRaw);       \
+    else if (form == kda::kInDense) KDA_LAUNCH_ST(KERNEL, KK, VV, GG, kda::kInDense); \
+    else KDA_LAUNCH_ST(KERNEL, KK, VV, GG, kda::kInStrided);                       \
   } while (0)
 #define KDA_LAUNCH_V(KK, GG)                                                 \
   do {                                                                       \

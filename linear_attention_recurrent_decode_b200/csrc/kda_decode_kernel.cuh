@@ -43,7 +43,7 @@
 //
 // Inputs may be row-strided views (q, k, v as slices of one packed buffer),
 // and the serving form takes a raw bf16 gate and beta activated in the kernel
-// (template parameter RAW): g = -exp(A_log[h]) softplus(raw_gate + dt_bias[h]),
+// (input form kInRaw): g = -exp(A_log[h]) softplus(raw_gate + dt_bias[h]),
 // beta = sigmoid(raw_beta).  The sources name these inputs but print no
 // activation; this is the usual KDA gate and is documented as a reading.
 //
@@ -75,6 +75,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace kda {
 
 constexpr int kThreads = 128;               // 4 warps
@@ -96,7 +98,19 @@ struct Params {
   __nv_bfloat16* out;
   const __nv_bfloat16* gate;         // gated variant only
   const __nv_bfloat16* norm_weight;  // gated variant only
-  // Serving input form (RAW kernels): g = -exp(A_log[h]) softplus(raw_gate + dt_bias[h]),
+  int64_t T;
+  int64_t HV;
+  int64_t V;
+  int32_t tiles;  // V / kBV
+  float scale;
+  float eps;
+};
+
+// Row-strided views and the serving input form.  Only the kernels of those
+// forms take this larger block: the dense kernels keep the small one (a larger
+// parameter block alone measurably slowed them, through register allocation).
+struct ParamsEx : Params {
+  // Serving input form: g = -exp(A_log[h]) softplus(raw_gate + dt_bias[h]),
   // beta = sigmoid(raw_beta).
   const __nv_bfloat16* raw_gate;
   const float* A_log;    // [HV]
@@ -106,13 +120,39 @@ struct Params {
   // element (n, t, h, i) of q sits at (n*T + t)*q_rs + h*K + i (v and gate with
   // V, beta with 1).  g_rs / b_rs apply to g / beta or to raw_gate / raw_beta.
   int64_t q_rs, k_rs, v_rs, g_rs, b_rs, z_rs;
-  int64_t T;
-  int64_t HV;
-  int64_t V;
-  int32_t tiles;  // V / kBV
-  float scale;
-  float eps;
 };
+
+// How a kernel addresses its per-token inputs and which decay/beta inputs it
+// reads.  Dense inputs take their row offsets from the shape alone, so the
+// offsets of q, k, v, g, beta and out share one (n, t, h) row index.
+enum InputForm : int {
+  kInDense = 0,    // q, k, v, g, beta, gate dense [N, T, HV, ...]; activated g and beta
+  kInStrided = 1,  // row-strided views; activated g and beta
+  kInRaw = 2,      // row-strided views; raw gate and beta, activated in the kernel
+};
+template <int IN>
+using ParamsOf = typename std::conditional<IN == kInDense, Params, ParamsEx>::type;
+
+// Which input an offset is taken in (selects the row stride).
+enum InputRow : int { kRowQ, kRowK, kRowG, kRowV, kRowZ, kRowB };
+
+// Element offset of head h in (n, t) row nt of input WHICH, `width` elements
+// per head.  `row` = nt * HV + h is the dense row index, computed once by the
+// caller (recomputing it per input measurably slowed the one-token kernel).
+template <int IN, int WHICH, typename P>
+__device__ __forceinline__ int64_t in_off(const P& p, int64_t row, int64_t nt, int64_t h, int64_t width) {
+  if constexpr (IN == kInDense) {
+    return row * width;
+  } else {
+    const int64_t rs = WHICH == kRowQ   ? p.q_rs
+                       : WHICH == kRowK ? p.k_rs
+                       : WHICH == kRowG ? p.g_rs
+                       : WHICH == kRowV ? p.v_rs
+                       : WHICH == kRowZ ? p.z_rs
+                                        : p.b_rs;
+    return nt * rs + h * width;
+  }
+}
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -248,9 +288,10 @@ struct alignas(16) TokenSmem {
 };
 
 // Issue cp.async copies of tokens [t0, t0 + cnt) into buf (all threads share the work).
-template <int K, bool GATED, bool RAW>
-__device__ __forceinline__ void stage_tokens(TokenSmem<K>* buf, const Params& p, int64_t V, int64_t n,
+template <int K, bool GATED, int IN>
+__device__ __forceinline__ void stage_tokens(TokenSmem<K>* buf, const ParamsOf<IN>& p, int64_t V, int64_t n,
                                              int64_t h, int64_t col0, int64_t t0, int cnt) {
+  constexpr bool RAW = IN == kInRaw;
   constexpr int kQ = K * 2 / 16;    // 16-byte chunks of q (and of k)
   constexpr int kG = (RAW ? K * 2 : K * 4) / 16;  // of g (fp32) or raw_gate (bf16, into the g slot)
   constexpr int kV = kBV * 2 / 16;  // of v (and of z)
@@ -259,24 +300,25 @@ __device__ __forceinline__ void stage_tokens(TokenSmem<K>* buf, const Params& p,
     const int j = c / kPer;
     int r = c - j * kPer;
     const int64_t nt = n * p.T + t0 + j;  // (n, t) row
+    const int64_t row = nt * p.HV + h;    // its dense (n, t, h) row
     TokenSmem<K>& s = buf[j];
-    if (r < kQ) { cp_async16(smem_u32(s.q) + 16 * r, p.q + nt * p.q_rs + h * K + 8 * r); continue; }
+    if (r < kQ) { cp_async16(smem_u32(s.q) + 16 * r, p.q + in_off<IN, kRowQ>(p, row, nt, h, K) + 8 * r); continue; }
     r -= kQ;
-    if (r < kQ) { cp_async16(smem_u32(s.k) + 16 * r, p.k + nt * p.k_rs + h * K + 8 * r); continue; }
+    if (r < kQ) { cp_async16(smem_u32(s.k) + 16 * r, p.k + in_off<IN, kRowK>(p, row, nt, h, K) + 8 * r); continue; }
     r -= kQ;
     if (r < kG) {
-      if constexpr (RAW) cp_async16(smem_u32(s.g) + 16 * r, p.raw_gate + nt * p.g_rs + h * K + 8 * r);
-      else cp_async16(smem_u32(s.g) + 16 * r, p.g + nt * p.g_rs + h * K + 4 * r);
+      if constexpr (RAW) cp_async16(smem_u32(s.g) + 16 * r, p.raw_gate + in_off<IN, kRowG>(p, row, nt, h, K) + 8 * r);
+      else cp_async16(smem_u32(s.g) + 16 * r, p.g + in_off<IN, kRowG>(p, row, nt, h, K) + 4 * r);
       continue;
     }
     r -= kG;
-    if (r < kV) { cp_async16(smem_u32(s.v) + 16 * r, p.v + nt * p.v_rs + h * V + col0 + 8 * r); continue; }
+    if (r < kV) { cp_async16(smem_u32(s.v) + 16 * r, p.v + in_off<IN, kRowV>(p, row, nt, h, V) + col0 + 8 * r); continue; }
     r -= kV;
     if (r < kV) {
-      if constexpr (GATED) cp_async16(smem_u32(s.z) + 16 * r, p.gate + nt * p.z_rs + h * V + col0 + 8 * r);
+      if constexpr (GATED) cp_async16(smem_u32(s.z) + 16 * r, p.gate + in_off<IN, kRowZ>(p, row, nt, h, V) + col0 + 8 * r);
       continue;
     }
-    cp_async4(smem_u32(s.beta), p.beta + nt * p.b_rs + h);
+    cp_async4(smem_u32(s.beta), p.beta + in_off<IN, kRowB>(p, row, nt, h, 1));
   }
 }
 
@@ -394,9 +436,10 @@ __device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], 
   if (writer) apply_norm(y, o, wgt, z, nrm, tiles, V, eps);
 }
 
-template <int K, int VS, bool GATED, typename ST, bool RAW>
+template <int K, int VS, bool GATED, typename ST, int IN>
 __global__ void __launch_bounds__(kThreads, (MinBlocksT1<K, VS, GATED>::value))
-kda_decode_kernel(const Params p) {
+kda_decode_kernel(const ParamsOf<IN> p) {
+  constexpr bool RAW = IN == kInRaw;
   constexpr int RPT = K / (kWarps * kRowGroups);
   static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
 
@@ -425,8 +468,8 @@ kda_decode_kernel(const Params p) {
 
   // Token inputs do not depend on the slot: issue them before it lands.
   TokenIn<RPT> cur;
-  ld_bf16_rows<RPT>(cur.q, p.q + n * p.q_rs + h * K + r0);
-  ld_bf16_rows<RPT>(cur.k, p.k + n * p.k_rs + h * K + r0);
+  ld_bf16_rows<RPT>(cur.q, p.q + in_off<IN, kRowQ>(p, row, n, h, K) + r0);
+  ld_bf16_rows<RPT>(cur.k, p.k + in_off<IN, kRowK>(p, row, n, h, K) + r0);
   // Serving form: the 8 column-quad lanes of a row group share its RPT rows,
   // so each lane activates the rows i = cq (mod 8) and the decays travel by
   // shuffle; otherwise every thread reads its rows' log-decays.
@@ -436,20 +479,20 @@ kda_decode_kernel(const Params p) {
 #pragma unroll
     for (int j = 0; j < kOwn; ++j) {
       const int i = (cq % RPT) + j * kColQuads;
-      graw[j] = __bfloat162float(p.raw_gate[n * p.g_rs + h * K + r0 + i]);
+      graw[j] = __bfloat162float(p.raw_gate[in_off<IN, kRowG>(p, row, n, h, K) + r0 + i]);
       dtb[j] = __ldg(p.dt_bias + h * K + r0 + i);
     }
   } else {
-    ld_f32_rows<RPT>(cur.g, p.g + n * p.g_rs + h * K + r0);
+    ld_f32_rows<RPT>(cur.g, p.g + in_off<IN, kRowG>(p, row, n, h, K) + r0);
   }
-  const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + n * p.v_rs + h * V + col));
+  const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + in_off<IN, kRowV>(p, row, n, h, V) + col));
   cur.v[0] = vv_raw.x; cur.v[1] = vv_raw.y;
   if constexpr (GATED) {
-    const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + n * p.z_rs + h * V + col));
+    const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + col));
     cur.z[0] = zz.x; cur.z[1] = zz.y;
   }
   if constexpr (RAW) {
-    cur.beta = sigmoid_f(__bfloat162float(p.raw_beta[n * p.b_rs + h]));
+    cur.beta = sigmoid_f(__bfloat162float(p.raw_beta[in_off<IN, kRowB>(p, row, n, h, 1)]));
     const float neg_a = -expf(__ldg(p.A_log + h));
     float gown[kOwn];
 #pragma unroll
@@ -459,7 +502,7 @@ kda_decode_kernel(const Params p) {
     for (int i = 0; i < RPT; ++i)
       cur.g[i] = __shfl_sync(0xffffffffu, gown[i / kColQuads], base + (i % kColQuads) % RPT);
   } else {
-    cur.beta = __ldg(p.beta + n * p.b_rs + h);
+    cur.beta = __ldg(p.beta + in_off<IN, kRowB>(p, row, n, h, 1));
   }
 
   if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
@@ -558,26 +601,35 @@ struct alignas(16) ChunkCoef {
 
 // Per-row chunk coefficients (one thread per key row) and each warp's partial
 // sums of the M/P scalars.
+//
+// Serving form: the caller passes neg_a = -exp(A_log[h]), this thread's rows'
+// dt_bias (rows threadIdx.x + j * kThreads) and the raw beta of chunk token
+// threadIdx.x, all loaded into registers ahead of time (a global load here
+// would wait behind the state loads).
+__host__ __device__ constexpr int rows_per_thread(int K) { return (K + kThreads - 1) / kThreads; }
+
 template <int K, bool RAW>
 __device__ __forceinline__ void chunk_prep(ChunkCoef<K>& cf, float (*mp_part)[kNumMP], TokenSmem<K>* raw,
-                                           int tc, int warp, int lane, const Params& p, int64_t h,
-                                           int64_t nt0) {
+                                           int tc, int warp, int lane, float neg_a,
+                                           const float (&dt_bias)[rows_per_thread(K)], float raw_beta) {
   if constexpr (RAW) {  // beta of each chunk token from its raw value
-    if (threadIdx.x < tc)
-      raw[threadIdx.x].beta[0] = sigmoid_f(__bfloat162float(p.raw_beta[(nt0 + threadIdx.x) * p.b_rs + h]));
+    if (threadIdx.x < tc) raw[threadIdx.x].beta[0] = sigmoid_f(raw_beta);
   }
-  [[maybe_unused]] const float neg_a = RAW ? -expf(__ldg(p.A_log + h)) : 0.f;
   float mp[kNumMP];
 #pragma unroll
   for (int i = 0; i < kNumMP; ++i) mp[i] = 0.f;
-  for (int r = threadIdx.x; r < K; r += kThreads) {
+#pragma unroll
+  for (int jr = 0; jr < rows_per_thread(K); ++jr) {
+    const int r = threadIdx.x + jr * kThreads;
+    if (K % kThreads != 0 && r >= K) break;
     float d[kChunk], kk[kChunk], qq[kChunk];
+    [[maybe_unused]] const float dtb = dt_bias[jr];
 #pragma unroll
     for (int t = 0; t < kChunk; ++t) {
       const bool live = t < tc;
       if constexpr (RAW) {
         const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(raw[t].g);
-        d[t] = live ? __expf(neg_a * softplus_f(__bfloat162float(graw[r]) + __ldg(p.dt_bias + h * K + r))) : 1.f;
+        d[t] = live ? __expf(neg_a * softplus_f(__bfloat162float(graw[r]) + dtb)) : 1.f;
       } else {
         d[t] = live ? __expf(raw[t].g[r]) : 1.f;
       }
@@ -669,9 +721,10 @@ __device__ __forceinline__ void chunk_pass(const float2 (&s)[RPT][2], const floa
   red[warp][rg][cq] = make_float4(mine[0].x, mine[0].y, mine[1].x, mine[1].y);
 }
 
-template <int K, int VS, bool GATED, typename ST, bool RAW>
+template <int K, int VS, bool GATED, typename ST, int IN>
 __global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
-kda_decode_chunked_kernel(const Params p) {
+kda_decode_chunked_kernel(const ParamsOf<IN> p) {
+  constexpr bool RAW = IN == kInRaw;
   constexpr int RPT = K / (kWarps * kRowGroups);
   static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
   static_assert(kChunk == 4 && kRowGroups == kChunk, "one row group per chunk token in the reduce-scatter");
@@ -705,8 +758,24 @@ kda_decode_chunked_kernel(const Params p) {
   const int32_t slot = __ldg(p.slot_idx + n);
 
   // Token inputs do not depend on the slot: stage the first chunk before it lands.
-  stage_tokens<K, GATED, RAW>(tok[0], p, V, n, h, col0, 0, static_cast<int>(p.T < kChunk ? p.T : kChunk));
+  stage_tokens<K, GATED, IN>(tok[0], p, V, n, h, col0, 0, static_cast<int>(p.T < kChunk ? p.T : kChunk));
   cp_async_commit();
+  // Serving-form scalars and the norm weight, also ahead of the state loads.
+  [[maybe_unused]] float neg_a = 0.f, raw_beta = 0.f, dt_bias[rows_per_thread(K)];
+  if constexpr (RAW) {
+    neg_a = -expf(__ldg(p.A_log + h));
+#pragma unroll
+    for (int jr = 0; jr < rows_per_thread(K); ++jr) {
+      const int r = threadIdx.x + jr * kThreads;
+      dt_bias[jr] = r < K ? __ldg(p.dt_bias + h * K + r) : 0.f;
+    }
+    if (threadIdx.x < p.T && threadIdx.x < kChunk)
+      raw_beta = __bfloat162float(p.raw_beta[(n * p.T + threadIdx.x) * p.b_rs + h]);
+  }
+  [[maybe_unused]] float wj = 0.f;  // gated: norm weight of this lane's solve column (warp 0)
+  if constexpr (GATED) {
+    if (warp == 0) wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + rg]);
+  }
 
   if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
     cp_async_wait<0>();
@@ -731,7 +800,7 @@ kda_decode_chunked_kernel(const Params p) {
     __syncthreads();  // every thread is done with the previous chunk's coefficients
     if (c0 + kChunk < p.T) {  // prefetch the next chunk into the other buffer
       const int64_t nl = p.T - c0 - kChunk;
-      stage_tokens<K, GATED, RAW>(tok[cb ^ 1], p, V, n, h, col0, c0 + kChunk,
+      stage_tokens<K, GATED, IN>(tok[cb ^ 1], p, V, n, h, col0, c0 + kChunk,
                              static_cast<int>(nl < kChunk ? nl : kChunk));
       cp_async_commit();
       cp_async_wait<1>();
@@ -739,7 +808,11 @@ kda_decode_chunked_kernel(const Params p) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    chunk_prep<K, RAW>(cf, mp_part, tok[cb], tc, warp, lane, p, h, n * p.T + c0);
+    chunk_prep<K, RAW>(cf, mp_part, tok[cb], tc, warp, lane, neg_a, dt_bias, raw_beta);
+    if constexpr (RAW) {  // the next chunk's raw beta, consumed by the next prep
+      const int64_t tn = c0 + kChunk + threadIdx.x;
+      if (threadIdx.x < kChunk && tn < p.T) raw_beta = __bfloat162float(p.raw_beta[(n * p.T + tn) * p.b_rs + h]);
+    }
     __syncthreads();
 
     chunk_pass<RPT, K>(s, cf.kt, redR, r0, warp, lane, rg, cq);
@@ -829,7 +902,6 @@ kda_decode_chunked_kernel(const Params p) {
       cluster_arrive_release();
       cluster_wait_acquire();
       if (warp == 0) {
-        const float wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + jc]);
 #pragma unroll
         for (int t = 0; t < kChunk; ++t) {
           if (t < tc) {

@@ -53,9 +53,10 @@ class Workload:
     gate: torch.Tensor | None = None
     norm_weight: torch.Tensor | None = None
     eps: float = 1e-6
-    # Serving form: raw gate / beta (then g and beta are None) and q, k, v
-    # read as slices of one packed row buffer.
+    # Serving form: raw gate / beta (then g and beta are None).
     raw: "RawGate | None" = None
+    # q, k, v read as slices of one packed row buffer (the serving form does).
+    packed: bool = False
 
     def tensors(self):
         """Dict of the call's tensors (gate/norm_weight only when gated; the raw
@@ -101,12 +102,14 @@ def _bf16(x: torch.Tensor) -> torch.Tensor:
 def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | None = None,
          gated: bool = False, seed: int = 0, name: str = "custom",
          decay: str = "softplus", inactive: int = 0, state_std: float = 0.02,
-         state_dtype: str = "fp32", serving: bool = False) -> Workload:
+         state_dtype: str = "fp32", serving: bool = False, packed: bool | None = None) -> Workload:
     """Draw one call's inputs.
 
     ``decay``: ``"softplus"`` (g = -softplus(N(0,1))) or ``"uniform"``
     (exp(g) ~ U[0.5, 1)).  ``inactive``: how many rows (the last ones) get a
-    negative slot index, as CUDA-graph padding rows do.
+    negative slot index, as CUDA-graph padding rows do.  ``serving``: raw gate
+    and beta inputs instead of g and beta.  ``packed``: q, k, v to be passed as
+    slices of one packed row buffer (default: as ``serving``).
     """
     gen = torch.Generator().manual_seed(seed)
     if num_slots is None:
@@ -146,7 +149,8 @@ def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | N
                     q=_bf16(q), k=_bf16(k), v=_bf16(v),
                     g=None if serving else g.contiguous(), beta=None if serving else beta.contiguous(),
                     state=state.contiguous(), slot_idx=slot_idx.contiguous(),
-                    scale=1.0 / math.sqrt(K), gate=gate, norm_weight=norm_weight, raw=raw)
+                    scale=1.0 / math.sqrt(K), gate=gate, norm_weight=norm_weight, raw=raw,
+                    packed=serving if packed is None else packed)
 
 
 # The five workloads: name -> keyword arguments of ``make``.
@@ -167,6 +171,10 @@ CONFIGS = {
     "n32_t1_hv8_raw": dict(N=32, T=1, HV=8, num_slots=64, serving=True),
     "n32_t1_hv16_gated_raw_bf16state": dict(N=32, T=1, HV=16, num_slots=128, gated=True, serving=True,
                                             state_dtype="bf16"),
+    "n32_t4_hv8_raw": dict(N=32, T=4, HV=8, num_slots=64, serving=True),
+    # q, k, v packed in one row buffer, activated g and beta (row-strided kernels)
+    "n32_t1_hv8_packed": dict(N=32, T=1, HV=8, num_slots=64, packed=True),
+    "n32_t4_hv8_packed": dict(N=32, T=4, HV=8, num_slots=64, packed=True),
 }
 
 

@@ -404,3 +404,49 @@ def test_ex_raw_gate_form(N, T, HV, K, V, gated, state, cuda_device):
     g, beta = oracle.activate(rg.raw_gate, rg.A_log, rg.dt_bias, rg.raw_beta)
     w_ref = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
     assert_parity(w_ref, o, d.state, before)
+
+
+SERVING_CONFIGS = [n for n in workloads.CONFIGS if "_raw" in n or "_packed" in n]
+
+
+@pytest.mark.parametrize("name", SERVING_CONFIGS)
+def test_named_serving_workload_parity(name, cuda_device):
+    """The packed and serving-form workloads, called as the benchmark calls them
+    (q, k, v packed in one row buffer; raw gate and beta, or activated ones)."""
+    w = workloads.config(name)
+    d = w.to(cuda_device)
+    _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
+    before = d.state.clone()
+    extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if w.gated else {}
+    if w.raw is not None:
+        extra.update(raw_gate=d.raw.raw_gate, A_log=d.raw.A_log, dt_bias=d.raw.dt_bias, raw_beta=d.raw.raw_beta)
+    else:
+        extra.update(g=d.g, beta=d.beta)
+    o = kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, scale=w.scale, **extra)
+    torch.cuda.synchronize()
+    if w.raw is not None:
+        g, beta = oracle.activate(w.raw.raw_gate, w.raw.A_log, w.raw.dt_bias, w.raw.raw_beta)
+        w = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
+    assert_parity(w, o, d.state, before)
+
+
+@pytest.mark.parametrize("T,gated,state", [(1, False, "fp32"), (1, True, "bf16"), (4, False, "fp32"),
+                                           (7, True, "fp32")])
+def test_strided_form_bit_identical_to_dense(T, gated, state, cuda_device):
+    """The strided-input kernels differ from the dense ones only in addressing:
+    the same values laid out in packed rows give bit-identical outputs and state."""
+    w = workloads.make(N=6, T=T, HV=4, K=128, V=128, num_slots=9, gated=gated, seed=60 + T,
+                       state_dtype=state, inactive=1)
+    d = w.to(cuda_device)
+    p_dense, p_strided = d.state.clone(), d.state.clone()
+    extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if gated else {}
+    o_dense = kda.kda_decode_ex(d.q, d.k, d.v, p_dense, d.slot_idx, g=d.g, beta=d.beta, **extra)
+    _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=16)
+    _, (g, beta) = workloads.pack_rows([d.g, d.beta.unsqueeze(-1)], pad=4)  # 520 floats: 16-byte rows
+    if gated:
+        _, (z,) = workloads.pack_rows([d.gate], pad=8)
+        extra["gate"] = z
+    o_strided = kda.kda_decode_ex(q, k, v, p_strided, d.slot_idx, g=g, beta=beta.squeeze(-1), **extra)
+    torch.cuda.synchronize()
+    assert torch.equal(o_dense, o_strided)
+    assert torch.equal(p_dense, p_strided)
