@@ -170,7 +170,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 def call_fn(kda, d, out, stream):
-    if d.packed or d.raw is not None:  # q, k, v packed in one row buffer; raw or activated gate and beta
+    if d.packed or d.raw is not None or d.state_layout != "kv":  # the general entry point
         from linear_attention_recurrent_decode_b200 import workloads
 
         q, k, v = d.q, d.k, d.v
@@ -183,7 +183,7 @@ def call_fn(kda, d, out, stream):
         else:
             extra.update(g=d.g, beta=d.beta)
         return lambda: kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, out=out, scale=d.scale,
-                                         stream=stream, **extra)
+                                         stream=stream, state_layout=d.state_layout, **extra)
     if d.gated:
         return lambda: kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx,
                                                     d.gate, d.norm_weight, eps=d.eps, out=out,
@@ -213,7 +213,7 @@ def time_cpu_oracle(w, budget_s: float = 8.0, max_calls: int = 200):
     import oracle
 
     threads = os.cpu_count() or 1
-    pool = w.state.double().numpy().copy()
+    pool = w.state_kv().double().numpy().copy()
     times = []
     t_end = time.perf_counter() + budget_s
     while len(times) < max_calls and (len(times) < 3 or time.perf_counter() < t_end):
@@ -425,7 +425,7 @@ def run_e2e(kda, w, dev, stream, steps, world):
 
     def step():
         dev_buf.copy_(host_buf, non_blocking=True)
-        if w.raw is not None or w.packed:
+        if w.raw is not None or w.packed or w.state_layout != "kv":
             extra = dict(gate=devv["gate"], norm_weight=devv["norm_weight"], eps=w.eps) if w.gated else {}
             if w.raw is not None:
                 extra.update(raw_gate=devv["raw_gate"], A_log=devv["A_log"], dt_bias=devv["dt_bias"],
@@ -433,7 +433,7 @@ def run_e2e(kda, w, dev, stream, steps, world):
             else:
                 extra.update(g=devv["g"], beta=devv["beta"])
             kda.kda_decode_ex(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], scale=w.scale, out=out_d,
-                              stream=stream, **extra)
+                              stream=stream, state_layout=w.state_layout, **extra)
         elif w.gated:
             kda.kda_decode_gated_rmsnorm(devv["q"], devv["k"], devv["v"], devv["g"], devv["beta"], pool,
                                          devv["slot_idx"], devv["gate"], devv["norm_weight"], eps=w.eps,
@@ -474,7 +474,7 @@ def run_reference(args):
     w = workloads.config(args.config)
     units = w.N * w.HV
     threads = os.cpu_count() or 1
-    pool = w.state.double().numpy().copy()
+    pool = w.state_kv().double().numpy().copy()
     kw = dict(gate=w.gate, norm_weight=w.norm_weight, eps=w.eps) if w.gated else dict(eps=w.eps)
 
     def one(lo, hi, thr):

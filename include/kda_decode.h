@@ -39,7 +39,8 @@
  *     g           fp32  [N, T, HV, K]     log-decay, decay = exp(g)
  *     beta        fp32  [N, T, HV]
  *     state_pool  fp32  [num_slots, HV, K, V], read and written in place
- *                 (bf16 for the *_bf16_state entry points)
+ *                 (bf16 for the *_bf16_state entry points; kda_decode_ex
+ *                 also takes [num_slots, HV, V, K] blocks, see below)
  *     slot_idx    int32 [N]               slot of each row; < 0 = inactive row
  *     out         bf16  [N, T, HV, V]
  *     gate (z)    bf16  [N, T, HV, V]     gated variant only
@@ -151,6 +152,16 @@ KDA_API kda_status kda_decode_gated_rmsnorm_bf16_state(const void *q, const void
 enum { KDA_STATE_FP32 = 0, KDA_STATE_BF16 = 1 };
 
 /*
+ * Layout of each (slot, head) state block (kda_decode_args.state_layout):
+ * KDA_LAYOUT_KV = [K][V] (value index fastest; the layout of the fixed entry
+ * points), KDA_LAYOUT_VK = [V][K] (key index fastest: each value column's K
+ * entries are contiguous, the layout FlashInfer #4562's kernels keep their
+ * recurrent state in).  The pool is [num_slots, HV, K, V] or
+ * [num_slots, HV, V, K] respectively; the operation is the same.
+ */
+enum { KDA_LAYOUT_KV = 0, KDA_LAYOUT_VK = 1 };
+
+/*
  * Arguments of kda_decode_ex: every operation above in one call, with row
  * strides and the serving input form.
  *
@@ -175,7 +186,9 @@ enum { KDA_STATE_FP32 = 0, KDA_STATE_BF16 = 1 };
  * exclusive (KDA_ERR_INVALID_ARG otherwise).
  *
  * gate and norm_weight both NULL selects the plain step, both set the gated
- * RMS norm.  state_dtype selects an fp32 or bf16 pool.  Pointers without a
+ * RMS norm.  state_dtype selects an fp32 or bf16 pool, state_layout its
+ * block layout (KDA_LAYOUT_KV or KDA_LAYOUT_VK; anything else is
+ * KDA_ERR_INVALID_ARG).  Pointers without a
  * use in the selected form must be NULL.  Alignment: q, k, v, g, raw_gate,
  * dt_bias, state_pool, out, gate, norm_weight 16 bytes; beta, A_log,
  * slot_idx 4 bytes; raw_beta 2 bytes.
@@ -190,7 +203,7 @@ typedef struct {
     const float *A_log;
     const float *dt_bias;
     const void *raw_beta;
-    void *state_pool;     int32_t state_dtype;
+    void *state_pool;     int32_t state_dtype;        int32_t state_layout;
     const int32_t *slot_idx;
     const void *gate;     int64_t gate_row_stride;
     const void *norm_weight;

@@ -24,7 +24,8 @@ import threading
 
 __all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
-           "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "LIBRARY_PATH", "EXPORTED_SYMBOLS"]
+           "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_STATE_FP32", "KDA_STATE_BF16",
+           "KDA_LAYOUT_KV", "KDA_LAYOUT_VK", "LIBRARY_PATH", "EXPORTED_SYMBOLS"]
 
 LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda_decode.so")
 
@@ -48,7 +49,7 @@ class DecodeArgs(ctypes.Structure):
         ("g", _P), ("g_row_stride", _I),
         ("beta", _P), ("beta_row_stride", _I),
         ("raw_gate", _P), ("A_log", _P), ("dt_bias", _P), ("raw_beta", _P),
-        ("state_pool", _P), ("state_dtype", ctypes.c_int32),
+        ("state_pool", _P), ("state_dtype", ctypes.c_int32), ("state_layout", ctypes.c_int32),
         ("slot_idx", _P),
         ("gate", _P), ("gate_row_stride", _I),
         ("norm_weight", _P),
@@ -61,6 +62,8 @@ class DecodeArgs(ctypes.Structure):
 
 KDA_STATE_FP32 = 0
 KDA_STATE_BF16 = 1
+KDA_LAYOUT_KV = 0
+KDA_LAYOUT_VK = 1
 
 # Every symbol include/kda_decode.h declares, with its ctypes signature.
 EXPORTED_SYMBOLS = {
@@ -222,7 +225,7 @@ def _rows(t, name, dtype, N, T, inner):
 
 def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
                   dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
-                  scale: float | None = None, stream=None):
+                  scale: float | None = None, stream=None, state_layout: str = "kv"):
     """General decode step (``kda_decode_ex`` of the C ABI).
 
     q, k [N,T,HV,K], v [N,T,HV,V] (bf16) may be strided views, e.g. slices of
@@ -231,7 +234,9 @@ def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=
     ``beta`` (fp32) or the serving form ``raw_gate``, ``A_log`` [HV],
     ``dt_bias`` [HV,K] (fp32) and ``raw_beta`` (bf16).  ``gate`` with
     ``norm_weight`` selects the fused gated RMS norm.  The pool may be fp32 or
-    bf16.  Returns ``out`` (dense bf16 [N,T,HV,V])."""
+    bf16, with blocks [K, V] (``state_layout="kv"``: pool [num_slots,HV,K,V])
+    or [V, K] (``"vk"``: pool [num_slots,HV,V,K], key index fastest).
+    Returns ``out`` (dense bf16 [N,T,HV,V])."""
     import torch
 
     N, T, HV, K = q.shape
@@ -253,9 +258,13 @@ def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=
     if state_pool.dtype not in (f32, bf):
         raise TypeError("state_pool must be float32 or bfloat16")
     _check(state_pool, "state_pool", state_pool.dtype)
-    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (HV, K, V):
-        raise ValueError(f"state_pool must be [num_slots, {HV}, {K}, {V}]")
+    if state_layout not in ("kv", "vk"):
+        raise ValueError("state_layout must be 'kv' or 'vk'")
+    block = (K, V) if state_layout == "kv" else (V, K)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (HV, *block):
+        raise ValueError(f"state_pool must be [num_slots, {HV}, {block[0]}, {block[1]}]")
     a.state_pool = state_pool.data_ptr()
+    a.state_layout = KDA_LAYOUT_KV if state_layout == "kv" else KDA_LAYOUT_VK
     a.state_dtype = KDA_STATE_BF16 if state_pool.dtype == bf else KDA_STATE_FP32
     _check(slot_idx, "slot_idx", torch.int32, (N,))
     a.slot_idx = slot_idx.data_ptr()

@@ -34,6 +34,23 @@ kda_status check_device() {
   return cc == 100 ? KDA_OK : KDA_ERR_DEVICE;
 }
 
+// Once per kernel and device: let the kernel take `bytes` of dynamic shared
+// memory (the [V][K] staging buffer; above 48 KB this needs the opt-in) and
+// prefer the shared-memory carveout.
+template <auto Kernel>
+cudaError_t allow_dynamic_smem(int bytes) {
+  static std::atomic<uint64_t> ready{0};  // bit d: done on device d (d < 64)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit && (ready.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && bit) ready.fetch_or(bit, std::memory_order_relaxed);
+  return e;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Range {
@@ -61,6 +78,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
   if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0) return KDA_ERR_INVALID_ARG;
   if (gated && !(a.eps >= 0.0f && a.eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
   if (a.state_dtype != KDA_STATE_FP32 && a.state_dtype != KDA_STATE_BF16) return KDA_ERR_INVALID_ARG;
+  if (a.state_layout != KDA_LAYOUT_KV && a.state_layout != KDA_LAYOUT_VK) return KDA_ERR_INVALID_ARG;
   if (HV < 1) return KDA_ERR_UNSUPPORTED;
   if (K != 64 && K != 128 && K != 256) return KDA_ERR_UNSUPPORTED;
   if (V < kda::kBV || V % kda::kBV != 0) return KDA_ERR_UNSUPPORTED;
@@ -193,15 +211,29 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
   const int form = raw ? kda::kInRaw : dense ? kda::kInDense : kda::kInStrided;
 
   cudaError_t err = cudaErrorInvalidValue;
+  const bool vk = a.state_layout == KDA_LAYOUT_VK;
   const bool multi = T > 1;
   const bool v128 = V == 128;
   // One instantiation per (K, V fixed at 128 or not, gated, state type, input
-  // form); T == 1 and T > 1 (chunked) kernels.
+  // form, state layout); T == 1 and T > 1 (chunked) kernels.
+#define KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, STT, RR, VKK)                                             \
+  do {                                                                                                \
+    constexpr auto kern = kda::KERNEL<KK, VV, GG, STT, RR, VKK>;                                      \
+    constexpr int smem = kda::KERNEL##_dyn_smem<KK, STT, VKK>;                                        \
+    cfg.dynamicSmemBytes = smem;                                                                      \
+    err = smem ? allow_dynamic_smem<kern>(smem) : cudaSuccess;                                        \
+    if (err == cudaSuccess) err = cudaLaunchKernelEx(&cfg, kern, pf);                                 \
+  } while (0)
 #define KDA_LAUNCH_ST(KERNEL, KK, VV, GG, RR)                                                         \
   do {                                                                                                \
     const kda::ParamsOf<RR>& pf = p; /* the dense form takes the smaller block */                     \
-    if (bf16_state) err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, __nv_bfloat16, RR>, pf);   \
-    else err = cudaLaunchKernelEx(&cfg, kda::KERNEL<KK, VV, GG, float, RR>, pf);                      \
+    if (vk) {                                                                                         \
+      if (bf16_state) KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, true);                    \
+      else KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, float, RR, true);                                       \
+    } else {                                                                                          \
+      if (bf16_state) KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, false);                   \
+      else KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, float, RR, false);                                      \
+    }                                                                                                 \
   } while (0)
 #define KDA_LAUNCH(KERNEL, KK, VV, GG)                                             \
   do {                                                                             \
@@ -234,6 +266,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
 #undef KDA_LAUNCH_V
 #undef KDA_LAUNCH
 #undef KDA_LAUNCH_ST
+#undef KDA_LAUNCH_ONE
   return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -255,6 +288,7 @@ kda_decode_args dense_args(const void* q, const void* k, const void* v, const fl
   a.beta_row_stride = HV;
   a.state_pool = state_pool;
   a.state_dtype = state_dtype;
+  a.state_layout = KDA_LAYOUT_KV;
   a.slot_idx = slot_idx;
   a.gate = gate;
   a.gate_row_stride = HV * V;
@@ -333,6 +367,6 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 2; }
+int32_t kda_abi_version(void) { return (1 << 16) | 3; }
 
 }  // extern "C"

@@ -274,6 +274,147 @@ __device__ __forceinline__ void allow_next_grid() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- state tile I/O
+// A thread's state tile: key rows r0 .. r0+RPT-1 of the value columns
+// c .. c+3 (c = col0 + 4 cq), held as s[row][pair] (pair 0: columns c, c+1;
+// pair 1: c+2, c+3).
+//   VK = false, pool blocks [K][V]: row i of the thread's tile is four
+//     consecutive values at base + i * V, base = element (r0, c); a warp's
+//     16-byte accesses cover 4 rows x 128 bytes.
+//   VK = true, pool blocks [V][K] (key index fastest, FlashInfer #4562's
+//     layout): the CTA's 32 value columns are 32 runs of K contiguous values.
+//     Read straight into the thread layout above, a warp access would touch 8
+//     runs at half a line each (measured 1.6x slower), so the tile moves
+//     through shared memory: cp.async copies the whole tile in 16-byte pieces
+//     (a warp copies whole runs), then each thread reads its rows from the
+//     staged columns; the write-back goes the same way in reverse.  Piece p of
+//     staged column c sits at piece p ^ ((c >> 2) & 7), so the eight column
+//     quads that a quarter-warp reads at once fall in eight different banks.
+template <typename ST, bool VK, int K, int RPT>
+struct TileIO {
+  static constexpr int kE = 16 / static_cast<int>(sizeof(ST));  // elements per 16-byte piece
+  static_assert(K / kE >= 8, "the swizzle permutes pieces within groups of eight");
+  // Staging buffer of the [V][K] form, in dynamic shared memory (the launch
+  // gives it kStageBytes; the [K][V] form takes none).
+  struct Stage {
+    alignas(16) ST v[VK ? kBV * K : 1];
+  };
+  static constexpr int kStageBytes = VK ? static_cast<int>(sizeof(Stage)) : 0;
+  // Staged position of element (column c, key row r).
+  static __device__ __forceinline__ int at(int c, int r) {
+    return c * K + (((r / kE) ^ ((c >> 2) & 7)) * kE) + r % kE;
+  }
+
+  // KV: the thread's first element; VK: the first element of the CTA's tile.
+  static __device__ __forceinline__ ST* base(void* pool, int64_t slot, int64_t HV, int64_t h, int64_t V,
+                                             int r0, int64_t col0, int cq) {
+    ST* const blk = static_cast<ST*>(pool) + (slot * HV + h) * K * V;  // the (slot, h) state block
+    if constexpr (VK) return blk + col0 * K;
+    else return blk + static_cast<int64_t>(r0) * V + col0 + 4 * cq;
+  }
+
+  static __device__ __forceinline__ void load(float2 (&s)[RPT][2], const ST* b, int64_t V, Stage& st, int r0,
+                                              int cq) {
+    if constexpr (!VK) {
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) StateIO<ST>::load(s[i], b + i * V);
+    } else {
+      constexpr int kPieces = K / kE;  // per column
+      for (int id = threadIdx.x; id < kBV * kPieces; id += kThreads) {
+        const int c = id / kPieces, pc = id - c * kPieces;
+        cp_async16(smem_u32(&st.v[at(c, pc * kE)]), b + static_cast<int64_t>(c) * K + pc * kE);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 4 * cq + j;
+        if constexpr (sizeof(ST) == 4) {
+#pragma unroll
+          for (int a = 0; a < RPT / 4; ++a) {
+            const float4 x = *reinterpret_cast<const float4*>(&st.v[at(c, r0 + 4 * a)]);
+            put(s[4 * a + 0][j >> 1], j & 1, x.x);
+            put(s[4 * a + 1][j >> 1], j & 1, x.y);
+            put(s[4 * a + 2][j >> 1], j & 1, x.z);
+            put(s[4 * a + 3][j >> 1], j & 1, x.w);
+          }
+        } else {
+          uint32_t w[RPT / 2];
+          if constexpr (RPT % 8 == 0) {
+#pragma unroll
+            for (int a = 0; a < RPT / 8; ++a) {
+              const uint4 x = *reinterpret_cast<const uint4*>(&st.v[at(c, r0 + 8 * a)]);
+              w[4 * a] = x.x; w[4 * a + 1] = x.y; w[4 * a + 2] = x.z; w[4 * a + 3] = x.w;
+            }
+          } else {
+            const uint2 x = *reinterpret_cast<const uint2*>(&st.v[at(c, r0)]);
+            w[0] = x.x; w[1] = x.y;
+          }
+#pragma unroll
+          for (int i = 0; i < RPT; ++i) put(s[i][j >> 1], j & 1, bf16_at(w, i));
+        }
+      }
+    }
+  }
+
+  // Every thread of the CTA calls store (VK: it holds two block barriers).
+  static __device__ __forceinline__ void store(ST* b, const float2 (&s)[RPT][2], int64_t V, Stage& st, int r0,
+                                               int cq) {
+    if constexpr (!VK) {
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) StateIO<ST>::store(b + i * V, s[i]);
+    } else {
+      __syncthreads();  // the staging buffer may still be read by other threads' loads
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 4 * cq + j;
+        if constexpr (sizeof(ST) == 4) {
+#pragma unroll
+          for (int a = 0; a < RPT / 4; ++a)
+            *reinterpret_cast<float4*>(&st.v[at(c, r0 + 4 * a)]) =
+                make_float4(get(s[4 * a][j >> 1], j & 1), get(s[4 * a + 1][j >> 1], j & 1),
+                            get(s[4 * a + 2][j >> 1], j & 1), get(s[4 * a + 3][j >> 1], j & 1));
+        } else {
+          uint32_t w[RPT / 2];
+#pragma unroll
+          for (int i = 0; i < RPT / 2; ++i)
+            w[i] = pack_bf16x2(get(s[2 * i][j >> 1], j & 1), get(s[2 * i + 1][j >> 1], j & 1));
+          if constexpr (RPT % 8 == 0) {
+#pragma unroll
+            for (int a = 0; a < RPT / 8; ++a)
+              *reinterpret_cast<uint4*>(&st.v[at(c, r0 + 8 * a)]) =
+                  make_uint4(w[4 * a], w[4 * a + 1], w[4 * a + 2], w[4 * a + 3]);
+          } else {
+            *reinterpret_cast<uint2*>(&st.v[at(c, r0)]) = make_uint2(w[0], w[1]);
+          }
+        }
+      }
+      __syncthreads();
+      constexpr int kPieces = K / kE;
+      for (int id = threadIdx.x; id < kBV * kPieces; id += kThreads) {
+        const int c = id / kPieces, pc = id - c * kPieces;
+        __stcs(reinterpret_cast<float4*>(b + static_cast<int64_t>(c) * K + pc * kE),
+               *reinterpret_cast<const float4*>(&st.v[at(c, pc * kE)]));
+      }
+    }
+  }
+
+ private:
+  static __device__ __forceinline__ void put(float2& p, int hi, float x) {
+    if (hi) p.y = x; else p.x = x;
+  }
+  static __device__ __forceinline__ float get(const float2& p, int hi) { return hi ? p.y : p.x; }
+};
+
+// Dynamic shared memory a kernel launch must give: the one-token kernel keeps a
+// [V][K] staging buffer there; the multi-token kernel overlays it on its own
+// static buffers.
+template <int K, typename ST, bool VK>
+constexpr int kda_decode_kernel_dyn_smem = TileIO<ST, VK, K, K / 16>::kStageBytes;
+template <int K, typename ST, bool VK>
+constexpr int kda_decode_chunked_kernel_dyn_smem = 0;
+
 // ---------------------------------------------------------------- token staging (T > 1 kernel)
 // Shared-memory image of one token's inputs for one CTA (K key rows, the
 // CTA's 32 value columns).  Every member starts on a 16-byte boundary.
@@ -436,7 +577,7 @@ __device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], 
   if (writer) apply_norm(y, o, wgt, z, nrm, tiles, V, eps);
 }
 
-template <int K, int VS, bool GATED, typename ST, int IN>
+template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
 __global__ void __launch_bounds__(kThreads, (MinBlocksT1<K, VS, GATED>::value))
 kda_decode_kernel(const ParamsOf<IN> p) {
   constexpr bool RAW = IN == kInRaw;
@@ -513,10 +654,12 @@ kda_decode_kernel(const ParamsOf<IN> p) {
     return;  // uniform over the cluster: every tile of this (n, h) sees the same slot
   }
 
-  ST* const sp = static_cast<ST*>(p.state) + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col;
+  using Tile = TileIO<ST, VK, K, RPT>;
+  extern __shared__ __align__(16) unsigned char dyn_smem[];  // [V][K] staging (VK kernels only)
+  auto& stage = *reinterpret_cast<typename Tile::Stage*>(dyn_smem);
+  ST* const sp = Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
   float2 s[RPT][2];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) StateIO<ST>::load(s[i], sp + i * V);
+  Tile::load(s, sp, V, stage, r0, cq);
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
@@ -572,8 +715,7 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   }
 
   allow_next_grid();
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) StateIO<ST>::store(sp + i * V, s[i]);
+  Tile::store(sp, s, V, stage, r0, cq);
 
   if constexpr (GATED) {
     // The norm needs the whole head's o; the state does not, so it is
@@ -723,7 +865,7 @@ __device__ __forceinline__ void chunk_pass(const float2 (&s)[RPT][2], const floa
   red[warp][rg][cq] = make_float4(mine[0].x, mine[0].y, mine[1].x, mine[1].y);
 }
 
-template <int K, int VS, bool GATED, typename ST, int IN>
+template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
 __global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
 kda_decode_chunked_kernel(const ParamsOf<IN> p) {
   constexpr bool RAW = IN == kInRaw;
@@ -731,14 +873,41 @@ kda_decode_chunked_kernel(const ParamsOf<IN> p) {
   static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
   static_assert(kChunk == 4 && kRowGroups == kChunk, "one row group per chunk token in the reduce-scatter");
 
-  __shared__ TokenSmem<K> tok[2][kChunk];  // raw token inputs, double-buffered by chunk
-  __shared__ ChunkCoef<K> cf;
-  __shared__ __align__(16) float4 redR[kWarps][kChunk][kColQuads];
-  __shared__ __align__(16) float4 redQ[kWarps][kChunk][kColQuads];
-  __shared__ float mp_part[kWarps][kNumMP];
-  __shared__ float mp_tot[kNumMP];
+  // Shared memory.  A [V][K] pool's staging buffer is needed only while the
+  // state tile moves in (before the first chunk) and out (after the last), so
+  // it overlays everything from the second token buffer on (a separate buffer
+  // would cost the seventh CTA per SM); the tail pads the overlay to its size.
+  using Tile = TileIO<ST, VK, K, RPT>;
+  struct Tail {
+    TokenSmem<K> tok1[kChunk];
+    ChunkCoef<K> cf;
+    float4 redR[kWarps][kChunk][kColQuads];
+    float4 redQ[kWarps][kChunk][kColQuads];
+    float mp_part[kWarps][kNumMP];
+    float mp_tot[kNumMP];
+  };
+  static constexpr int kPad = Tile::kStageBytes > static_cast<int>(sizeof(Tail))
+                                  ? Tile::kStageBytes - static_cast<int>(sizeof(Tail)) : 1;
+  struct Shared {
+    TokenSmem<K> tok[2][kChunk];  // raw token inputs, double-buffered by chunk
+    ChunkCoef<K> cf;
+    float4 redR[kWarps][kChunk][kColQuads];
+    float4 redQ[kWarps][kChunk][kColQuads];
+    float mp_part[kWarps][kNumMP];
+    float mp_tot[kNumMP];
+    alignas(16) unsigned char pad[kPad];
+  };
+  static_assert(sizeof(Shared) - sizeof(TokenSmem<K>) * kChunk >= static_cast<size_t>(Tile::kStageBytes),
+                "the staging overlay must fit behind the first token buffer");
+  __shared__ __align__(16) Shared sh;
   __shared__ float nrm[2][kChunk][kMaxClusterTiles];  // gated: per-tile sums of o^2, by chunk parity
   __shared__ float osm[GATED ? kChunk : 1][kBV];  // gated: warp 0's o per token and column
+  auto& tok = sh.tok;
+  auto& cf = sh.cf;
+  auto& redR = sh.redR;
+  auto& redQ = sh.redQ;
+  auto& mp_part = sh.mp_part;
+  auto& mp_tot = sh.mp_tot;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -779,10 +948,10 @@ kda_decode_chunked_kernel(const ParamsOf<IN> p) {
     return;
   }
 
-  ST* const sp = static_cast<ST*>(p.state) + ((static_cast<int64_t>(slot) * p.HV + h) * K + r0) * V + col;
+  auto& stage = *reinterpret_cast<typename Tile::Stage*>(&sh.tok[1][0]);
+  ST* const sp = Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
   float2 s[RPT][2];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) StateIO<ST>::load(s[i], sp + i * V);
+  Tile::load(s, sp, V, stage, r0, cq);
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
@@ -917,8 +1086,7 @@ kda_decode_chunked_kernel(const ParamsOf<IN> p) {
   }
 
   allow_next_grid();
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) StateIO<ST>::store(sp + i * V, s[i]);
+  Tile::store(sp, s, V, stage, r0, cq);
 }
 
 }  // namespace kda

@@ -57,6 +57,13 @@ class Workload:
     raw: "RawGate | None" = None
     # q, k, v read as slices of one packed row buffer (the serving form does).
     packed: bool = False
+    # Block layout of the state pool: "kv" [num_slots, HV, K, V] or "vk"
+    # [num_slots, HV, V, K] (key index fastest).
+    state_layout: str = "kv"
+
+    def state_kv(self) -> torch.Tensor:
+        """The state pool as [num_slots, HV, K, V] (a transposed view for "vk")."""
+        return self.state if self.state_layout == "kv" else self.state.transpose(-1, -2)
 
     def tensors(self):
         """Dict of the call's tensors (gate/norm_weight only when gated; the raw
@@ -102,14 +109,16 @@ def _bf16(x: torch.Tensor) -> torch.Tensor:
 def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | None = None,
          gated: bool = False, seed: int = 0, name: str = "custom",
          decay: str = "softplus", inactive: int = 0, state_std: float = 0.02,
-         state_dtype: str = "fp32", serving: bool = False, packed: bool | None = None) -> Workload:
+         state_dtype: str = "fp32", serving: bool = False, packed: bool | None = None,
+         state_layout: str = "kv") -> Workload:
     """Draw one call's inputs.
 
     ``decay``: ``"softplus"`` (g = -softplus(N(0,1))) or ``"uniform"``
     (exp(g) ~ U[0.5, 1)).  ``inactive``: how many rows (the last ones) get a
     negative slot index, as CUDA-graph padding rows do.  ``serving``: raw gate
     and beta inputs instead of g and beta.  ``packed``: q, k, v to be passed as
-    slices of one packed row buffer (default: as ``serving``).
+    slices of one packed row buffer (default: as ``serving``).  ``state_layout``:
+    "kv" or "vk" (the same draw, stored with the key index fastest).
     """
     gen = torch.Generator().manual_seed(seed)
     if num_slots is None:
@@ -137,6 +146,10 @@ def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | N
         state = state.to(torch.bfloat16)
     elif state_dtype != "fp32":
         raise ValueError(state_dtype)
+    if state_layout == "vk":
+        state = state.transpose(-1, -2)
+    elif state_layout != "kv":
+        raise ValueError(state_layout)
     slot_idx = torch.randperm(num_slots, generator=gen)[:N].to(torch.int32)
     if inactive:
         slot_idx[N - inactive:] = -1
@@ -150,7 +163,7 @@ def make(N: int, T: int, HV: int, K: int = 128, V: int = 128, num_slots: int | N
                     g=None if serving else g.contiguous(), beta=None if serving else beta.contiguous(),
                     state=state.contiguous(), slot_idx=slot_idx.contiguous(),
                     scale=1.0 / math.sqrt(K), gate=gate, norm_weight=norm_weight, raw=raw,
-                    packed=serving if packed is None else packed)
+                    packed=serving if packed is None else packed, state_layout=state_layout)
 
 
 # The five workloads: name -> keyword arguments of ``make``.
@@ -175,6 +188,10 @@ CONFIGS = {
     # q, k, v packed in one row buffer, activated g and beta (row-strided kernels)
     "n32_t1_hv8_packed": dict(N=32, T=1, HV=8, num_slots=64, packed=True),
     "n32_t4_hv8_packed": dict(N=32, T=4, HV=8, num_slots=64, packed=True),
+    # [V, K] state blocks (key index fastest)
+    "n32_t1_hv8_vk": dict(N=32, T=1, HV=8, num_slots=64, state_layout="vk"),
+    "n32_t1_hv8_bf16state_vk": dict(N=32, T=1, HV=8, num_slots=64, state_dtype="bf16", state_layout="vk"),
+    "n32_t4_hv8_vk": dict(N=32, T=4, HV=8, num_slots=64, state_layout="vk"),
 }
 
 

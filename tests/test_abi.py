@@ -55,7 +55,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 2
+    assert lib.kda_abi_version() == (1 << 16) | 3
 
 
 # ----------------------------------------------------------------- validation
@@ -181,6 +181,8 @@ def test_ex_entry_point_validation(lib):
     assert args(q_row_stride=260) == E.KDA_ERR_MISALIGNED              # not a multiple of 8
     assert args(q_row_stride=512, T=1, N=2) == E.KDA_ERR_DEVICE        # a padded packed row
     assert args(state_dtype=2) == E.KDA_ERR_INVALID_ARG
+    assert args(state_layout=kda.KDA_LAYOUT_VK) == E.KDA_ERR_DEVICE     # [V, K] blocks, valid
+    assert args(state_layout=2) == E.KDA_ERR_INVALID_ARG
     assert args(raw_gate=BASE + 10 * step) == E.KDA_ERR_INVALID_ARG    # raw gate mixed with g
     assert args(gate=BASE + 10 * step) == E.KDA_ERR_INVALID_ARG        # gate without norm_weight
     raw = dict(g=0, beta=0, raw_gate=BASE + 3 * step, raw_beta=BASE + 4 * step + 2,

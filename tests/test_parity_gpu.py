@@ -406,28 +406,31 @@ def test_ex_raw_gate_form(N, T, HV, K, V, gated, state, cuda_device):
     assert_parity(w_ref, o, d.state, before)
 
 
-SERVING_CONFIGS = [n for n in workloads.CONFIGS if "_raw" in n or "_packed" in n]
+SERVING_CONFIGS = [n for n in workloads.CONFIGS if "_raw" in n or "_packed" in n or n.endswith("_vk")]
 
 
 @pytest.mark.parametrize("name", SERVING_CONFIGS)
 def test_named_serving_workload_parity(name, cuda_device):
-    """The packed and serving-form workloads, called as the benchmark calls them
-    (q, k, v packed in one row buffer; raw gate and beta, or activated ones)."""
+    """The packed, serving-form and [V, K]-pool workloads, called as the
+    benchmark calls them (kda_decode_ex; q, k, v packed in one row buffer when
+    the workload says so; raw gate and beta, or activated ones)."""
     w = workloads.config(name)
     d = w.to(cuda_device)
-    _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
-    before = d.state.clone()
+    q, k, v = d.q, d.k, d.v
+    if w.packed:
+        _, (q, k, v) = workloads.pack_rows([d.q, d.k, d.v], pad=8)
+    before = d.state_kv().clone()
     extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if w.gated else {}
     if w.raw is not None:
         extra.update(raw_gate=d.raw.raw_gate, A_log=d.raw.A_log, dt_bias=d.raw.dt_bias, raw_beta=d.raw.raw_beta)
     else:
         extra.update(g=d.g, beta=d.beta)
-    o = kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, scale=w.scale, **extra)
+    o = kda.kda_decode_ex(q, k, v, d.state, d.slot_idx, scale=w.scale, state_layout=w.state_layout, **extra)
     torch.cuda.synchronize()
     if w.raw is not None:
         g, beta = oracle.activate(w.raw.raw_gate, w.raw.A_log, w.raw.dt_bias, w.raw.raw_beta)
         w = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
-    assert_parity(w, o, d.state, before)
+    assert_parity(dataclasses.replace(w, state=w.state_kv()), o, d.state_kv(), before)
 
 
 @pytest.mark.parametrize("T,gated,state", [(1, False, "fp32"), (1, True, "bf16"), (4, False, "fp32"),
@@ -450,3 +453,57 @@ def test_strided_form_bit_identical_to_dense(T, gated, state, cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(o_dense, o_strided)
     assert torch.equal(p_dense, p_strided)
+
+
+VK_CASES = [  # N, T, HV, K, V, gated, state dtype, input form
+    (5, 1, 3, 128, 128, False, "fp32", "dense"),
+    (5, 1, 3, 128, 128, True, "fp32", "dense"),
+    (4, 1, 2, 64, 96, False, "fp32", "dense"),
+    (3, 1, 2, 256, 64, True, "fp32", "dense"),
+    (5, 4, 3, 128, 128, False, "fp32", "dense"),
+    (3, 9, 2, 128, 160, True, "fp32", "dense"),
+    (4, 1, 3, 128, 128, False, "bf16", "dense"),
+    (4, 1, 3, 64, 128, True, "bf16", "dense"),
+    (3, 6, 2, 256, 128, False, "bf16", "dense"),
+    (4, 1, 3, 128, 128, False, "fp32", "raw"),
+    (3, 5, 2, 128, 128, True, "bf16", "raw"),
+]
+
+
+def _vk_call(w, d, pool, layout, form):
+    extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if w.gated else {}
+    if form == "raw":
+        r = d.raw
+        extra.update(raw_gate=r.raw_gate, A_log=r.A_log, dt_bias=r.dt_bias, raw_beta=r.raw_beta)
+    else:
+        extra.update(g=d.g, beta=d.beta)
+    return kda.kda_decode_ex(d.q, d.k, d.v, pool, d.slot_idx, scale=w.scale, state_layout=layout, **extra)
+
+
+@pytest.mark.parametrize("N,T,HV,K,V,gated,state,form", VK_CASES)
+def test_vk_layout_parity(N, T, HV, K, V, gated, state, form, cuda_device):
+    """[V, K] state blocks: against the oracle on the same state read as [K, V],
+    and bit-identical to the [K, V] pool (the same arithmetic, another address
+    map)."""
+    w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 3, gated=gated, seed=70 + N + T + K,
+                       state_dtype=state, inactive=1, serving=form == "raw", packed=False)
+    d = w.to(cuda_device)
+    pool_kv = d.state.clone()
+    pool_vk = d.state.transpose(-1, -2).contiguous()
+    before = d.state.clone()
+    o_kv = _vk_call(w, d, pool_kv, "kv", form)
+    o_vk = _vk_call(w, d, pool_vk, "vk", form)
+    torch.cuda.synchronize()
+    assert torch.equal(o_kv, o_vk), "outputs differ between the [K, V] and [V, K] pools"
+    assert torch.equal(pool_kv, pool_vk.transpose(-1, -2)), "states differ between the [K, V] and [V, K] pools"
+    if form == "raw":
+        g, beta = oracle.activate(w.raw.raw_gate, w.raw.A_log, w.raw.dt_bias, w.raw.raw_beta)
+        w = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
+    assert_parity(w, o_vk, pool_vk.transpose(-1, -2), before)
+
+
+def test_vk_layout_rejects_wrong_pool_shape(cuda_device):
+    w = workloads.make(N=2, T=1, HV=2, K=128, V=64, num_slots=3, seed=5)
+    d = w.to(cuda_device)
+    with pytest.raises(ValueError):
+        kda.kda_decode_ex(d.q, d.k, d.v, d.state, d.slot_idx, g=d.g, beta=d.beta, state_layout="vk")
