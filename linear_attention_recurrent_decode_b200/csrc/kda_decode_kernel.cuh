@@ -865,49 +865,33 @@ __device__ __forceinline__ void chunk_pass(const float2 (&s)[RPT][2], const floa
   red[warp][rg][cq] = make_float4(mine[0].x, mine[0].y, mine[1].x, mine[1].y);
 }
 
+// Shared buffers of the multi-token kernel.
+template <int K, bool GATED>
+struct ChunkBuffers {
+  TokenSmem<K> (&tok)[2][kChunk];  // raw token inputs, double-buffered by chunk
+  ChunkCoef<K>& cf;
+  float4 (&redR)[kWarps][kChunk][kColQuads];
+  float4 (&redQ)[kWarps][kChunk][kColQuads];
+  float (&mp_part)[kWarps][kNumMP];
+  float (&mp_tot)[kNumMP];
+  float (&nrm)[2][kChunk][kMaxClusterTiles];  // gated: per-tile sums of o^2, by chunk parity
+  float (&osm)[GATED ? kChunk : 1][kBV];      // gated: warp 0's o per token and column
+};
+
 template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
-__global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
-kda_decode_chunked_kernel(const ParamsOf<IN> p) {
+__device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkBuffers<K, GATED>& b,
+                                             typename TileIO<ST, VK, K, K / 16>::Stage& stage) {
   constexpr bool RAW = IN == kInRaw;
   constexpr int RPT = K / (kWarps * kRowGroups);
-  static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
-  static_assert(kChunk == 4 && kRowGroups == kChunk, "one row group per chunk token in the reduce-scatter");
-
-  // Shared memory.  A [V][K] pool's staging buffer is needed only while the
-  // state tile moves in (before the first chunk) and out (after the last), so
-  // it overlays everything from the second token buffer on (a separate buffer
-  // would cost the seventh CTA per SM); the tail pads the overlay to its size.
   using Tile = TileIO<ST, VK, K, RPT>;
-  struct Tail {
-    TokenSmem<K> tok1[kChunk];
-    ChunkCoef<K> cf;
-    float4 redR[kWarps][kChunk][kColQuads];
-    float4 redQ[kWarps][kChunk][kColQuads];
-    float mp_part[kWarps][kNumMP];
-    float mp_tot[kNumMP];
-  };
-  static constexpr int kPad = Tile::kStageBytes > static_cast<int>(sizeof(Tail))
-                                  ? Tile::kStageBytes - static_cast<int>(sizeof(Tail)) : 1;
-  struct Shared {
-    TokenSmem<K> tok[2][kChunk];  // raw token inputs, double-buffered by chunk
-    ChunkCoef<K> cf;
-    float4 redR[kWarps][kChunk][kColQuads];
-    float4 redQ[kWarps][kChunk][kColQuads];
-    float mp_part[kWarps][kNumMP];
-    float mp_tot[kNumMP];
-    alignas(16) unsigned char pad[kPad];
-  };
-  static_assert(sizeof(Shared) - sizeof(TokenSmem<K>) * kChunk >= static_cast<size_t>(Tile::kStageBytes),
-                "the staging overlay must fit behind the first token buffer");
-  __shared__ __align__(16) Shared sh;
-  __shared__ float nrm[2][kChunk][kMaxClusterTiles];  // gated: per-tile sums of o^2, by chunk parity
-  __shared__ float osm[GATED ? kChunk : 1][kBV];  // gated: warp 0's o per token and column
-  auto& tok = sh.tok;
-  auto& cf = sh.cf;
-  auto& redR = sh.redR;
-  auto& redQ = sh.redQ;
-  auto& mp_part = sh.mp_part;
-  auto& mp_tot = sh.mp_tot;
+  auto& tok = b.tok;
+  auto& cf = b.cf;
+  auto& redR = b.redR;
+  auto& redQ = b.redQ;
+  auto& mp_part = b.mp_part;
+  auto& mp_tot = b.mp_tot;
+  auto& nrm = b.nrm;
+  auto& osm = b.osm;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -948,7 +932,6 @@ kda_decode_chunked_kernel(const ParamsOf<IN> p) {
     return;
   }
 
-  auto& stage = *reinterpret_cast<typename Tile::Stage*>(&sh.tok[1][0]);
   ST* const sp = Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
   float2 s[RPT][2];
   Tile::load(s, sp, V, stage, r0, cq);
@@ -1087,6 +1070,57 @@ kda_decode_chunked_kernel(const ParamsOf<IN> p) {
 
   allow_next_grid();
   Tile::store(sp, s, V, stage, r0, cq);
+}
+
+template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
+__global__ void __launch_bounds__(kThreads, (MinBlocks<K>::value))
+kda_decode_chunked_kernel(const ParamsOf<IN> p) {
+  constexpr int RPT = K / (kWarps * kRowGroups);
+  static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
+  static_assert(kChunk == 4 && kRowGroups == kChunk, "one row group per chunk token in the reduce-scatter");
+  using Tile = TileIO<ST, VK, K, RPT>;
+  __shared__ float nrm[2][kChunk][kMaxClusterTiles];
+  __shared__ float osm[GATED ? kChunk : 1][kBV];
+  if constexpr (!VK) {
+    __shared__ TokenSmem<K> tok[2][kChunk];
+    __shared__ ChunkCoef<K> cf;
+    __shared__ __align__(16) float4 redR[kWarps][kChunk][kColQuads];
+    __shared__ __align__(16) float4 redQ[kWarps][kChunk][kColQuads];
+    __shared__ float mp_part[kWarps][kNumMP];
+    __shared__ float mp_tot[kNumMP];
+    chunked_body<K, VS, GATED, ST, IN, VK>(p, ChunkBuffers<K, GATED>{tok, cf, redR, redQ, mp_part, mp_tot, nrm, osm},
+                                           *reinterpret_cast<typename Tile::Stage*>(&mp_tot[0]));
+  } else {
+    // A [V][K] pool's staging buffer is needed only while the state tile moves
+    // in (before the first chunk) and out (after the last), so it overlays
+    // everything from the second token buffer on (a separate buffer would cost
+    // the seventh CTA per SM); the pad makes the overlay fit.
+    struct Tail {
+      TokenSmem<K> tok1[kChunk];
+      ChunkCoef<K> cf;
+      float4 redR[kWarps][kChunk][kColQuads];
+      float4 redQ[kWarps][kChunk][kColQuads];
+      float mp_part[kWarps][kNumMP];
+      float mp_tot[kNumMP];
+    };
+    constexpr int kPad = Tile::kStageBytes > static_cast<int>(sizeof(Tail))
+                             ? Tile::kStageBytes - static_cast<int>(sizeof(Tail)) : 1;
+    struct Shared {
+      TokenSmem<K> tok[2][kChunk];
+      ChunkCoef<K> cf;
+      float4 redR[kWarps][kChunk][kColQuads];
+      float4 redQ[kWarps][kChunk][kColQuads];
+      float mp_part[kWarps][kNumMP];
+      float mp_tot[kNumMP];
+      alignas(16) unsigned char pad[kPad];
+    };
+    static_assert(sizeof(Shared) - sizeof(TokenSmem<K>) * kChunk >= static_cast<size_t>(Tile::kStageBytes),
+                  "the staging overlay must fit behind the first token buffer");
+    __shared__ __align__(16) Shared sh;
+    chunked_body<K, VS, GATED, ST, IN, VK>(
+        p, ChunkBuffers<K, GATED>{sh.tok, sh.cf, sh.redR, sh.redQ, sh.mp_part, sh.mp_tot, nrm, osm},
+        *reinterpret_cast<typename Tile::Stage*>(&sh.tok[1][0]));
+  }
 }
 
 }  // namespace kda
