@@ -406,10 +406,12 @@ def copy_floor(w, dev, stream, R, steps):
 
 def run_e2e(kda, w, dev, stream, steps, world):
     """µs per call with each step's inputs copied from pinned host memory and its
-    output read back, through the public Python API, eager launches.  A step's
-    inputs live in one packed pinned buffer (as a serving host would stage
-    them), so each step is one host-to-device copy, the decode call and one
-    device-to-host copy of the output; the state pool stays resident on the GPU."""
+    output read back, through the public API (``HostStep``, the C ABI's
+    ``kda_decode_host``), eager launches.  A step's inputs live in one packed
+    pinned buffer (as a serving host would stage them), so each step is one
+    host-to-device copy, the decode kernel and one device-to-host copy of the
+    output, enqueued by one library call; the state pool stays resident on the
+    GPU."""
     import torch
 
     inputs = {k: t for k, t in w.tensors().items() if k != "state"}
@@ -420,28 +422,20 @@ def run_e2e(kda, w, dev, stream, steps, world):
     pool = w.state.to(dev)
     out_d = torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=dev)
     out_h = torch.empty(out_d.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in inputs.values())
+    h2d = host_buf.numel()  # the packed buffer each step copies (inputs and their 16-byte alignment)
     d2h = out_h.numel() * out_h.element_size()
 
-    def step():
-        dev_buf.copy_(host_buf, non_blocking=True)
-        if w.raw is not None or w.packed or w.state_layout != "kv":
-            extra = dict(gate=devv["gate"], norm_weight=devv["norm_weight"], eps=w.eps) if w.gated else {}
-            if w.raw is not None:
-                extra.update(raw_gate=devv["raw_gate"], A_log=devv["A_log"], dt_bias=devv["dt_bias"],
-                             raw_beta=devv["raw_beta"])
-            else:
-                extra.update(g=devv["g"], beta=devv["beta"])
-            kda.kda_decode_ex(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], scale=w.scale, out=out_d,
-                              stream=stream, state_layout=w.state_layout, **extra)
-        elif w.gated:
-            kda.kda_decode_gated_rmsnorm(devv["q"], devv["k"], devv["v"], devv["g"], devv["beta"], pool,
-                                         devv["slot_idx"], devv["gate"], devv["norm_weight"], eps=w.eps,
-                                         scale=w.scale, out=out_d, stream=stream)
-        else:
-            kda.kda_decode(devv["q"], devv["k"], devv["v"], devv["g"], devv["beta"], pool,
-                           devv["slot_idx"], scale=w.scale, out=out_d, stream=stream)
-        out_h.copy_(out_d, non_blocking=True)
+    extra = dict(gate=devv["gate"], norm_weight=devv["norm_weight"], eps=w.eps) if w.gated else {}
+    if w.raw is not None:
+        extra.update(raw_gate=devv["raw_gate"], A_log=devv["A_log"], dt_bias=devv["dt_bias"],
+                     raw_beta=devv["raw_beta"])
+    else:
+        extra.update(g=devv["g"], beta=devv["beta"])
+    # One library call per step: it enqueues the copy of the packed inputs, the
+    # decode step and the copy of the output back.
+    step = kda.HostStep(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], host_in=host_buf,
+                        dev_in=dev_buf, host_out=out_h, out=out_d, stream=stream, scale=w.scale,
+                        state_layout=w.state_layout, **extra)
 
     with torch.cuda.stream(stream):
         for _ in range(10):
@@ -458,8 +452,8 @@ def run_e2e(kda, w, dev, stream, steps, world):
     ms = reduce_max(e0.elapsed_time(e1), dev)
     return {"value": round(ms * 1e3 / (steps * world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
-            "how": "eager public-API calls; each step copies its inputs from one packed pinned host "
-                   "buffer and its output back; the state pool stays resident on the GPU"}
+            "how": "one kda_decode_host call per step (HostStep): copy of the packed inputs from pinned host "
+                   "memory, the decode kernel, copy of the output back; the state pool stays resident on the GPU"}
 
 
 # ------------------------------------------------------------------ reference arm

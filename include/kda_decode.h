@@ -220,6 +220,28 @@ typedef struct {
  */
 KDA_API kda_status kda_decode_ex(const kda_decode_args *args, kda_stream_t stream);
 
+/*
+ * The step fed from and returning to host memory, in one call.  It enqueues on
+ * `stream`, in order: a host-to-device copy of in_bytes bytes from host_in to
+ * dev_in; the step that kda_decode_ex(args) enqueues; a device-to-host copy of
+ * the output (N*T*HV*V bf16 from args->out) to host_out.  The caller stages a
+ * step's inputs in host_in so that, once copied, args' input pointers (q, k,
+ * v, g/beta or the raw inputs, slot_idx, gate, norm_weight) point at them
+ * inside dev_in; the state pool stays on the device.  For the copies to run
+ * asynchronously host_in and host_out must be page-locked; host_out holds the
+ * output once the stream has reached the end of the call.  The library
+ * allocates nothing: dev_in is caller-owned device memory.  None of the pages
+ * describes such an entry point: it is this library's own, for callers that
+ * measure or run the step end to end from host memory.
+ *
+ * Errors: those of kda_decode_ex; KDA_ERR_INVALID_ARG also for in_bytes < 0,
+ * a NULL host_in or dev_in with in_bytes > 0, or a NULL host_out;
+ * KDA_ERR_ALIAS if dev_in overlaps the state pool's visible extent.  Nothing
+ * is enqueued unless validation passes; N == 0 or T == 0 enqueues nothing.
+ */
+KDA_API kda_status kda_decode_host(const kda_decode_args *args, const void *host_in, void *dev_in,
+                                   int64_t in_bytes, void *host_out, kda_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 

@@ -22,7 +22,7 @@ import math
 import os
 import threading
 
-__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "KdaError", "library", "status_string",
+__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_STATE_FP32", "KDA_STATE_BF16",
            "KDA_LAYOUT_KV", "KDA_LAYOUT_VK", "LIBRARY_PATH", "EXPORTED_SYMBOLS"]
@@ -72,6 +72,7 @@ EXPORTED_SYMBOLS = {
     "kda_decode_bf16_state": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_gated_rmsnorm_bf16_state": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_ex": ([ctypes.POINTER(DecodeArgs), _P], ctypes.c_int),
+    "kda_decode_host": ([ctypes.POINTER(DecodeArgs), _P, _P, _I, _P, _P], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_abi_version": ([], ctypes.c_int32),
 }
@@ -223,20 +224,10 @@ def _rows(t, name, dtype, N, T, inner):
     return rs if (N * T) > 1 else max(rs, want)
 
 
-def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
+def _ex_args(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
                   dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
-                  scale: float | None = None, stream=None, state_layout: str = "kv"):
-    """General decode step (``kda_decode_ex`` of the C ABI).
-
-    q, k [N,T,HV,K], v [N,T,HV,V] (bf16) may be strided views, e.g. slices of
-    one packed ``mixed_qkv`` row buffer; so may g / raw_gate [N,T,HV,K] and
-    beta / raw_beta [N,T,HV] and gate [N,T,HV,V].  Give either ``g`` and
-    ``beta`` (fp32) or the serving form ``raw_gate``, ``A_log`` [HV],
-    ``dt_bias`` [HV,K] (fp32) and ``raw_beta`` (bf16).  ``gate`` with
-    ``norm_weight`` selects the fused gated RMS norm.  The pool may be fp32 or
-    bf16, with blocks [K, V] (``state_layout="kv"``: pool [num_slots,HV,K,V])
-    or [V, K] (``"vk"``: pool [num_slots,HV,V,K], key index fastest).
-    Returns ``out`` (dense bf16 [N,T,HV,V])."""
+                  scale: float | None = None, state_layout: str = "kv"):
+    """The kda_decode_args of a call (and its output tensor); see kda_decode_ex."""
     import torch
 
     N, T, HV, K = q.shape
@@ -279,7 +270,70 @@ def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=
     a.out = out.data_ptr()
     a.N, a.T, a.HV, a.K, a.V = N, T, HV, K, V
     a.scale = float(1.0 / math.sqrt(K) if scale is None else scale)
+    return a, out
+
+
+def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
+                  dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
+                  scale: float | None = None, stream=None, state_layout: str = "kv"):
+    """General decode step (``kda_decode_ex`` of the C ABI).
+
+    q, k [N,T,HV,K], v [N,T,HV,V] (bf16) may be strided views, e.g. slices of
+    one packed ``mixed_qkv`` row buffer; so may g / raw_gate [N,T,HV,K] and
+    beta / raw_beta [N,T,HV] and gate [N,T,HV,V].  Give either ``g`` and
+    ``beta`` (fp32) or the serving form ``raw_gate``, ``A_log`` [HV],
+    ``dt_bias`` [HV,K] (fp32) and ``raw_beta`` (bf16).  ``gate`` with
+    ``norm_weight`` selects the fused gated RMS norm.  The pool may be fp32 or
+    bf16, with blocks [K, V] (``state_layout="kv"``: pool [num_slots,HV,K,V])
+    or [V, K] (``"vk"``: pool [num_slots,HV,V,K], key index fastest).
+    Returns ``out`` (dense bf16 [N,T,HV,V])."""
+    a, out = _ex_args(q, k, v, state_pool, slot_idx, g=g, beta=beta, raw_gate=raw_gate, A_log=A_log,
+                      dt_bias=dt_bias, raw_beta=raw_beta, gate=gate, norm_weight=norm_weight, eps=eps, out=out,
+                      scale=scale, state_layout=state_layout)
     st = library().kda_decode_ex(ctypes.byref(a), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_ex")
     return out
+
+
+class HostStep:
+    """One decode step run from host memory (``kda_decode_host`` of the C ABI),
+    bound once and run many times, as a serving loop with static buffers does.
+
+    ``host_in`` (pinned uint8) is copied to ``dev_in`` (device uint8) each
+    call; the tensors given for the step's inputs must be views into
+    ``dev_in``.  The output goes to ``out`` on the device and is copied to
+    ``host_out`` (pinned, same shape and dtype).  Keyword arguments are those of
+    :func:`kda_decode_ex`.  Calling the object enqueues the copy in, the step
+    and the copy out on ``stream``: one call into the library per step.
+    """
+
+    def __init__(self, q, k, v, state_pool, slot_idx, *, host_in, dev_in, host_out, out, stream=None, **kw):
+        import torch
+
+        for name, t in (("host_in", host_in), ("host_out", host_out)):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError(f"{name} must be pinned host memory")
+        if not dev_in.is_cuda or not dev_in.is_contiguous() or not host_in.is_contiguous():
+            raise ValueError("dev_in must be a contiguous device tensor, host_in contiguous")
+        nbytes = host_in.numel() * host_in.element_size()
+        if dev_in.numel() * dev_in.element_size() < nbytes:
+            raise ValueError("dev_in is smaller than host_in")
+        if host_out.shape != out.shape or host_out.dtype != out.dtype or not host_out.is_contiguous():
+            raise ValueError("host_out must match out")
+        lo, hi = dev_in.data_ptr(), dev_in.data_ptr() + nbytes
+        for name, t in (("q", q), ("k", k), ("v", v), ("slot_idx", slot_idx)):
+            if not lo <= t.data_ptr() < hi:
+                raise ValueError(f"{name} must be a view into dev_in")
+        self.args, self.out = _ex_args(q, k, v, state_pool, slot_idx, out=out, **kw)
+        self._keep = (q, k, v, state_pool, slot_idx, host_in, dev_in, host_out, out, kw)
+        self._ptrs = (host_in.data_ptr(), dev_in.data_ptr(), nbytes, host_out.data_ptr())
+        self._torch_stream = stream if stream is not None else torch.cuda.current_stream()
+        self._stream = _stream_handle(self._torch_stream)
+        self._fn = library().kda_decode_host
+        self._ref = ctypes.byref(self.args)
+
+    def __call__(self):
+        st = self._fn(self._ref, *self._ptrs, self._stream)
+        if st != KDA_OK:
+            raise KdaError(st, "kda_decode_host")

@@ -72,8 +72,19 @@ bool span_bytes(int64_t rows, int64_t stride, int64_t width, int64_t elem, int64
   return mul_ok(a, elem, bytes);
 }
 
-kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
+// Host staging of kda_decode_host: the step's inputs are copied from host_in to
+// dev_in before the kernel, the output from out to host_out after it.
+struct HostCopies {
+  const void* host_in;
+  void* dev_in;
+  int64_t in_bytes;
+  void* host_out;
+};
+
+kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, const HostCopies* hc = nullptr) {
   const int64_t N = a.N, T = a.T, HV = a.HV, K = a.K, V = a.V;
+  if (hc && (hc->in_bytes < 0 || (hc->in_bytes > 0 && (!hc->host_in || !hc->dev_in)) || !hc->host_out))
+    return KDA_ERR_INVALID_ARG;
   // ---- sizes
   if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0) return KDA_ERR_INVALID_ARG;
   if (gated && !(a.eps >= 0.0f && a.eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
@@ -146,6 +157,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
     return overlaps(r, r_slot0) || (r.lo <= pool_base && pool_base < r.hi);
   };
   if (touches_pool(r_out)) return KDA_ERR_ALIAS;
+  if (hc && hc->in_bytes > 0 && touches_pool(range_of(hc->dev_in, hc->in_bytes))) return KDA_ERR_ALIAS;
   for (const Range& r : inputs) {
     if (r.hi == r.lo) continue;
     if (overlaps(r, r_out) || touches_pool(r)) return KDA_ERR_ALIAS;
@@ -211,6 +223,10 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
   const int form = raw ? kda::kInRaw : dense ? kda::kInDense : kda::kInStrided;
 
   cudaError_t err = cudaErrorInvalidValue;
+  if (hc && hc->in_bytes > 0 &&
+      cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
+                      cfg.stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
   const bool vk = a.state_layout == KDA_LAYOUT_VK;
   const bool multi = T > 1;
   const bool v128 = V == 128;
@@ -267,7 +283,11 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream) {
 #undef KDA_LAUNCH
 #undef KDA_LAUNCH_ST
 #undef KDA_LAUNCH_ONE
-  return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  if (err != cudaSuccess) return KDA_ERR_CUDA;
+  if (hc && cudaMemcpyAsync(hc->host_out, a.out, static_cast<size_t>(out_elems) * 2, cudaMemcpyDeviceToHost,
+                            cfg.stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return KDA_OK;
 }
 
 // Dense (contiguous) arguments of the four fixed-layout entry points.
@@ -352,6 +372,14 @@ kda_status kda_decode_ex(const kda_decode_args* args, kda_stream_t stream) {
   return launch(*args, /*gated=*/args->gate != nullptr, stream);
 }
 
+kda_status kda_decode_host(const kda_decode_args* args, const void* host_in, void* dev_in, int64_t in_bytes,
+                           void* host_out, kda_stream_t stream) {
+  if (args == nullptr) return KDA_ERR_INVALID_ARG;
+  if ((args->gate == nullptr) != (args->norm_weight == nullptr)) return KDA_ERR_INVALID_ARG;
+  const HostCopies hc{host_in, dev_in, in_bytes, host_out};
+  return launch(*args, /*gated=*/args->gate != nullptr, stream, &hc);
+}
+
 const char* kda_status_string(kda_status status) {
   switch (status) {
     case KDA_OK: return "ok";
@@ -367,6 +395,6 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 3; }
+int32_t kda_abi_version(void) { return (1 << 16) | 4; }
 
 }  // extern "C"

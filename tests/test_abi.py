@@ -35,7 +35,7 @@ def declared_functions():
 def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
-                                    "kda_status_string", "kda_abi_version"}
+                                    "kda_decode_host", "kda_status_string", "kda_abi_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -55,7 +55,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 3
+    assert lib.kda_abi_version() == (1 << 16) | 4
 
 
 # ----------------------------------------------------------------- validation
@@ -190,3 +190,32 @@ def test_ex_entry_point_validation(lib):
     assert args(**raw) == E.KDA_ERR_DEVICE                             # raw form, 2-byte raw_beta is fine
     assert args(**{**raw, "dt_bias": BASE + 12 * step + 4}) == E.KDA_ERR_MISALIGNED
     assert args(**{**raw, "A_log": 0}) == E.KDA_ERR_INVALID_ARG
+
+
+@no_gpu
+def test_host_entry_point_validation(lib):
+    """kda_decode_host validates its host staging before anything is enqueued."""
+    E = kda
+    step = 1 << 30
+    a = kda.DecodeArgs()
+    N, T, HV, K, V = 2, 1, 2, 128, 128
+    a.q, a.q_row_stride = BASE, HV * K
+    a.k, a.k_row_stride = BASE + step, HV * K
+    a.v, a.v_row_stride = BASE + 2 * step, HV * V
+    a.g, a.g_row_stride = BASE + 3 * step, HV * K
+    a.beta, a.beta_row_stride = BASE + 4 * step, HV
+    a.state_pool, a.slot_idx, a.out = BASE + 5 * step, BASE + 8 * step, BASE + 9 * step
+    a.N, a.T, a.HV, a.K, a.V, a.scale = N, T, HV, K, V, 0.1
+    host_in, dev_in, host_out = BASE + 20 * step, BASE + 21 * step, BASE + 22 * step
+
+    def call(hin=host_in, din=dev_in, nbytes=4096, hout=host_out):
+        return lib.kda_decode_host(ctypes.byref(a), hin, din, nbytes, hout, None)
+
+    assert lib.kda_decode_host(None, host_in, dev_in, 4096, host_out, None) == E.KDA_ERR_INVALID_ARG
+    assert call() == E.KDA_ERR_DEVICE                      # valid, no device here
+    assert call(nbytes=-1) == E.KDA_ERR_INVALID_ARG
+    assert call(hin=None) == E.KDA_ERR_INVALID_ARG
+    assert call(din=None) == E.KDA_ERR_INVALID_ARG
+    assert call(hin=None, din=None, nbytes=0) == E.KDA_ERR_DEVICE  # nothing to copy in
+    assert call(hout=None) == E.KDA_ERR_INVALID_ARG
+    assert call(din=BASE + 5 * step - 64, nbytes=128) == E.KDA_ERR_ALIAS  # staging runs into the pool

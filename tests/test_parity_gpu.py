@@ -507,3 +507,60 @@ def test_vk_layout_rejects_wrong_pool_shape(cuda_device):
     d = w.to(cuda_device)
     with pytest.raises(ValueError):
         kda.kda_decode_ex(d.q, d.k, d.v, d.state, d.slot_idx, g=d.g, beta=d.beta, state_layout="vk")
+
+
+@pytest.mark.parametrize("name", ["n32_t1_hv8", "n32_t1_hv16_gated", "n8_t4_hv8", "n32_t1_hv8_raw"])
+def test_host_step_equals_device_call(name, cuda_device):
+    """HostStep (kda_decode_host): inputs staged in pinned host memory, copied in,
+    decoded and the output copied back by one library call per step.  Two
+    steps on one pool give the same outputs and state as two kda_decode_ex
+    calls on device tensors."""
+    w = workloads.config(name)
+    inputs = {key: t for key, t in w.tensors().items() if key != "state"}
+    nbytes = sum((t.numel() * t.element_size() + 15) // 16 * 16 for t in inputs.values())
+    host_in = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dev_in = torch.empty(nbytes, dtype=torch.uint8, device=cuda_device)
+    hv, dv, off = {}, {}, 0
+    for key, t in inputs.items():
+        b = t.numel() * t.element_size()
+        hv[key] = host_in[off:off + b].view(t.dtype).view(t.shape)
+        dv[key] = dev_in[off:off + b].view(t.dtype).view(t.shape)
+        hv[key].copy_(t)
+        off += (b + 15) // 16 * 16
+    extra = dict(gate=dv["gate"], norm_weight=dv["norm_weight"], eps=w.eps) if w.gated else {}
+    if w.raw is not None:
+        extra.update(raw_gate=dv["raw_gate"], A_log=dv["A_log"], dt_bias=dv["dt_bias"], raw_beta=dv["raw_beta"])
+    else:
+        extra.update(g=dv["g"], beta=dv["beta"])
+    pool_h = w.state.to(cuda_device)
+    out_d = torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=cuda_device)
+    host_out = torch.empty(out_d.shape, dtype=torch.bfloat16).pin_memory()
+    step = kda.HostStep(dv["q"], dv["k"], dv["v"], pool_h, dv["slot_idx"], host_in=host_in, dev_in=dev_in,
+                        host_out=host_out, out=out_d, scale=w.scale, **extra)
+    d = w.to(cuda_device)
+    pool_ref = d.state.clone()
+    ref_extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if w.gated else {}
+    if w.raw is not None:
+        ref_extra.update(raw_gate=d.raw.raw_gate, A_log=d.raw.A_log, dt_bias=d.raw.dt_bias, raw_beta=d.raw.raw_beta)
+    else:
+        ref_extra.update(g=d.g, beta=d.beta)
+    for _ in range(2):
+        dev_in.zero_()  # the step must bring its own inputs in
+        step()
+        torch.cuda.synchronize()
+        ref = kda.kda_decode_ex(d.q, d.k, d.v, pool_ref, d.slot_idx, scale=w.scale, **ref_extra)
+        torch.cuda.synchronize()
+        assert torch.equal(host_out, ref.cpu())
+        assert torch.equal(pool_h, pool_ref)
+
+
+def test_host_step_rejects_views_outside_the_staging_buffer(cuda_device):
+    w = workloads.make(N=2, T=1, HV=2, K=128, V=64, num_slots=3, seed=9)
+    d = w.to(cuda_device)
+    host_in = torch.empty(1 << 16, dtype=torch.uint8).pin_memory()
+    dev_in = torch.empty(1 << 16, dtype=torch.uint8, device=cuda_device)
+    out = torch.empty(2, 1, 2, 64, dtype=torch.bfloat16, device=cuda_device)
+    host_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    with pytest.raises(ValueError):
+        kda.HostStep(d.q, d.k, d.v, d.state, d.slot_idx, host_in=host_in, dev_in=dev_in, host_out=host_out,
+                     out=out, g=d.g, beta=d.beta)
