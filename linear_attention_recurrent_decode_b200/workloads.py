@@ -171,6 +171,7 @@ CONFIGS = {
     "n1_t1_hv8": dict(N=1, T=1, HV=8, num_slots=1),
     "n32_t1_hv8": dict(N=32, T=1, HV=8, num_slots=64),
     "n32_t1_hv16_gated": dict(N=32, T=1, HV=16, num_slots=128, gated=True),
+    "n32_t1_hv16": dict(N=32, T=1, HV=16, num_slots=128),  # the gated workload without the norm
     "n1_t4_hv8": dict(N=1, T=4, HV=8, num_slots=2),
     "n8_t4_hv8": dict(N=8, T=4, HV=8, num_slots=16),
     "n32_t4_hv8": dict(N=32, T=4, HV=8, num_slots=64),

@@ -564,3 +564,29 @@ def test_host_step_rejects_views_outside_the_staging_buffer(cuda_device):
     with pytest.raises(ValueError):
         kda.HostStep(d.q, d.k, d.v, d.state, d.slot_idx, host_in=host_in, dev_in=dev_in, host_out=host_out,
                      out=out, g=d.g, beta=d.beta)
+
+
+@pytest.mark.parametrize("N,T,HV,K,V,gated,state,layout,form", [
+    # long token runs: many chunks, a ragged last chunk, every input form and pool format
+    (2, 37, 2, 128, 128, False, "fp32", "kv", "dense"),
+    (2, 37, 2, 128, 96, True, "fp32", "vk", "dense"),
+    (2, 33, 2, 64, 128, False, "bf16", "vk", "raw"),
+    (2, 23, 2, 256, 64, True, "bf16", "kv", "raw"),
+    (3, 13, 2, 128, 128, True, "fp32", "vk", "raw"),
+    (2, 29, 3, 256, 128, False, "fp32", "vk", "dense"),
+])
+def test_long_token_runs_every_form(N, T, HV, K, V, gated, state, layout, form, cuda_device):
+    """T up to 37 tokens in one call (ten chunks of four with a ragged tail),
+    across pool dtypes, pool layouts and input forms, against the oracle."""
+    w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 2, gated=gated, seed=80 + T + K,
+                       state_dtype=state, inactive=1 if N > 2 else 0, serving=form == "raw", packed=False,
+                       decay="uniform")
+    d = w.to(cuda_device)
+    before = d.state.clone()
+    pool = d.state.clone() if layout == "kv" else d.state.transpose(-1, -2).contiguous()
+    o = _vk_call(w, d, pool, layout, form)
+    torch.cuda.synchronize()
+    if form == "raw":
+        g, beta = oracle.activate(w.raw.raw_gate, w.raw.A_log, w.raw.dt_bias, w.raw.raw_beta)
+        w = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
+    assert_parity(w, o, pool if layout == "kv" else pool.transpose(-1, -2), before)
