@@ -940,7 +940,7 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
 
   for (int64_t c0 = 0; c0 < p.T; c0 += kChunk) {
     const int64_t left = p.T - c0;
-    const int tc = static_cast<int>(left < kChunk ? left : kChunk);
+    const int tc_rt = static_cast<int>(left < kChunk ? left : kChunk);
     const int cb = static_cast<int>((c0 / kChunk) & 1);
     __syncthreads();  // every thread is done with the previous chunk's coefficients
     if (c0 + kChunk < p.T) {  // prefetch the next chunk into the other buffer
@@ -953,119 +953,131 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
       cp_async_wait<0>();
     }
     __syncthreads();
-    [[maybe_unused]] float neg_a = 0.f, raw_beta = 0.f, dt_bias[rows_per_thread(K)];
-    if constexpr (RAW) {
-      neg_a = -expf(__ldg(p.A_log + h));
+    // The chunk's work, with the token count a compile-time 4 for full chunks
+    // (no per-token guards) and a run-time count for the ragged last one.  On
+    // B200 the full-chunk copy speeds up the bf16-pool and [V, K] kernels (4 %,
+    // 5 % at N = 32, T = 4) but makes the fp32 [K, V] kernel spill (5 %
+    // slower), which therefore keeps the run-time count only.
+    auto process = [&](auto tc_const) {
+      constexpr int kTC = decltype(tc_const)::value;
+      const int tc = kTC ? kTC : tc_rt;
+      [[maybe_unused]] float neg_a = 0.f, raw_beta = 0.f, dt_bias[rows_per_thread(K)];
+      if constexpr (RAW) {
+        neg_a = -expf(__ldg(p.A_log + h));
 #pragma unroll
-      for (int jr = 0; jr < rows_per_thread(K); ++jr) {
-        const int r = threadIdx.x + jr * kThreads;
-        dt_bias[jr] = r < K ? __ldg(p.dt_bias + h * K + r) : 0.f;
+        for (int jr = 0; jr < rows_per_thread(K); ++jr) {
+          const int r = threadIdx.x + jr * kThreads;
+          dt_bias[jr] = r < K ? __ldg(p.dt_bias + h * K + r) : 0.f;
+        }
+        raw_beta = threadIdx.x < tc ? __bfloat162float(p.raw_beta[(n * p.T + c0 + threadIdx.x) * p.b_rs + h]) : 0.f;
       }
-      raw_beta = threadIdx.x < tc ? __bfloat162float(p.raw_beta[(n * p.T + c0 + threadIdx.x) * p.b_rs + h]) : 0.f;
-    }
-    chunk_prep<K, RAW>(cf, mp_part, tok[cb], tc, warp, lane, neg_a, dt_bias, raw_beta);
-    __syncthreads();
+      chunk_prep<K, RAW>(cf, mp_part, tok[cb], tc, warp, lane, neg_a, dt_bias, raw_beta);
+      __syncthreads();
 
-    chunk_pass<RPT, K>(s, cf.kt, redR, r0, warp, lane, rg, cq);
-    chunk_pass<RPT, K>(s, cf.qt, redQ, r0, warp, lane, rg, cq);
-    if (threadIdx.x < kNumMP) {
-      float tot = 0.f;
+      chunk_pass<RPT, K>(s, cf.kt, redR, r0, warp, lane, rg, cq);
+      chunk_pass<RPT, K>(s, cf.qt, redQ, r0, warp, lane, rg, cq);
+      if (threadIdx.x < kNumMP) {
+        float tot = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) tot += mp_part[w][threadIdx.x];
-      mp_tot[threadIdx.x] = tot;
-    }
-    __syncthreads();
+        for (int w = 0; w < kWarps; ++w) tot += mp_part[w][threadIdx.x];
+        mp_tot[threadIdx.x] = tot;
+      }
+      __syncthreads();
 
-    // Per token, in order: each lane solves one column of its quad (column
-    // 4cq + rg), the 32 lanes of warp 0 read out the tile's 32 columns, and
-    // the quad's four u values are then gathered by shuffles for the write.
-    const int jc = rg;
-    float uu[kChunk];
+      // Per token, in order: each lane solves one column of its quad (column
+      // 4cq + rg), the 32 lanes of warp 0 read out the tile's 32 columns, and
+      // the quad's four u values are then gathered by shuffles for the write.
+      const int jc = rg;
+      float uu[kChunk];
 #pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      uu[t] = 0.f;
-      if (t < tc) {
-        const TokenSmem<K>& raw = tok[cb][t];
-        float R = 0.f;
+      for (int t = 0; t < kChunk; ++t) {
+        uu[t] = 0.f;
+        if (t < tc) {
+          const TokenSmem<K>& raw = tok[cb][t];
+          float R = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) R += reinterpret_cast<const float*>(&redR[w][t][cq])[jc];
-        float x = __bfloat162float(raw.v[4 * cq + jc]) - R;
+          for (int w = 0; w < kWarps; ++w) R += reinterpret_cast<const float*>(&redR[w][t][cq])[jc];
+          float x = __bfloat162float(raw.v[4 * cq + jc]) - R;
 #pragma unroll
-        for (int sj = 0; sj < t; ++sj) x = fmaf(-mp_tot[m_index(t, sj)], uu[sj], x);
-        uu[t] = raw.beta[0] * x;
+          for (int sj = 0; sj < t; ++sj) x = fmaf(-mp_tot[m_index(t, sj)], uu[sj], x);
+          uu[t] = raw.beta[0] * x;
+          if (warp == 0) {
+            float o = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) o += reinterpret_cast<const float*>(&redQ[w][t][cq])[jc];
+#pragma unroll
+            for (int sj = 0; sj <= t; ++sj) o = fmaf(mp_tot[p_index(t, sj)], uu[sj], o);
+            o *= p.scale;
+            if constexpr (GATED) {
+              osm[t][4 * cq + jc] = o;  // until the chunk's exchange
+            } else {
+              p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(o);
+            }
+          }
+        }
+      }
+      float2 u[kChunk][2];
+#pragma unroll
+      for (int t = 0; t < kChunk; ++t) {
+        const float a0 = __shfl_sync(0xffffffffu, uu[t], cq);
+        const float a1 = __shfl_sync(0xffffffffu, uu[t], kColQuads + cq);
+        const float a2 = __shfl_sync(0xffffffffu, uu[t], 2 * kColQuads + cq);
+        const float a3 = __shfl_sync(0xffffffffu, uu[t], 3 * kColQuads + cq);
+        u[t][0] = make_float2(a0, a1);
+        u[t][1] = make_float2(a2, a3);
+      }
+
+      // chunk-end state: S = A_last S0 + sum_t c_t u_t^T
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const float4 c = cf.c[r0 + i];
+        const float2 a2 = f2(cf.a[r0 + i]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float2 x = __fmul2_rn(a2, s[i][j]);
+          x = __ffma2_rn(f2(c.x), u[0][j], x);
+          x = __ffma2_rn(f2(c.y), u[1][j], x);
+          x = __ffma2_rn(f2(c.z), u[2][j], x);
+          s[i][j] = __ffma2_rn(f2(c.w), u[3][j], x);
+        }
+      }
+
+      if constexpr (GATED) {
+        // one cluster exchange for the whole chunk's per-token sums of o^2
+        if (c0 == 0) cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
         if (warp == 0) {
-          float o = 0.f;
 #pragma unroll
-          for (int w = 0; w < kWarps; ++w) o += reinterpret_cast<const float*>(&redQ[w][t][cq])[jc];
+          for (int t = 0; t < kChunk; ++t) {
+            if (t < tc) {
+              const float o = osm[t][4 * cq + jc];
+              float ss = o * o;
 #pragma unroll
-          for (int sj = 0; sj <= t; ++sj) o = fmaf(mp_tot[p_index(t, sj)], uu[sj], o);
-          o *= p.scale;
-          if constexpr (GATED) {
-            osm[t][4 * cq + jc] = o;  // until the chunk's exchange
-          } else {
-            p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(o);
+              for (int m = 1; m < 32; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+              if (lane < tiles)
+                cluster_store_f32(cluster_map(smem_u32(&nrm[cb][t][tile]), static_cast<uint32_t>(lane)), ss);
+            }
+          }
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();
+        if (warp == 0) {
+#pragma unroll
+          for (int t = 0; t < kChunk; ++t) {
+            if (t < tc) {
+              float tot = 0.f;
+              for (int r = 0; r < tiles; ++r) tot += nrm[cb][t][r];
+              const float inv = rsqrtf(tot / static_cast<float>(V) + p.eps);
+              const float z = __bfloat162float(tok[cb][t].z[4 * cq + jc]);
+              const float y = osm[t][4 * cq + jc] * inv * wj * (1.0f / (1.0f + __expf(-z)));
+              p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(y);
+            }
           }
         }
       }
-    }
-    float2 u[kChunk][2];
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      const float a0 = __shfl_sync(0xffffffffu, uu[t], cq);
-      const float a1 = __shfl_sync(0xffffffffu, uu[t], kColQuads + cq);
-      const float a2 = __shfl_sync(0xffffffffu, uu[t], 2 * kColQuads + cq);
-      const float a3 = __shfl_sync(0xffffffffu, uu[t], 3 * kColQuads + cq);
-      u[t][0] = make_float2(a0, a1);
-      u[t][1] = make_float2(a2, a3);
-    }
-
-    // chunk-end state: S = A_last S0 + sum_t c_t u_t^T
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-      const float4 c = cf.c[r0 + i];
-      const float2 a2 = f2(cf.a[r0 + i]);
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float2 x = __fmul2_rn(a2, s[i][j]);
-        x = __ffma2_rn(f2(c.x), u[0][j], x);
-        x = __ffma2_rn(f2(c.y), u[1][j], x);
-        x = __ffma2_rn(f2(c.z), u[2][j], x);
-        s[i][j] = __ffma2_rn(f2(c.w), u[3][j], x);
-      }
-    }
-
-    if constexpr (GATED) {
-      // one cluster exchange for the whole chunk's per-token sums of o^2
-      if (c0 == 0) cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
-      if (warp == 0) {
-#pragma unroll
-        for (int t = 0; t < kChunk; ++t) {
-          if (t < tc) {
-            const float o = osm[t][4 * cq + jc];
-            float ss = o * o;
-#pragma unroll
-            for (int m = 1; m < 32; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-            if (lane < tiles)
-              cluster_store_f32(cluster_map(smem_u32(&nrm[cb][t][tile]), static_cast<uint32_t>(lane)), ss);
-          }
-        }
-      }
-      cluster_arrive_release();
-      cluster_wait_acquire();
-      if (warp == 0) {
-#pragma unroll
-        for (int t = 0; t < kChunk; ++t) {
-          if (t < tc) {
-            float tot = 0.f;
-            for (int r = 0; r < tiles; ++r) tot += nrm[cb][t][r];
-            const float inv = rsqrtf(tot / static_cast<float>(V) + p.eps);
-            const float z = __bfloat162float(tok[cb][t].z[4 * cq + jc]);
-            const float y = osm[t][4 * cq + jc] * inv * wj * (1.0f / (1.0f + __expf(-z)));
-            p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(y);
-          }
-        }
-      }
-    }
+    };
+    constexpr bool kFullChunkCopy = sizeof(ST) == 2 || VK;
+    if (kFullChunkCopy && tc_rt == kChunk) process(std::integral_constant<int, kFullChunkCopy ? kChunk : 0>{});
+    else process(std::integral_constant<int, 0>{});
   }
 
   allow_next_grid();
