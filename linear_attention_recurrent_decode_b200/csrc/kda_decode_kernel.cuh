@@ -914,10 +914,19 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
 
   // Token inputs do not depend on the slot: stage the first chunk before it lands.
   stage_tokens<K, GATED, IN>(tok[0], p, V, n, h, col0, 0, static_cast<int>(p.T < kChunk ? p.T : kChunk));
+  // Serving form: dt_bias[h, :] and A_log[h] staged with the first chunk, and
+  // the raw bf16 beta of the chunk's tokens kept as bits until the prep: all
+  // issued ahead of the state loads, none waited on before the prep.
+  __shared__ __align__(16) float dtb_s[RAW ? K + 4 : 4];  // dt_bias[h, :], then A_log[h]
+  [[maybe_unused]] uint32_t rb_bits = 0;
+  if constexpr (RAW) {
+    for (int c = threadIdx.x; c < K / 4; c += kThreads) cp_async16(smem_u32(&dtb_s[4 * c]), p.dt_bias + h * K + 4 * c);
+    if (threadIdx.x == 0) cp_async4(smem_u32(&dtb_s[K]), p.A_log + h);
+    if (threadIdx.x < p.T && threadIdx.x < kChunk)
+      rb_bits = __ldg(reinterpret_cast<const unsigned short*>(p.raw_beta) + (n * p.T + threadIdx.x) * p.b_rs + h);
+  }
   cp_async_commit();
-  // The norm weight, also ahead of the state loads.  (The serving-form scalars
-  // are loaded per chunk, right before the prep: loading them here, ahead of
-  // the state, measured 5 % slower at N = 32, T = 4.)
+  // The norm weight, also ahead of the state loads.
   [[maybe_unused]] float wj = 0.f;  // gated: norm weight of this lane's solve column (warp 0)
   if constexpr (GATED) {
     if (warp == 0) wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + rg]);
@@ -963,15 +972,21 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
       const int tc = kTC ? kTC : tc_rt;
       [[maybe_unused]] float neg_a = 0.f, raw_beta = 0.f, dt_bias[rows_per_thread(K)];
       if constexpr (RAW) {
-        neg_a = -expf(__ldg(p.A_log + h));
+        neg_a = -expf(dtb_s[K]);
 #pragma unroll
         for (int jr = 0; jr < rows_per_thread(K); ++jr) {
           const int r = threadIdx.x + jr * kThreads;
-          dt_bias[jr] = r < K ? __ldg(p.dt_bias + h * K + r) : 0.f;
+          dt_bias[jr] = r < K ? dtb_s[r] : 0.f;
         }
-        raw_beta = threadIdx.x < tc ? __bfloat162float(p.raw_beta[(n * p.T + c0 + threadIdx.x) * p.b_rs + h]) : 0.f;
+        raw_beta = __uint_as_float(rb_bits << 16);
       }
       chunk_prep<K, RAW>(cf, mp_part, tok[cb], tc, warp, lane, neg_a, dt_bias, raw_beta);
+      if constexpr (RAW) {  // the next chunk's raw beta bits, consumed by the next prep
+        const int64_t tn = c0 + kChunk + threadIdx.x;
+        rb_bits = 0;
+        if (threadIdx.x < kChunk && tn < p.T)
+          rb_bits = __ldg(reinterpret_cast<const unsigned short*>(p.raw_beta) + (n * p.T + tn) * p.b_rs + h);
+      }
       __syncthreads();
 
       chunk_pass<RPT, K>(s, cf.kt, redR, r0, warp, lane, rg, cq);
