@@ -4,8 +4,9 @@
 // Host side only: argument validation, a per-device compute-capability cache
 // (queried once per device, as the FlashInfer #4562 review of `CheckTarget`
 // asks for a latency-sensitive decode path), and one kernel launch on the
-// caller's stream.  Nothing here allocates, synchronises or falls back to
-// another implementation.
+// caller's stream (kda_decode_host adds the copies in and out around it).
+// Nothing here allocates, synchronises or falls back to another
+// implementation.
 #include <atomic>
 #include <cstddef>
 #include <cstdint>

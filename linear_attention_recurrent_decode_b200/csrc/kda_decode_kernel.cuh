@@ -5,7 +5,10 @@
 //   1. reads slot_idx[n] and issues every 128-bit load of its K x 32 state tile
 //      at once (8..32 KiB in flight per CTA), straight into registers: the tile
 //      is touched exactly once, so staging it in shared memory would only add
-//      a copy (a bulk-TMA staging of the same tile measured no faster on B200);
+//      a copy (a bulk-TMA staging of the same tile measured no faster on B200).
+//      A pool with [V][K] blocks (K contiguous) is the exception: its tile
+//      moves through shared memory so that global accesses stay whole-line
+//      (TileIO below);
 //   2. for each token: decays its rows by exp(g), forms the two reductions
 //      S'^T k and S'^T q over K (in-thread over its rows, a reduce-scatter of
 //      warp shuffles across the 4 row groups of a warp, shared memory across
