@@ -307,6 +307,20 @@ def run_ours(args):
     ms_max = reduce_max(ms_rank, dev)
     del g_full, g_rem
 
+    # the same calls launched one at a time from Python (no graph): what an
+    # eager caller sees, host launch cost included
+    n_eager = min(args.steps, 20_000)
+    torch.cuda.synchronize()
+    ea = torch.cuda.Event(enable_timing=True)
+    eb = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ea.record(stream)
+        for i in range(n_eager):
+            calls[i % R]()
+        eb.record(stream)
+    torch.cuda.synchronize()
+    eager_us = reduce_max(ea.elapsed_time(eb), dev) * 1e3 / n_eager
+
     # end to end through the public API: pinned host inputs in, output back out
     e2e = run_e2e(kda, base, dev, stream, min(args.steps, args.e2e_steps), world)
     floor = None if args.no_floor else copy_floor(base, dev, stream, R, min(args.steps, 20_000))
@@ -345,6 +359,9 @@ def run_ours(args):
                      "traffic": profiled_traffic(args.config)},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "eager": {"value": round(eager_us, 3), "unit": UNIT, "steps": n_eager,
+                  "how": "the same calls on the same rotating replicas, launched one at a time from "
+                         "Python (no CUDA graph)"},
         "clocks": clocks,
         "floor": floor,
         "gpu_launches": args.steps,
