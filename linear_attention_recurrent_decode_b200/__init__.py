@@ -22,6 +22,8 @@ import math
 import os
 import threading
 
+import torch
+
 __all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_STATE_FP32", "KDA_STATE_BF16",
@@ -92,6 +94,9 @@ class KdaError(RuntimeError):
 def library() -> ctypes.CDLL:
     """The loaded C-ABI library (raises if it has not been built)."""
     global _lib
+    lib = _lib
+    if lib is not None:  # loaded: no lock on the per-call path
+        return lib
     with _lock:
         if _lib is None:
             if not os.path.exists(LIBRARY_PATH):
@@ -112,16 +117,19 @@ def status_string(status: int) -> str:
 
 
 def _stream_handle(stream):
-    import torch
-
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
 def _check(t, name, dtype, shape=None):
-    import torch
+    # one combined test on the per-call path; the detailed reason only on failure
+    if (not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda or not t.is_contiguous()
+            or (shape is not None and t.shape != shape)):
+        _check_failed(t, name, dtype, shape)
 
+
+def _check_failed(t, name, dtype, shape):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
@@ -130,13 +138,10 @@ def _check(t, name, dtype, shape=None):
         raise ValueError(f"{name} must be on a CUDA device")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if shape is not None and tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
 def _common(q, k, v, g, beta, state_pool, slot_idx, out):
-    import torch
-
     if q.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be [N, T, HV, K|V]")
     N, T, HV, K = q.shape
@@ -164,8 +169,6 @@ def kda_decode(q, k, v, g, beta, state_pool, slot_idx, out=None, scale: float | 
     place and returns ``out`` (allocated if not given).  ``scale`` defaults to
     1/sqrt(K).  A bf16 ``state_pool`` runs the bf16-state entry point (fp32
     math, state rounded to bf16 once per call)."""
-    import torch
-
     N, T, HV, K, V, out = _common(q, k, v, g, beta, state_pool, slot_idx, out)
     if scale is None:
         scale = 1.0 / math.sqrt(K)
@@ -182,8 +185,6 @@ def kda_decode_gated_rmsnorm(q, k, v, g, beta, state_pool, slot_idx, gate, norm_
                              eps: float = 1e-6, out=None, scale: float | None = None, stream=None):
     """Decode step fused with the gated RMS norm over V:
     out = bf16(o / sqrt(mean(o^2) + eps) * norm_weight * sigmoid(gate))."""
-    import torch
-
     N, T, HV, K, V, out = _common(q, k, v, g, beta, state_pool, slot_idx, out)
     _check(gate, "gate", torch.bfloat16, (N, T, HV, V))
     _check(norm_weight, "norm_weight", torch.bfloat16, (V,))
@@ -203,8 +204,6 @@ def kda_decode_gated_rmsnorm(q, k, v, g, beta, state_pool, slot_idx, gate, norm_
 def _rows(t, name, dtype, N, T, inner):
     """Validate a [N, T, ...inner] view whose (n, t) rows are uniformly strided and
     whose per-row part is dense; return its row stride in elements (0 for None)."""
-    import torch
-
     if t is None:
         return 0
     if not isinstance(t, torch.Tensor) or t.dtype != dtype:
@@ -228,8 +227,6 @@ def _ex_args(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None,
                   dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
                   scale: float | None = None, state_layout: str = "kv"):
     """The kda_decode_args of a call (and its output tensor); see kda_decode_ex."""
-    import torch
-
     N, T, HV, K = q.shape
     V = v.shape[-1]
     bf, f32 = torch.bfloat16, torch.float32
@@ -309,7 +306,6 @@ class HostStep:
     """
 
     def __init__(self, q, k, v, state_pool, slot_idx, *, host_in, dev_in, host_out, out, stream=None, **kw):
-        import torch
 
         for name, t in (("host_in", host_in), ("host_out", host_out)):
             if t.is_cuda or not t.is_pinned():
