@@ -89,3 +89,21 @@ def test_regrouping_check_sees_a_wrong_coupling():
     wrong_o3 = w.scale * ((A[3] * q[3]) @ S0 + sum(np.sum(k[s] * np.prod(d[s + 1:4], axis=0) * q[3]) * u[s]
                                                    for s in range(4)))
     assert not np.allclose(wrong_o3, ref_out[0, 3, 0], rtol=1e-6)
+
+
+def test_one_pass_readout_identity():
+    """The one-token kernel reads out o = scale (S'^T q + (q . k) u) from the
+    decayed state S' and the correction u, without a second pass over the
+    updated state; in fp64 this equals the oracle's scale S^T q."""
+    w = workloads.make(N=3, T=1, HV=2, K=32, V=16, num_slots=4, seed=77)
+    ref_out, ref_state = oracle.kda_decode_ref(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx, w.scale)
+    for n in range(w.N):
+        slot = int(w.slot_idx[n])
+        for h in range(w.HV):
+            q, k, v = (x.double().numpy()[n, 0, h] for x in (w.q, w.k, w.v))
+            g, beta = w.g.double().numpy()[n, 0, h], float(w.beta[n, 0, h])
+            Sd = np.exp(g)[:, None] * w.state.double().numpy()[slot, h]     # S'
+            u = beta * (v - Sd.T @ k)
+            o = w.scale * (Sd.T @ q + float(q @ k) * u)
+            np.testing.assert_allclose(o, ref_out[n, 0, h], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(Sd + np.outer(k, u), ref_state[slot, h], rtol=1e-12, atol=1e-14)
