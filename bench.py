@@ -488,9 +488,10 @@ def run_reference(args):
     pool = w.state_kv().double().numpy().copy()
     kw = dict(gate=w.gate, norm_weight=w.norm_weight, eps=w.eps) if w.gated else dict(eps=w.eps)
 
+    g, beta = _oracle_gate(oracle, w)  # the serving form's activation, once
+
     def one(lo, hi, thr):
         t0 = time.perf_counter()
-        g, beta = _oracle_gate(oracle, w)
         oracle.kda_decode_ref(w.q, w.k, w.v, g, beta, None, w.slot_idx, w.scale, threads=thr,
                               units=(lo, hi), state_inplace=pool, **kw)
         return time.perf_counter() - t0
@@ -501,8 +502,15 @@ def run_reference(args):
     if total * t_full <= budget:
         per_step, thr = units, threads
     else:
-        per_step = max(1, min(units, int(units * budget / (total * t_full))))
-        thr = max(1, min(threads, per_step))
+        # Bounded samples: single-threaded (no per-call thread start-up), as
+        # many (n, h) units per step as the budget allows given the measured
+        # fixed cost of a call and cost of a unit.
+        t1 = min(one(0, 1, 1) for _ in range(3))
+        t8 = min(one(0, min(8, units), 1) for _ in range(3))
+        t_unit = max((t8 - t1) / max(1, min(8, units) - 1), 1e-7)
+        overhead = max(t1 - t_unit, 0.0)
+        per_step = int(max(1, min(units, (budget / total - overhead) / t_unit)))
+        thr = 1
     times = []
     lo = 0
     for i in range(total):
@@ -512,7 +520,8 @@ def run_reference(args):
             times.append(dt * units / (hi - lo))
         lo = 0 if hi >= units else hi
     us = statistics.mean(times) * 1e6
-    sample = (f"each step: units [{per_step} of {units}] (n,h) of {args.config}, scaled to a full call"
+    sample = (f"each step: {per_step} of the {units} (n,h) units of {args.config}, single-threaded, "
+              f"scaled to a full call (the run is bounded to about {budget:.0f} s)"
               if per_step < units else f"each step: one full call of {args.config}")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world,
