@@ -18,9 +18,12 @@ Parity status of each entry point (what pins it, see ``tests/test_oracle_pins.py
   * ``round_bf16`` (bf16 state write-back) -- pinned by the format's definition
                                              and torch's conversion.
   * ``activate`` (raw gate / raw beta)  -- PARITY UNPINNED by the sources: no page
-                                             prints the activation; the code is pinned
-                                             only against library routines for the
-                                             formula it takes as its reading.
+                                             prints the activation.  The tests pin only
+                                             properties every softplus-style gate and
+                                             logistic beta has (g <= 0, monotone in the
+                                             raw gate, its two limits, the dt_bias shift;
+                                             beta in (0,1), increasing, symmetric), not
+                                             the formula taken as the reading.
 """
 from __future__ import annotations
 

@@ -216,9 +216,10 @@ void kda_oracle_round_bf16(const double *in, uint16_t *out, int64_t n)
  * FlashInfer #4562's kernel launch takes raw_gate, raw_beta, A_log and
  * dt_bias and b12x #249 takes raw_g and raw_beta, but neither page prints the
  * activation: this formula is a reading (the usual one for KDA's gate), not
- * something the pages fix -- parity unpinned by the sources (its steps are
- * pinned against library routines in the tests).  softplus(x) = log(1 + e^x), evaluated as
- * x + log1p(e^-x) for x > 0 so that it neither overflows nor cancels.
+ * something the pages fix -- parity unpinned by the sources (the tests pin
+ * only properties any softplus-style gate and logistic beta share).
+ * softplus(x) = log(1 + e^x), evaluated as x + log1p(e^-x) for x > 0 so that
+ * it neither overflows nor cancels.
  * Layouts: raw_gate bf16 [N*T, HV*K], raw_beta bf16 [N*T, HV] (dense),
  * A_log [HV], dt_bias [HV*K]; outputs g [N*T, HV*K], beta [N*T, HV].
  */

@@ -374,23 +374,72 @@ def test_bf16_state_closed_forms():
 
 
 # ---------------------------------------------------------------------------
-# raw gate / raw beta activation (a reading: the sources name the inputs but
-# print no formula; pinned here only against library routines for that formula)
+# raw gate / raw beta activation.  PARITY UNPINNED: the sources name the raw
+# inputs (FlashInfer #4562's kernel launch passes raw_gate, A_log, dt_bias and
+# raw_beta) but print no activation, so the formula the oracle uses is a
+# reading.  What can be pinned without repeating that formula are properties
+# any softplus-style decay gate and logistic beta must have; each slip the
+# mutation tests plant in the activation breaks one of them.
 # ---------------------------------------------------------------------------
-def test_activation_matches_library_routines():
-    rng = np.random.default_rng(11)
-    N, T, HV, K = 2, 3, 4, 8
-    raw_gate = bf16(rng.standard_normal((N, T, HV, K)) * 4)
-    raw_gate[0, 0, 0, :4] = bf16([80.0, -80.0, 0.0, 30.0])
-    raw_beta = bf16(rng.standard_normal((N, T, HV)) * 3)
-    A_log = torch.as_tensor(rng.standard_normal(HV), dtype=torch.float32)
-    dt_bias = torch.as_tensor(rng.standard_normal((HV, K)), dtype=torch.float32)
-    g, beta = oracle.activate(raw_gate, A_log, dt_bias, raw_beta)
-    x = bf16_vals(raw_gate) + dt_bias.double().numpy()[None, None]
-    g_ref = -np.exp(A_log.double().numpy())[None, None, :, None] * np.logaddexp(0.0, x)
-    np.testing.assert_allclose(g, g_ref, rtol=1e-14, atol=0)
-    np.testing.assert_allclose(beta, expit(bf16_vals(raw_beta)), rtol=1e-14, atol=0)
-    assert np.all(g <= 0) and np.all(np.isfinite(g))
+def _activate_1head(raw, A_log=0.3, dt_bias=0.0, raw_beta=None):
+    """Activate a 1-D sweep of raw gate values (one head, K = len(raw))."""
+    raw = np.asarray(raw, dtype=np.float64)
+    K = raw.size
+    rb = np.zeros(1) if raw_beta is None else np.asarray(raw_beta, dtype=np.float64)
+    g, beta = oracle.activate(bf16_exact(raw.reshape(1, 1, 1, K)), torch.tensor([A_log], dtype=torch.float32),
+                              torch.full((1, K), dt_bias, dtype=torch.float32), bf16_exact(rb.reshape(1, 1, 1)))
+    return g.reshape(K), float(beta.reshape(-1)[0])
+
+
+def _bf16_grid(lo, hi, n):
+    return np.unique(bf16(np.linspace(lo, hi, n)).float().numpy().astype(np.float64))
+
+
+def test_activation_gate_is_a_nonpositive_nonincreasing_log_decay():
+    """g <= 0 (a decay exp(g) never amplifies the state) and g does not
+    increase as the raw gate grows (a larger raw gate forgets more)."""
+    x = _bf16_grid(-60.0, 60.0, 4001)
+    for A_log in (-2.0, 0.0, 1.5):
+        g, _ = _activate_1head(x, A_log=A_log)
+        assert np.all(np.isfinite(g)) and np.all(g <= 0.0)
+        assert np.all(np.diff(g) <= 0.0)
+        assert g[-1] < g[0]  # strictly forgets more at the top of the range
+
+
+def test_activation_gate_limits():
+    """raw gate -> -inf: g -> 0 (no decay); raw gate -> +inf: g is linear with
+    slope -exp(A_log) (the rate per unit of raw gate is the head's A)."""
+    for A_log in (-1.0, 0.0, 2.0):
+        a = math.exp(float(np.float32(A_log)))
+        g, _ = _activate_1head([-80.0, -60.0, 40.0, 64.0], A_log=A_log)
+        assert abs(g[0]) < 1e-30 and abs(g[1]) < 1e-20
+        slope = (g[3] - g[2]) / (64.0 - 40.0)
+        assert slope == pytest.approx(-a, rel=1e-12)
+        assert g[3] == pytest.approx(-a * 64.0, rel=1e-12)
+
+
+def test_activation_dt_bias_shifts_the_raw_gate():
+    """dt_bias adds to the raw gate before the nonlinearity: raw + b with bias 0
+    equals raw with bias b (values chosen so raw + b is exact in bf16)."""
+    raw = np.array([-3.0, -1.0, -0.5, 0.0, 0.25, 1.0, 2.0, 6.0])
+    for b in (-1.5, 0.5, 2.0):
+        shifted, _ = _activate_1head(raw + b, A_log=0.7, dt_bias=0.0)
+        biased, _ = _activate_1head(raw, A_log=0.7, dt_bias=b)
+        np.testing.assert_array_equal(biased, shifted)
+
+
+def test_activation_beta_is_a_logistic_gate():
+    """beta in (0, 1), increasing in the raw beta, beta(0) = 1/2 and
+    beta(-x) = 1 - beta(x)."""
+    xs = _bf16_grid(-12.0, 12.0, 97)
+    betas = np.array([_activate_1head([0.0], raw_beta=[x])[1] for x in xs])
+    assert np.all(betas > 0.0) and np.all(betas < 1.0)
+    assert np.all(np.diff(betas) > 0.0)
+    assert _activate_1head([0.0], raw_beta=[0.0])[1] == 0.5
+    for x in xs:
+        bp = _activate_1head([0.0], raw_beta=[x])[1]
+        bm = _activate_1head([0.0], raw_beta=[-x])[1]
+        assert bp + bm == pytest.approx(1.0, abs=1e-15)
 
 
 def test_activation_feeds_the_recurrence():

@@ -388,9 +388,11 @@ def test_ex_packed_mixed_qkv_and_strided_gate(T, gated, state, cuda_device):
     (3, 1, 2, 256, 64, False, "bf16"),
     (2, 5, 2, 128, 128, True, "bf16"),
 ])
-def test_ex_raw_gate_form(N, T, HV, K, V, gated, state, cuda_device):
+def test_ex_raw_gate_form_against_the_reading(N, T, HV, K, V, gated, state, cuda_device):
     """Raw gate / beta activated in the kernel, inputs packed like mixed_qkv;
-    against the oracle's activation feeding its recurrence."""
+    against the oracle's activation feeding its recurrence.  The activation
+    formula is a reading no page prints (parity unpinned): this checks the
+    kernel against that reading, not against the pages."""
     w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 3, gated=gated, seed=50 + N + T,
                        state_dtype=state, inactive=1 if N > 2 else 0)
     rg = workloads.raw_gate_inputs(N, T, HV, K, seed=51)
@@ -413,7 +415,9 @@ SERVING_CONFIGS = [n for n in workloads.CONFIGS if "_raw" in n or "_packed" in n
 def test_named_serving_workload_parity(name, cuda_device):
     """The packed, serving-form and [V, K]-pool workloads, called as the
     benchmark calls them (kda_decode_ex; q, k, v packed in one row buffer when
-    the workload says so; raw gate and beta, or activated ones)."""
+    the workload says so; raw gate and beta, or activated ones).  For the
+    ``*_raw*`` workloads the reference is the oracle's activation reading
+    (parity unpinned by the pages), not a formula the pages print."""
     w = workloads.config(name)
     d = w.to(cuda_device)
     q, k, v = d.q, d.k, d.v
@@ -484,7 +488,8 @@ def _vk_call(w, d, pool, layout, form):
 def test_vk_layout_parity(N, T, HV, K, V, gated, state, form, cuda_device):
     """[V, K] state blocks: against the oracle on the same state read as [K, V],
     and bit-identical to the [K, V] pool (the same arithmetic, another address
-    map)."""
+    map).  The ``raw`` cases check against the oracle's activation reading
+    (parity unpinned by the pages)."""
     w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 3, gated=gated, seed=70 + N + T + K,
                        state_dtype=state, inactive=1, serving=form == "raw", packed=False)
     d = w.to(cuda_device)
@@ -577,7 +582,9 @@ def test_host_step_rejects_views_outside_the_staging_buffer(cuda_device):
 ])
 def test_long_token_runs_every_form(N, T, HV, K, V, gated, state, layout, form, cuda_device):
     """T up to 37 tokens in one call (ten chunks of four with a ragged tail),
-    across pool dtypes, pool layouts and input forms, against the oracle."""
+    across pool dtypes, pool layouts and input forms, against the oracle (the
+    ``raw`` cases against its activation reading, parity unpinned by the
+    pages)."""
     w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 2, gated=gated, seed=80 + T + K,
                        state_dtype=state, inactive=1 if N > 2 else 0, serving=form == "raw", packed=False,
                        decay="uniform")
