@@ -5,12 +5,15 @@
 
 One step = one ``kda_decode`` call over one batch (default workload
 ``n32_t1_hv8``: N=32 sequences, T=1 token, HV=8 value heads, K=V=128, fp32
-state pool of 64 slots).  The timed region replays, from a CUDA graph, K calls
-that rotate over R independent replicas of the inputs and pool whose combined
-touched bytes exceed twice the L2 cache, so every call reads its state from
-HBM (the pages' cold-L2 graph-replay method).  Timing uses CUDA events on the
-launching stream with a device synchronize on both sides; under torchrun each
-rank runs its own batch (weak scaling, no collective on the data path) and the
+state pool of 64 slots).  A timed region replays, from CUDA graphs, exactly K
+calls that rotate over R independent replicas of the inputs and pool whose
+combined touched bytes exceed twice the L2 cache, so every call reads its state
+from HBM (the pages' cold-L2 graph-replay method).  The regions are enqueued
+behind an untimed pre-roll of replays with no host sync in between, so neither
+an idle GPU nor a graph-launch gap is counted; each region sits between CUDA
+events on the launching stream, the reported time is the median region, with a
+device synchronize on both sides of the whole run.  Under torchrun each rank
+runs its own batch (weak scaling, no collective on the data path) and the
 reported time is the maximum over ranks.
 
 Printed (rank 0, one JSON line): µs per call for the whole job, the achieved
@@ -227,6 +230,94 @@ def time_cpu_oracle(w, budget_s: float = 8.0, max_calls: int = 200):
     return statistics.median(times), threads, len(times)
 
 
+class GraphRegion:
+    """Exactly ``steps`` calls, rotating over the given callables (one per
+    replica), timed on the device from CUDA graphs.
+
+    Graphs: ``cycle`` (one call per replica, in order); the timed region (one
+    graph of ``steps`` calls when that is at most ``SINGLE_GRAPH_MAX``, else
+    ``cycle`` replayed steps // R times and a graph of the remainder); and
+    ``tail``, the rest of the cycle after the remainder, replayed untimed after
+    every region so that each region starts on replica 0 with every replica last
+    touched R calls earlier (inputs larger than L2 stay cold).
+
+    ``run`` enqueues, with no host synchronisation in between: a pre-roll of
+    ``cycle`` replays lasting about ``preroll_s`` (so the clocks are at load and
+    the first region starts on a busy stream, with no launch gap or idle GPU
+    counted), then ``repeats`` regions, each between two CUDA events on the
+    launching stream and followed by ``tail``.  Returns each region's
+    milliseconds.  ``repeats`` = 0 picks an odd count (1..9) that keeps the
+    regions to about a second in all."""
+
+    SINGLE_GRAPH_MAX = 4096
+
+    def __init__(self, calls, steps, stream, preroll_s, repeats):
+        import torch
+
+        self.stream = stream
+        R = len(calls)
+        rem = steps % R
+        self.cycle = self._capture(calls)
+        if steps <= self.SINGLE_GRAPH_MAX:
+            self.timed = [self._capture([calls[i % R] for i in range(steps)])]
+        else:
+            self.timed = [self.cycle] * (steps // R) + ([self._capture(calls[:rem])] if rem else [])
+        self.tail = self._capture(calls[rem:]) if rem else None
+        # upload every graph, then estimate the time of one cycle (all untimed)
+        with torch.cuda.stream(stream):
+            self.cycle.replay()
+            self.timed[0].replay()
+            self.timed[-1].replay()
+            if self.tail:
+                self.tail.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(3):
+                self.cycle.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        cycle_s = max(a.elapsed_time(b) / 3e3, 1e-6)
+        self.preroll = max(2, int(math.ceil(preroll_s / cycle_s)))
+        region_s = cycle_s * steps / R
+        if repeats <= 0:
+            repeats = max(1, min(9, int(1.0 / max(region_s, 1e-9))))
+            repeats -= (repeats + 1) % 2  # odd: the median is one of the regions
+        self.repeats = repeats
+
+    def _capture(self, fns):
+        import torch
+
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(self.stream):
+            with torch.cuda.graph(g, stream=self.stream):
+                for fn in fns:
+                    fn()
+        return g
+
+    def run(self):
+        import torch
+
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(self.repeats)]
+        with torch.cuda.stream(self.stream):
+            for _ in range(self.preroll):
+                self.cycle.replay()
+            for e0, e1 in ev:
+                e0.record(self.stream)
+                for g in self.timed:
+                    g.replay()
+                e1.record(self.stream)
+                if self.tail:
+                    self.tail.replay()
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    def release(self):
+        self.cycle = self.timed = self.tail = None
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -261,51 +352,23 @@ def run_ours(args):
             calls[i % R]()
     torch.cuda.synchronize()
 
-    # CUDA graphs: one of R calls (replayed) and one of the K mod R remainder
-    def capture(fns):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(g, stream=stream):
-                for fn in fns:
-                    fn()
-        return g
-
-    full, rem = divmod(args.steps, R)
-    g_full = capture(calls) if full else None
-    g_rem = capture(calls[:rem]) if rem else None
-    with torch.cuda.stream(stream):  # graph upload + one more untimed pass
-        if g_full:
-            g_full.replay()
-        if g_rem:
-            g_rem.replay()
-    torch.cuda.synchronize()
-
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    timer = GraphRegion(calls, args.steps, stream, args.preroll_ms / 1e3, args.repeats)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank) if (rank == 0 and not args.no_clocks) else None
     if sampler:
         sampler.__enter__()
-        time.sleep(0.25)
     t_wall0 = time.perf_counter()
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(full):
-            g_full.replay()
-        if g_rem:
-            g_rem.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    region_ms = timer.run()
     t_wall = time.perf_counter() - t_wall0
     if sampler:
         sampler.__exit__(None, None, None)
     if world > 1:
         dist.barrier()
-    ms_rank = e0.elapsed_time(e1)
+    ms_rank = statistics.median(region_ms)
     ms_max = reduce_max(ms_rank, dev)
-    del g_full, g_rem
+    timer.release()
 
     # the same calls launched one at a time from Python (no graph): what an
     # eager caller sees, host launch cost included
@@ -314,6 +377,8 @@ def run_ours(args):
     ea = torch.cuda.Event(enable_timing=True)
     eb = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        for i in range(min(R, 8)):  # untimed lead-in: the first event is recorded on a busy stream
+            calls[(n_eager + i) % R]()
         ea.record(stream)
         for i in range(n_eager):
             calls[i % R]()
@@ -323,7 +388,7 @@ def run_ours(args):
 
     # end to end through the public API: pinned host inputs in, output back out
     e2e = run_e2e(kda, base, dev, stream, min(args.steps, args.e2e_steps), world)
-    floor = None if args.no_floor else copy_floor(base, dev, stream, R, min(args.steps, 20_000))
+    floor = None if args.no_floor else copy_floor(base, dev, stream, R, args.steps, args.preroll_ms / 1e3)
 
     if world > 1:
         dist.barrier()
@@ -350,7 +415,11 @@ def run_ours(args):
                    "V": base.V, "num_slots": base.num_slots, "gated": base.gated,
                    "replicas": R, "l2": f"inputs larger than L2: {R} rotating replicas touch "
                    f"{R * (base.state_bytes_touched() + base.io_bytes()) / 1e6:.0f} MB > 2 x "
-                   f"{l2 / 1e6:.0f} MB L2", "timing": "CUDA graph replay, CUDA events",
+                   f"{l2 / 1e6:.0f} MB L2",
+                   "timing": f"CUDA graph replay, CUDA events on the launching stream: {timer.repeats} "
+                             f"regions of exactly {args.steps} calls behind a {timer.preroll}-replay "
+                             "untimed pre-roll, no host sync in between; value from the median region",
+                   "region_us_per_call": [round(x * 1e3 / args.steps, 4) for x in region_ms],
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "gbs": round(achieved, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -385,39 +454,23 @@ def _packed(tensors: dict, alloc):
     return buf, views
 
 
-def copy_floor(w, dev, stream, R, steps):
+def copy_floor(w, dev, stream, R, steps, preroll_s):
     """Per-call time of a plain in-place elementwise op (torch's x.mul_(c)) over
     exactly the state bytes one decode call reads and writes, with the same
-    rotation over R buffers and CUDA-graph replay: the practical floor for
-    moving those bytes once each way per call on this GPU."""
+    rotation over R buffers and the same graph-replay timing as the decode: the
+    practical floor for moving those bytes once each way per call on this GPU."""
     import torch
 
     n = w.state_bytes_touched() // 4
     bufs = [torch.randn(n, device=dev) for _ in range(R)]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        for b in bufs:
-            b.mul_(0.999)
-        torch.cuda.current_stream().synchronize()
-        with torch.cuda.graph(g, stream=stream):
-            for b in bufs:
-                b.mul_(1.0001)
-    reps = max(1, steps // R)
-    with torch.cuda.stream(stream):
-        g.replay()
+    fns = [(lambda b=b: b.mul_(1.0001)) for b in bufs]
+    timer = GraphRegion(fns, steps, stream, preroll_s, repeats=0)
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(reps):
-            g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / (reps * R)
-    del g
+    ms = statistics.median(timer.run())
+    timer.release()
+    us = ms * 1e3 / steps
     return {"what": "torch in-place x.mul_(c) over the same state bytes (read + write), same replica "
-                    "rotation and graph replay", "us_per_call": round(us, 3),
+                    "rotation and graph-replay timing", "us_per_call": round(us, 3),
             "bytes_per_call": 2 * n * 4, "gbs": round(2 * n * 4 / (us * 1e-6) / 1e9, 1)}
 
 
@@ -461,6 +514,8 @@ def run_e2e(kda, w, dev, stream, steps, world):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        for _ in range(4):  # untimed lead-in: the first event is recorded on a busy stream
+            step()
         e0.record(stream)
         for _ in range(steps):
             step()
@@ -551,6 +606,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-floor", action="store_true", help="skip the in-place copy-floor reference")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
+    ap.add_argument("--preroll-ms", type=float, default=300.0,
+                    help="untimed graph replays enqueued ahead of the timed regions")
+    ap.add_argument("--repeats", type=int, default=0,
+                    help="timed regions of --steps calls (0 = an odd count filling about a second)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

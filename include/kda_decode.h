@@ -59,8 +59,9 @@
  * once and caches it.
  *
  * Caller contract (checked only where noted):
- *   - active slots in slot_idx are distinct and < num_slots (the pool size is
- *     not an argument, so the library cannot check the upper bound);
+ *   - active slots in slot_idx are distinct and < num_slots (the fixed entry
+ *     points take no pool size and do not check the upper bound;
+ *     kda_decode_ex checks it when kda_decode_args.num_slots is set);
  *   - rows with slot_idx[n] < 0 get an all-zero output and do not touch the
  *     pool (CUDA-graph padding rows);
  *   - out overlaps no input and no part of the pool; the library rejects an
@@ -211,6 +212,22 @@ typedef struct {
     void *out;
     int64_t N, T, HV, K, V;
     float scale;
+    /*
+     * Checked slots.  num_slots = 0 leaves slot_idx unchecked (the caller
+     * contract above).  num_slots > 0 declares the pool's size: an active row
+     * whose slot_idx[n] >= num_slots is then treated as an inactive row (all-zero
+     * output, no pool access) and, when status is not NULL, the kernel stores 1
+     * to *status (device int32, 4-byte aligned, caller-owned; the library never
+     * clears it, so the caller zeroes it before the calls it wants to watch).
+     * FlashInfer #4562 (PR description) runs the step on an indexed, non-compact
+     * recurrent state: the slot table is data on the device that the host cannot
+     * validate before the launch, so the check is made by the kernel.  A checked
+     * call also lets the library see the pool's whole extent for its aliasing
+     * check.  Checked calls run the row-strided kernels (one integer compare per
+     * CTA); the fixed entry points are unchecked.
+     */
+    int64_t num_slots;
+    int32_t *status;
 } kda_decode_args;
 
 /*

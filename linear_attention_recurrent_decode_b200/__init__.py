@@ -59,6 +59,7 @@ class DecodeArgs(ctypes.Structure):
         ("out", _P),
         ("N", _I), ("T", _I), ("HV", _I), ("K", _I), ("V", _I),
         ("scale", _F),
+        ("num_slots", _I), ("status", _P),
     ]
 
 
@@ -117,25 +118,36 @@ def status_string(status: int) -> str:
 
 
 def _stream_handle(stream):
+    """The raw handle of ``stream`` (default: the current stream), which must
+    belong to the current device: the library launches on the current device."""
     if stream is None:
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    if hasattr(stream, "cuda_stream"):
+        if stream.device_index != torch.cuda.current_device():
+            raise ValueError(f"stream is on cuda:{stream.device_index}, the current device is "
+                             f"cuda:{torch.cuda.current_device()}")
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
 
 
-def _check(t, name, dtype, shape=None):
-    # one combined test on the per-call path; the detailed reason only on failure
+def _check(t, name, dtype, shape=None, device=None):
+    # one combined test on the per-call path; the detailed reason only on failure.
+    # ``device`` is the current device index: the library launches there, so a
+    # tensor on another GPU would be reached through peer addressing.
     if (not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda or not t.is_contiguous()
-            or (shape is not None and t.shape != shape)):
-        _check_failed(t, name, dtype, shape)
+            or (shape is not None and t.shape != shape) or (device is not None and t.get_device() != device)):
+        _check_failed(t, name, dtype, shape, device)
 
 
-def _check_failed(t, name, dtype, shape):
+def _check_failed(t, name, dtype, shape, device=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device")
+    if device is not None and t.get_device() != device:
+        raise ValueError(f"{name} is on cuda:{t.get_device()}, the current device is cuda:{device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
@@ -146,20 +158,21 @@ def _common(q, k, v, g, beta, state_pool, slot_idx, out):
         raise ValueError("q, k, v must be [N, T, HV, K|V]")
     N, T, HV, K = q.shape
     V = v.shape[-1]
-    _check(q, "q", torch.bfloat16)
-    _check(k, "k", torch.bfloat16, (N, T, HV, K))
-    _check(v, "v", torch.bfloat16, (N, T, HV, V))
-    _check(g, "g", torch.float32, (N, T, HV, K))
-    _check(beta, "beta", torch.float32, (N, T, HV))
-    _check(slot_idx, "slot_idx", torch.int32, (N,))
+    dev = torch.cuda.current_device() if q.is_cuda else None  # a CPU q is refused by _check
+    _check(q, "q", torch.bfloat16, None, dev)
+    _check(k, "k", torch.bfloat16, (N, T, HV, K), dev)
+    _check(v, "v", torch.bfloat16, (N, T, HV, V), dev)
+    _check(g, "g", torch.float32, (N, T, HV, K), dev)
+    _check(beta, "beta", torch.float32, (N, T, HV), dev)
+    _check(slot_idx, "slot_idx", torch.int32, (N,), dev)
     if state_pool.dtype not in (torch.float32, torch.bfloat16):
         raise TypeError(f"state_pool must be float32 or bfloat16, got {state_pool.dtype}")
-    _check(state_pool, "state_pool", state_pool.dtype)
+    _check(state_pool, "state_pool", state_pool.dtype, None, dev)
     if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (HV, K, V):
         raise ValueError(f"state_pool must be [num_slots, {HV}, {K}, {V}]")
     if out is None:
         out = torch.empty((N, T, HV, V), dtype=torch.bfloat16, device=q.device)
-    _check(out, "out", torch.bfloat16, (N, T, HV, V))
+    _check(out, "out", torch.bfloat16, (N, T, HV, V), dev)
     return N, T, HV, K, V, out
 
 
@@ -225,11 +238,19 @@ def _rows(t, name, dtype, N, T, inner):
 
 def _ex_args(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
                   dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
-                  scale: float | None = None, state_layout: str = "kv"):
+                  scale: float | None = None, state_layout: str = "kv", num_slots: int | None = None,
+                  status=None):
     """The kda_decode_args of a call (and its output tensor); see kda_decode_ex."""
     N, T, HV, K = q.shape
     V = v.shape[-1]
     bf, f32 = torch.bfloat16, torch.float32
+    dev = torch.cuda.current_device() if q.is_cuda else -1  # CPU tensors are refused below
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("raw_gate", raw_gate),
+                    ("A_log", A_log), ("dt_bias", dt_bias), ("raw_beta", raw_beta), ("state_pool", state_pool),
+                    ("slot_idx", slot_idx), ("gate", gate), ("norm_weight", norm_weight), ("out", out),
+                    ("status", status)):
+        if isinstance(t, torch.Tensor) and t.is_cuda and t.get_device() != dev:
+            raise ValueError(f"{name} is on cuda:{t.get_device()}, the current device is cuda:{dev}")
     a = DecodeArgs()
     a.q, a.q_row_stride = q.data_ptr(), _rows(q, "q", bf, N, T, (HV, K))
     a.k, a.k_row_stride = k.data_ptr(), _rows(k, "k", bf, N, T, (HV, K))
@@ -267,12 +288,21 @@ def _ex_args(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None,
     a.out = out.data_ptr()
     a.N, a.T, a.HV, a.K, a.V = N, T, HV, K, V
     a.scale = float(1.0 / math.sqrt(K) if scale is None else scale)
+    a.num_slots = int(state_pool.shape[0] if num_slots is None else num_slots)
+    if a.num_slots < 0 or a.num_slots > state_pool.shape[0]:
+        raise ValueError(f"num_slots must be in [0, {state_pool.shape[0]}] (0 = unchecked)")
+    if status is not None:
+        _check(status, "status", torch.int32, None, dev)
+        if status.numel() < 1:
+            raise ValueError("status must hold at least one int32")
+        a.status = status.data_ptr()
     return a, out
 
 
 def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=None, A_log=None,
                   dt_bias=None, raw_beta=None, gate=None, norm_weight=None, eps: float = 1e-6, out=None,
-                  scale: float | None = None, stream=None, state_layout: str = "kv"):
+                  scale: float | None = None, stream=None, state_layout: str = "kv",
+                  num_slots: int | None = None, status=None):
     """General decode step (``kda_decode_ex`` of the C ABI).
 
     q, k [N,T,HV,K], v [N,T,HV,V] (bf16) may be strided views, e.g. slices of
@@ -283,10 +313,15 @@ def kda_decode_ex(q, k, v, state_pool, slot_idx, *, g=None, beta=None, raw_gate=
     ``norm_weight`` selects the fused gated RMS norm.  The pool may be fp32 or
     bf16, with blocks [K, V] (``state_layout="kv"``: pool [num_slots,HV,K,V])
     or [V, K] (``"vk"``: pool [num_slots,HV,V,K], key index fastest).
+
+    Slots are checked against ``num_slots`` (default: the pool's first
+    dimension; 0 = unchecked): an active row naming a slot at or beyond it gets
+    a zero output, leaves the pool untouched and, when ``status`` (a device
+    int32 tensor the caller zeroes) is given, sets ``status[0]`` to 1.
     Returns ``out`` (dense bf16 [N,T,HV,V])."""
     a, out = _ex_args(q, k, v, state_pool, slot_idx, g=g, beta=beta, raw_gate=raw_gate, A_log=A_log,
                       dt_bias=dt_bias, raw_beta=raw_beta, gate=gate, norm_weight=norm_weight, eps=eps, out=out,
-                      scale=scale, state_layout=state_layout)
+                      scale=scale, state_layout=state_layout, num_slots=num_slots, status=status)
     st = library().kda_decode_ex(ctypes.byref(a), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_ex")

@@ -87,7 +87,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   if (hc && (hc->in_bytes < 0 || (hc->in_bytes > 0 && (!hc->host_in || !hc->dev_in)) || !hc->host_out))
     return KDA_ERR_INVALID_ARG;
   // ---- sizes
-  if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0) return KDA_ERR_INVALID_ARG;
+  if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0 || a.num_slots < 0) return KDA_ERR_INVALID_ARG;
   if (gated && !(a.eps >= 0.0f && a.eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
   if (a.state_dtype != KDA_STATE_FP32 && a.state_dtype != KDA_STATE_BF16) return KDA_ERR_INVALID_ARG;
   if (a.state_layout != KDA_LAYOUT_KV && a.state_layout != KDA_LAYOUT_VK) return KDA_ERR_INVALID_ARG;
@@ -123,6 +123,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
       !aligned(a.slot_idx, 4))
     return KDA_ERR_MISALIGNED;
   if (raw && (!aligned(a.dt_bias, 16) || !aligned(a.A_log, 4))) return KDA_ERR_MISALIGNED;
+  if (a.status && !aligned(a.status, 4)) return KDA_ERR_MISALIGNED;
   if (gated && (!aligned(a.gate, 16) || !aligned(a.norm_weight, 16))) return KDA_ERR_MISALIGNED;
 
   // ---- row strides: at least one row, and 16-byte aligned rows for the vector loads
@@ -149,19 +150,26 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
       range_of(gated ? a.norm_weight : nullptr, gated ? V * 2 : 0),
       range_of(raw ? a.A_log : nullptr, raw ? HV * 4 : 0),
       range_of(raw ? a.dt_bias : nullptr, raw ? hk * 4 : 0)};
-  // The pool's extent depends on slot values held on the device; the visible
-  // part is slot 0 plus the base address itself.
+  // The pool's extent: all num_slots blocks when the call declares the pool's
+  // size; otherwise it depends on slot values held on the device, and the
+  // visible part is slot 0 plus the base address itself.
   const bool bf16_state = a.state_dtype == KDA_STATE_BF16;
-  const Range r_slot0 = range_of(a.state_pool, hk * V * (bf16_state ? 2 : 4));
+  int64_t block_bytes, pool_bytes = 0;
+  if (!mul_ok(hk, V * (bf16_state ? 2 : 4), &block_bytes) ||
+      (a.num_slots > 0 && !mul_ok(block_bytes, a.num_slots, &pool_bytes)))
+    return KDA_ERR_UNSUPPORTED;
+  const Range r_pool = range_of(a.state_pool, a.num_slots > 0 ? pool_bytes : block_bytes);
   const uintptr_t pool_base = reinterpret_cast<uintptr_t>(a.state_pool);
   auto touches_pool = [&](Range r) {
-    return overlaps(r, r_slot0) || (r.lo <= pool_base && pool_base < r.hi);
+    return overlaps(r, r_pool) || (r.lo <= pool_base && pool_base < r.hi);
   };
   if (touches_pool(r_out)) return KDA_ERR_ALIAS;
   if (hc && hc->in_bytes > 0 && touches_pool(range_of(hc->dev_in, hc->in_bytes))) return KDA_ERR_ALIAS;
+  const Range r_status = range_of(a.status, a.status ? 4 : 0);
+  if (a.status && (overlaps(r_status, r_out) || touches_pool(r_status))) return KDA_ERR_ALIAS;
   for (const Range& r : inputs) {
     if (r.hi == r.lo) continue;
-    if (overlaps(r, r_out) || touches_pool(r)) return KDA_ERR_ALIAS;
+    if (overlaps(r, r_out) || touches_pool(r) || (a.status && overlaps(r, r_status))) return KDA_ERR_ALIAS;
   }
 
   // ---- device
@@ -195,6 +203,8 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   p.tiles = static_cast<int32_t>(tiles);
   p.scale = a.scale;
   p.eps = a.eps;
+  p.num_slots = a.num_slots;
+  p.status = a.status;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -218,72 +228,94 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   }
 
   // Input form: raw serving inputs; dense rows (offsets from the shape alone,
-  // whatever entry point was called); any other row strides.
+  // whatever entry point was called) when the slots are unchecked; any other
+  // row strides, or checked slots (only the larger parameter block carries the
+  // pool size and the status word).
   const bool dense = a.q_row_stride == hk && a.k_row_stride == hk && a.v_row_stride == hvv &&
-                     a.g_row_stride == hk && a.beta_row_stride == HV && (!gated || a.gate_row_stride == hvv);
+                     a.g_row_stride == hk && a.beta_row_stride == HV && (!gated || a.gate_row_stride == hvv) &&
+                     a.num_slots == 0;
   const int form = raw ? kda::kInRaw : dense ? kda::kInDense : kda::kInStrided;
 
-  cudaError_t err = cudaErrorInvalidValue;
-  if (hc && hc->in_bytes > 0 &&
-      cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
-                      cfg.stream) != cudaSuccess)
-    return KDA_ERR_CUDA;
+  // Pick the kernel (and make its dynamic shared memory allowance) before
+  // anything is enqueued.
   const bool vk = a.state_layout == KDA_LAYOUT_VK;
   const bool multi = T > 1;
   const bool v128 = V == 128;
+  const void* func = nullptr;
+  cudaError_t err = cudaSuccess;
   // One instantiation per (K, V fixed at 128 or not, gated, state type, input
   // form, state layout); T == 1 and T > 1 (chunked) kernels.
-#define KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, STT, RR, VKK)                                             \
+#define KDA_PICK_ONE(KERNEL, KK, VV, GG, STT, RR, VKK)                                               \
   do {                                                                                                \
     constexpr auto kern = kda::KERNEL<KK, VV, GG, STT, RR, VKK>;                                      \
     constexpr int smem = kda::KERNEL##_dyn_smem<KK, STT, VKK>;                                        \
     cfg.dynamicSmemBytes = smem;                                                                      \
     err = smem ? allow_dynamic_smem<kern>(smem) : cudaSuccess;                                        \
-    if (err == cudaSuccess) err = cudaLaunchKernelEx(&cfg, kern, pf);                                 \
+    func = reinterpret_cast<const void*>(kern);                                                       \
   } while (0)
-#define KDA_LAUNCH_ST(KERNEL, KK, VV, GG, RR)                                                         \
+#define KDA_PICK_ST(KERNEL, KK, VV, GG, RR)                                                           \
   do {                                                                                                \
-    const kda::ParamsOf<RR>& pf = p; /* the dense form takes the smaller block */                     \
     if (vk) {                                                                                         \
-      if (bf16_state) KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, true);                    \
-      else KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, float, RR, true);                                       \
+      if (bf16_state) KDA_PICK_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, true);                      \
+      else KDA_PICK_ONE(KERNEL, KK, VV, GG, float, RR, true);                                         \
     } else {                                                                                          \
-      if (bf16_state) KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, false);                   \
-      else KDA_LAUNCH_ONE(KERNEL, KK, VV, GG, float, RR, false);                                      \
+      if (bf16_state) KDA_PICK_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, false);                     \
+      else KDA_PICK_ONE(KERNEL, KK, VV, GG, float, RR, false);                                        \
     }                                                                                                 \
   } while (0)
-#define KDA_LAUNCH(KERNEL, KK, VV, GG)                                             \
-  do {                                                                             \
-    if (form == kda::kInRaw) KDA_LAUNCH_ST(KERNEL, KK, VV, GG, kda::kInRaw);       \
-    else if (form == kda::kInDense) KDA_LAUNCH_ST(KERNEL, KK, VV, GG, kda::kInDense); \
-    else KDA_LAUNCH_ST(KERNEL, KK, VV, GG, kda::kInStrided);                       \
+#define KDA_PICK(KERNEL, KK, VV, GG)                                                  \
+  do {                                                                                \
+    if (form == kda::kInRaw) KDA_PICK_ST(KERNEL, KK, VV, GG, kda::kInRaw);            \
+    else if (form == kda::kInDense) KDA_PICK_ST(KERNEL, KK, VV, GG, kda::kInDense);   \
+    else KDA_PICK_ST(KERNEL, KK, VV, GG, kda::kInStrided);                            \
   } while (0)
-#define KDA_LAUNCH_V(KK, GG)                                                 \
+#define KDA_PICK_V(KK, GG)                                                   \
   do {                                                                       \
     if (multi) {                                                             \
-      if (v128) KDA_LAUNCH(kda_decode_chunked_kernel, KK, 128, GG);          \
-      else KDA_LAUNCH(kda_decode_chunked_kernel, KK, 0, GG);                 \
+      if (v128) KDA_PICK(kda_decode_chunked_kernel, KK, 128, GG);            \
+      else KDA_PICK(kda_decode_chunked_kernel, KK, 0, GG);                   \
     } else {                                                                 \
-      if (v128) KDA_LAUNCH(kda_decode_kernel, KK, 128, GG);                  \
-      else KDA_LAUNCH(kda_decode_kernel, KK, 0, GG);                         \
+      if (v128) KDA_PICK(kda_decode_kernel, KK, 128, GG);                    \
+      else KDA_PICK(kda_decode_kernel, KK, 0, GG);                           \
     }                                                                        \
   } while (0)
-#define KDA_LAUNCH_K(KK)                   \
+#define KDA_PICK_K(KK)                     \
   do {                                     \
-    if (gated) KDA_LAUNCH_V(KK, true);     \
-    else KDA_LAUNCH_V(KK, false);          \
+    if (gated) KDA_PICK_V(KK, true);       \
+    else KDA_PICK_V(KK, false);            \
   } while (0)
   switch (K) {
-    case 64: KDA_LAUNCH_K(64); break;
-    case 128: KDA_LAUNCH_K(128); break;
-    case 256: KDA_LAUNCH_K(256); break;
+    case 64: KDA_PICK_K(64); break;
+    case 128: KDA_PICK_K(128); break;
+    case 256: KDA_PICK_K(256); break;
     default: return KDA_ERR_UNSUPPORTED;
   }
-#undef KDA_LAUNCH_K
-#undef KDA_LAUNCH_V
-#undef KDA_LAUNCH
-#undef KDA_LAUNCH_ST
-#undef KDA_LAUNCH_ONE
+#undef KDA_PICK_K
+#undef KDA_PICK_V
+#undef KDA_PICK
+#undef KDA_PICK_ST
+#undef KDA_PICK_ONE
+  if (err != cudaSuccess || func == nullptr) return KDA_ERR_CUDA;
+  if (hc) {
+    // With host copies around the step, check what can be checked about the
+    // launch before the copy in is enqueued: the kernel loads on this device
+    // and, for a cluster launch, at least one cluster fits.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, func) != cudaSuccess) return KDA_ERR_CUDA;
+    if (gated) {
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, func, &cfg) != cudaSuccess || clusters < 1)
+        return KDA_ERR_CUDA;
+    }
+    if (hc->in_bytes > 0 &&
+        cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
+                        cfg.stream) != cudaSuccess)
+      return KDA_ERR_CUDA;
+  }
+  // The dense form's kernels take the smaller parameter block, which is the
+  // leading part of p.
+  void* kargs[] = {&p};
+  err = cudaLaunchKernelExC(&cfg, func, kargs);
   if (err != cudaSuccess) return KDA_ERR_CUDA;
   if (hc && cudaMemcpyAsync(hc->host_out, a.out, static_cast<size_t>(out_elems) * 2, cudaMemcpyDeviceToHost,
                             cfg.stream) != cudaSuccess)
@@ -396,6 +428,6 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 4; }
+int32_t kda_abi_version(void) { return (1 << 16) | 5; }
 
 }  // extern "C"

@@ -123,6 +123,10 @@ struct ParamsEx : Params {
   // element (n, t, h, i) of q sits at (n*T + t)*q_rs + h*K + i (v and gate with
   // V, beta with 1).  g_rs / b_rs apply to g / beta or to raw_gate / raw_beta.
   int64_t q_rs, k_rs, v_rs, g_rs, b_rs, z_rs;
+  // Checked slots: num_slots > 0 makes a row whose slot is >= num_slots an
+  // inactive row and stores 1 to *status (when not null).
+  int64_t num_slots;
+  int32_t* status;
 };
 
 // How a kernel addresses its per-token inputs and which decay/beta inputs it
@@ -135,6 +139,21 @@ enum InputForm : int {
 };
 template <int IN>
 using ParamsOf = typename std::conditional<IN == kInDense, Params, ParamsEx>::type;
+
+// Whether row n takes part in the call: slot >= 0, and (checked forms with a
+// declared pool size) slot < num_slots.  The first thread of a CTA that meets
+// an out-of-range slot raises the status word.  Every CTA of one (n, h) sees
+// the same slot, so the decision is uniform over a cluster.
+template <int IN, typename P>
+__device__ __forceinline__ bool row_active(const P& p, int32_t slot) {
+  if constexpr (IN != kInDense) {
+    if (p.num_slots > 0 && slot >= p.num_slots) {
+      if (threadIdx.x == 0 && p.status != nullptr) atomicOr(p.status, 1);
+      return false;
+    }
+  }
+  return slot >= 0;
+}
 
 // Which input an offset is taken in (selects the row stride).
 enum InputRow : int { kRowQ, kRowK, kRowG, kRowV, kRowZ, kRowB };
@@ -652,7 +671,7 @@ kda_decode_kernel(const ParamsOf<IN> p) {
     cur.beta = __ldg(p.beta + (IN == kInDense ? row : in_off<IN, kRowB>(p, row, n, h, 1)));
   }
 
-  if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
+  if (!row_active<IN>(p, slot)) {  // inactive (padding) row: zero output, pool untouched
     if (writer) *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(0u, 0u);
     return;  // uniform over the cluster: every tile of this (n, h) sees the same slot
   }
@@ -935,7 +954,7 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
     if (warp == 0) wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + rg]);
   }
 
-  if (slot < 0) {  // inactive (padding) row: zero output, pool untouched
+  if (!row_active<IN>(p, slot)) {  // inactive (padding) row: zero output, pool untouched
     cp_async_wait<0>();
     if (writer) {
       for (int64_t t = 0; t < p.T; ++t)

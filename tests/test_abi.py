@@ -2,13 +2,16 @@
 host-side validation answers without touching a GPU.
 
 The validation tests pass fabricated addresses that the library must reject
-before any launch; they only run where no CUDA device is present, so a
-validation bug can never launch a kernel on them.  The GPU tests repeat the
-rejections with real buffers.
+before any launch; they only run in a process that sees no CUDA device, so a
+validation bug can never launch a kernel on them.  On a GPU machine the GPU
+test at the end reruns them in a child process with no visible device; the GPU
+parity tests repeat the rejections with real buffers.
 """
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -55,7 +58,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 4
+    assert lib.kda_abi_version() == (1 << 16) | 5
 
 
 # ----------------------------------------------------------------- validation
@@ -190,6 +193,19 @@ def test_ex_entry_point_validation(lib):
     assert args(**raw) == E.KDA_ERR_DEVICE                             # raw form, 2-byte raw_beta is fine
     assert args(**{**raw, "dt_bias": BASE + 12 * step + 4}) == E.KDA_ERR_MISALIGNED
     assert args(**{**raw, "A_log": 0}) == E.KDA_ERR_INVALID_ARG
+    # checked slots: a declared pool size and an optional status word
+    status = BASE + 13 * step
+    assert args(num_slots=-1) == E.KDA_ERR_INVALID_ARG
+    assert args(num_slots=4, status=status) == E.KDA_ERR_DEVICE          # valid
+    assert args(num_slots=4, status=status + 2) == E.KDA_ERR_MISALIGNED
+    assert args(num_slots=4, status=BASE + 9 * step + 8) == E.KDA_ERR_ALIAS   # inside out
+    assert args(num_slots=4, status=BASE + 5 * step + 8) == E.KDA_ERR_ALIAS   # inside the pool
+    assert args(num_slots=4, status=BASE + 2 * step) == E.KDA_ERR_ALIAS       # on an input
+    # with the pool's size declared, every slot's block counts for aliasing
+    block = 2 * 128 * 128 * 4
+    assert args(g=BASE + 5 * step + 3 * block) == E.KDA_ERR_DEVICE            # slot 3: unseen unchecked
+    assert args(g=BASE + 5 * step + 3 * block, num_slots=4) == E.KDA_ERR_ALIAS
+    assert args(g=BASE + 5 * step + 4 * block, num_slots=4) == E.KDA_ERR_DEVICE  # just past the pool
 
 
 @no_gpu
@@ -219,3 +235,18 @@ def test_host_entry_point_validation(lib):
     assert call(hin=None, din=None, nbytes=0) == E.KDA_ERR_DEVICE  # nothing to copy in
     assert call(hout=None) == E.KDA_ERR_INVALID_ARG
     assert call(din=BASE + 5 * step - 64, nbytes=128) == E.KDA_ERR_ALIAS  # staging runs into the pool
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a machine with a GPU")
+def test_host_validation_suite_with_no_visible_device():
+    """Rerun every fabricated-pointer validation test of this file in a child
+    process that sees no CUDA device: a call that passes validation stops at
+    KDA_ERR_DEVICE there, so none can launch, and the rejections are checked in
+    full on the GPU machine too."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "not gpu",
+                        os.path.abspath(__file__)], env=env, cwd=ROOT, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout and " skipped" not in r.stdout, r.stdout[-1000:]

@@ -597,3 +597,60 @@ def test_long_token_runs_every_form(N, T, HV, K, V, gated, state, layout, form, 
         g, beta = oracle.activate(w.raw.raw_gate, w.raw.A_log, w.raw.dt_bias, w.raw.raw_beta)
         w = dataclasses.replace(w, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
     assert_parity(w, o, pool if layout == "kv" else pool.transpose(-1, -2), before)
+
+
+# ---------------------------------------------------------------------------
+# checked slots (kda_decode_args.num_slots / status)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("T,gated,state,form", [
+    (1, False, "fp32", "dense"), (1, True, "bf16", "dense"), (1, False, "fp32", "raw"),
+    (6, True, "fp32", "dense"), (5, False, "bf16", "raw"),
+])
+def test_checked_slots_skip_rows_beyond_the_declared_pool(T, gated, state, form, cuda_device):
+    """With the pool's size declared, a row naming a slot at or past it is
+    skipped like a padding row (zero output, pool untouched) and raises the
+    status word.  The pool is allocated with two slots more than declared, so
+    the out-of-range slots still lie inside the allocation: a guard that failed
+    would change those slots (checked bit for bit) but could not fault."""
+    declared = 6
+    w = workloads.make(N=4, T=T, HV=2, K=128, V=128, num_slots=declared + 2, gated=gated, seed=90 + T,
+                       state_dtype=state, serving=form == "raw", packed=False)
+    w.slot_idx.copy_(torch.tensor([0, declared, 3, declared + 1], dtype=torch.int32))
+    d = w.to(cuda_device)
+    before = d.state.clone()
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    extra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if gated else {}
+    if form == "raw":
+        r = d.raw
+        extra.update(raw_gate=r.raw_gate, A_log=r.A_log, dt_bias=r.dt_bias, raw_beta=r.raw_beta)
+    else:
+        extra.update(g=d.g, beta=d.beta)
+    o = kda.kda_decode_ex(d.q, d.k, d.v, d.state, d.slot_idx, scale=w.scale, num_slots=declared,
+                          status=status, **extra)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1, "an out-of-range slot did not raise the status word"
+    ref = dataclasses.replace(w, slot_idx=torch.tensor([0, -1, 3, -1], dtype=torch.int32))
+    if form == "raw":
+        g, beta = oracle.activate(w.raw.raw_gate, w.raw.A_log, w.raw.dt_bias, w.raw.raw_beta)
+        ref = dataclasses.replace(ref, g=torch.from_numpy(g), beta=torch.from_numpy(beta))
+    assert_parity(ref, o, d.state, before)
+    assert torch.equal(d.state[declared:], before[declared:])
+
+    # every slot in range: the status word stays as the caller left it (zero)
+    status.zero_()
+    d.slot_idx.copy_(torch.tensor([0, 5, 3, -1], dtype=torch.int32, device=cuda_device))
+    kda.kda_decode_ex(d.q, d.k, d.v, d.state, d.slot_idx, scale=w.scale, num_slots=declared,
+                      status=status, **extra)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
+def test_checked_slots_equal_unchecked_when_in_range(cuda_device):
+    """Declaring the pool's size changes nothing for in-range slots: the checked
+    call (row-strided kernels) is bit-identical to the unchecked dense one."""
+    w = workloads.make(N=8, T=1, HV=4, K=128, V=128, num_slots=12, seed=95, inactive=2)
+    d1, d2 = w.to(cuda_device), w.to(cuda_device)
+    o1 = kda.kda_decode_ex(d1.q, d1.k, d1.v, d1.state, d1.slot_idx, g=d1.g, beta=d1.beta, num_slots=0)
+    o2 = kda.kda_decode_ex(d2.q, d2.k, d2.v, d2.state, d2.slot_idx, g=d2.g, beta=d2.beta, num_slots=12)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(d1.state, d2.state)
