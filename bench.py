@@ -72,12 +72,13 @@ def rank_seed(base: int, rank: int) -> int:
     return base + 100_003 * rank
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(names=("kda_decode_kernel.cuh", "kda_decode_api.cu")) -> str:
+    """Hash of the source files that define a kernel and its launch (by default
+    the decode kernels): a profile taken from other sources is stale."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(names):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -173,6 +174,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 def call_fn(kda, d, out, stream):
+    if d.name.startswith("prefill_"):  # the chunked prefill over the workload's T tokens
+        import torch
+
+        ws = torch.empty(kda.prefill_workspace_bytes(d.N, d.T, d.HV, d.K, d.V), dtype=torch.uint8,
+                         device=d.q.device)
+        return lambda: kda.kda_prefill(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, out=out, scale=d.scale,
+                                       workspace=ws, stream=stream)
     if d.packed or d.raw is not None or d.state_layout != "kv":  # the general entry point
         from linear_attention_recurrent_decode_b200 import workloads
 
@@ -263,13 +271,14 @@ class GraphRegion:
         else:
             self.timed = [self.cycle] * (steps // R) + ([self._capture(calls[:rem])] if rem else [])
         self.tail = self._capture(calls[rem:]) if rem else None
-        # upload every graph, then estimate the time of one cycle (all untimed)
+        # upload every graph (keeping the rotation: tail after each region), then
+        # estimate the time of one cycle (all untimed)
         with torch.cuda.stream(stream):
             self.cycle.replay()
-            self.timed[0].replay()
-            self.timed[-1].replay()
-            if self.tail:
-                self.tail.replay()
+            for g in (self.timed[0], self.timed[-1]):
+                g.replay()
+                if self.tail:
+                    self.tail.replay()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
@@ -387,7 +396,8 @@ def run_ours(args):
     eager_us = reduce_max(ea.elapsed_time(eb), dev) * 1e3 / n_eager
 
     # end to end through the public API: pinned host inputs in, output back out
-    e2e = run_e2e(kda, base, dev, stream, min(args.steps, args.e2e_steps), world)
+    e2e_fn = run_e2e_prefill if args.config.startswith("prefill_") else run_e2e
+    e2e = e2e_fn(kda, base, dev, stream, min(args.steps, args.e2e_steps), world)
     floor = None if args.no_floor else copy_floor(base, dev, stream, R, args.steps, args.preroll_ms / 1e3)
 
     if world > 1:
@@ -526,6 +536,49 @@ def run_e2e(kda, w, dev, stream, steps, world):
             "d2h_bytes_per_step": d2h, "steps": steps,
             "how": "one kda_decode_host call per step (HostStep): copy of the packed inputs from pinned host "
                    "memory, the decode kernel, copy of the output back; the state pool stays resident on the GPU"}
+
+
+def run_e2e_prefill(kda, w, dev, stream, steps, world):
+    """µs per prefill call with the call's inputs copied from pinned host memory
+    (one copy per input tensor) and its output copied back, through the public
+    Python API; the state pool and the workspace stay on the device."""
+    import torch
+
+    inputs = {k: t for k, t in w.tensors().items() if k != "state"}
+    host = {k: t.pin_memory() for k, t in inputs.items()}
+    devv = {k: torch.empty_like(t, device=dev) for k, t in inputs.items()}
+    pool = w.state.to(dev)
+    out_d = torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty(out_d.shape, dtype=torch.bfloat16).pin_memory()
+    ws = torch.empty(kda.prefill_workspace_bytes(w.N, w.T, w.HV, w.K, w.V), dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for k, t in host.items():
+            devv[k].copy_(t, non_blocking=True)
+        kda.kda_prefill(devv["q"], devv["k"], devv["v"], devv["g"], devv["beta"], pool, devv["slot_idx"],
+                        out=out_d, scale=w.scale, workspace=ws, stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        step()  # untimed lead-in: the first event is recorded on a busy stream
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1), dev)
+    return {"value": round(ms * 1e3 / (steps * world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "how": "per step: copies of the inputs from pinned host memory, kda_prefill, copy of the output back "
+                   "(torch copies around the library call); state pool and workspace resident on the GPU"}
 
 
 # ------------------------------------------------------------------ reference arm

@@ -1,0 +1,81 @@
+/*
+ * kda_prefill.h -- C ABI of the chunked KDA prefill on B200 (sm_100a).
+ *
+ * The operation is the decode step of kda_decode.h taken over a long token
+ * run: for every sequence n in [0, N), value head h in [0, HV) and token t in
+ * [0, T), in token order, on the fp32 state S[K][V] held in slot slot_idx[n]:
+ *
+ *     S   <- Diag(exp(g[n,t,h,:])) S
+ *     u   <- beta[n,t,h] * (v[n,t,h,:] - S^T k[n,t,h,:])
+ *     S   <- S + k[n,t,h,:] u^T
+ *     out[n,t,h,:] <- bf16(scale * S^T q[n,t,h,:])
+ *
+ * with the final state written back to the slot.  The result equals T calls of
+ * the decode step up to fp32 rounding; what differs is how it is computed: the
+ * tokens are taken in chunks of 64 in the WY / UT chunk form (a triangular
+ * solve inside each chunk, a short state recurrence across chunks and the
+ * chunk outputs as dense products), which turns the work of a long run into
+ * parallel per-chunk products instead of a token-by-token chain.
+ *
+ * Source: vLLM #57585 "Tune recurrent KDA launch configuration on SM90",
+ * Details: the related work it names (FlashInfer's fused KDA on Blackwell)
+ * adds a prefill path for the SM100 family next to its decode kernels.  The
+ * page prints no prefill algorithm; the chunk form used here is the delta rule
+ * regrouped exactly (see kda_prefill_kernel.cuh for the formulas).
+ *
+ * Layouts: as kda_decode (dense, row-major, current device): q, k bf16
+ * [N, T, HV, K]; v bf16 [N, T, HV, V]; g fp32 [N, T, HV, K] (log-decay);
+ * beta fp32 [N, T, HV]; state_pool fp32 [num_slots, HV, K, V] (in place);
+ * slot_idx int32 [N] (< 0 = inactive row: zero output, pool untouched);
+ * out bf16 [N, T, HV, V].
+ *
+ * Supported sizes: K = V = 128; HV >= 1; N, T >= 0 (N == 0 or T == 0 is a
+ * no-op that touches no pointer).  Other K or V: KDA_ERR_UNSUPPORTED.
+ *
+ * Workspace: the caller passes device memory of at least
+ * kda_prefill_workspace_bytes(N, T, HV, K, V) bytes (16-byte aligned); the
+ * library allocates nothing.  Per (sequence, head, chunk of 64 tokens) it holds
+ * about 240 KB of fp32 intermediates (the chunk's solve results, decayed keys
+ * and queries, its start state and corrections).  Its contents are not
+ * meaningful between calls; calls that share a workspace must not overlap on
+ * the device (stream order is enough).
+ *
+ * Execution: three kernels enqueued on `stream` in order (chunk preparation,
+ * the state recurrence across chunks, the chunk outputs); no host sync; can be
+ * captured in a CUDA graph.  Alignment: q, k, v, g, state_pool, out, workspace
+ * on 16 bytes; beta, slot_idx on 4 bytes.
+ *
+ * Errors: the host-side validation of kda_decode (KDA_ERR_INVALID_ARG for a
+ * null pointer with work to do, a negative size or a workspace smaller than
+ * required; KDA_ERR_ALIAS if out, or the workspace, overlaps an input, the
+ * pool's slot-0 block or each other; KDA_ERR_MISALIGNED; KDA_ERR_DEVICE;
+ * KDA_ERR_CUDA if the runtime refuses a launch).  Nothing is enqueued unless
+ * validation passes; the three launches are configured before the first is
+ * enqueued.
+ */
+#ifndef KDA_PREFILL_H
+#define KDA_PREFILL_H
+
+#include "kda_decode.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Bytes of workspace kda_prefill needs for these sizes (0 when N, T or HV is
+ * 0; -1 for sizes it does not support or negative sizes). */
+KDA_API int64_t kda_prefill_workspace_bytes(int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V);
+
+/* Chunked prefill (see the top of this file).  Writes bf16 outputs for every
+ * token and the final state of each active row back to its slot. */
+KDA_API kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, float *state_pool, const int32_t *slot_idx,
+                               void *out, void *workspace, int64_t workspace_bytes, int64_t N,
+                               int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
+                               kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_PREFILL_H */

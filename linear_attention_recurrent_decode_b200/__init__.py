@@ -24,7 +24,8 @@ import threading
 
 import torch
 
-__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "KdaError", "library", "status_string",
+__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "kda_prefill",
+           "prefill_workspace_bytes", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_STATE_FP32", "KDA_STATE_BF16",
            "KDA_LAYOUT_KV", "KDA_LAYOUT_VK", "LIBRARY_PATH", "EXPORTED_SYMBOLS"]
@@ -68,7 +69,7 @@ KDA_STATE_BF16 = 1
 KDA_LAYOUT_KV = 0
 KDA_LAYOUT_VK = 1
 
-# Every symbol include/kda_decode.h declares, with its ctypes signature.
+# Every symbol include/kda_decode.h and include/kda_prefill.h declare, with its ctypes signature.
 EXPORTED_SYMBOLS = {
     "kda_decode": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_gated_rmsnorm": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
@@ -78,6 +79,9 @@ EXPORTED_SYMBOLS = {
     "kda_decode_host": ([ctypes.POINTER(DecodeArgs), _P, _P, _I, _P, _P], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_abi_version": ([], ctypes.c_int32),
+    # include/kda_prefill.h
+    "kda_prefill_workspace_bytes": ([_I] * 5, ctypes.c_int64),
+    "kda_prefill": ([_P] * 9 + [_I] * 6 + [_F, _P], ctypes.c_int),
 }
 
 _lock = threading.Lock()
@@ -368,3 +372,36 @@ class HostStep:
         st = self._fn(self._ref, *self._ptrs, self._stream)
         if st != KDA_OK:
             raise KdaError(st, "kda_decode_host")
+
+
+# ---------------------------------------------------------------- chunked prefill
+def prefill_workspace_bytes(N: int, T: int, HV: int, K: int = 128, V: int = 128) -> int:
+    """Device workspace ``kda_prefill`` needs for these sizes (bytes)."""
+    n = library().kda_prefill_workspace_bytes(N, T, HV, K, V)
+    if n < 0:
+        raise ValueError(f"kda_prefill does not support N={N}, T={T}, HV={HV}, K={K}, V={V}")
+    return n
+
+
+def kda_prefill(q, k, v, g, beta, state_pool, slot_idx, out=None, scale: float | None = None, workspace=None,
+                stream=None):
+    """Chunked prefill (``kda_prefill`` of the C ABI): the decode recurrence over
+    all T tokens of each sequence, taken in chunks of 64 tokens; updates
+    ``state_pool`` (fp32 [num_slots, HV, K, V]) in place and returns ``out``
+    (bf16 [N, T, HV, V]).  ``workspace``: a device uint8 tensor of at least
+    :func:`prefill_workspace_bytes` bytes (allocated here if not given)."""
+    N, T, HV, K, V, out = _common(q, k, v, g, beta, state_pool, slot_idx, out)
+    if state_pool.dtype != torch.float32:
+        raise TypeError("kda_prefill takes an fp32 state pool")
+    if scale is None:
+        scale = 1.0 / math.sqrt(K)
+    need = prefill_workspace_bytes(N, T, HV, K, V)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace", torch.uint8, None, torch.cuda.current_device())
+    st = library().kda_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
+                               state_pool.data_ptr(), slot_idx.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                               workspace.numel(), N, T, HV, K, V, float(scale), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill")
+    return out

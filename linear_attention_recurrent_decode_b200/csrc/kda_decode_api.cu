@@ -12,66 +12,19 @@
 #include <cstdint>
 
 #include "kda_decode.h"
-#include "kda_decode_kernel.cuh"
+#include "kda_decode_pick.cuh"
+#include "kda_host_util.h"
+
+// The kernels are instantiated in kda_decode_k{64,128,256}.cu.
+namespace kda {
+extern template cudaError_t pick_decode_kernel<64>(const KernelChoice&, const void**, int*);
+extern template cudaError_t pick_decode_kernel<128>(const KernelChoice&, const void**, int*);
+extern template cudaError_t pick_decode_kernel<256>(const KernelChoice&, const void**, int*);
+}  // namespace kda
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::atomic<int32_t> g_cc_cache[kMaxDevices];  // 0 = unknown, else major*10 + minor
-
-kda_status check_device() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return KDA_ERR_DEVICE;
-  int32_t cc = dev < kMaxDevices ? g_cc_cache[dev].load(std::memory_order_relaxed) : 0;
-  if (cc == 0) {
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-      return KDA_ERR_DEVICE;
-    cc = major * 10 + minor;
-    if (dev < kMaxDevices) g_cc_cache[dev].store(cc, std::memory_order_relaxed);
-  }
-  // The library carries sm_100a code only; it runs on compute capability 10.0.
-  return cc == 100 ? KDA_OK : KDA_ERR_DEVICE;
-}
-
-// Once per kernel and device: let the kernel take `bytes` of dynamic shared
-// memory (the [V][K] staging buffer; above 48 KB this needs the opt-in) and
-// prefer the shared-memory carveout.
-template <auto Kernel>
-cudaError_t allow_dynamic_smem(int bytes) {
-  static std::atomic<uint64_t> ready{0};  // bit d: done on device d (d < 64)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
-  if (bit && (ready.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess && bit) ready.fetch_or(bit, std::memory_order_relaxed);
-  return e;
-}
-
-bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-struct Range {
-  uintptr_t lo, hi;  // [lo, hi)
-};
-Range range_of(const void* p, int64_t bytes) {
-  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
-  return Range{lo, lo + static_cast<uintptr_t>(bytes)};
-}
-bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
-
-// Multiply non-negative sizes, flagging overflow of int64.
-bool mul_ok(int64_t a, int64_t b, int64_t* r) { return !__builtin_mul_overflow(a, b, r); }
-
-// Bytes spanned by `rows` rows of `width` elements, `stride` elements apart.
-bool span_bytes(int64_t rows, int64_t stride, int64_t width, int64_t elem, int64_t* bytes) {
-  int64_t a;
-  if (!mul_ok(rows - 1, stride, &a) || __builtin_add_overflow(a, width, &a)) return false;
-  return mul_ok(a, elem, bytes);
-}
+using namespace kda_host;
 
 // Host staging of kda_decode_host: the step's inputs are copied from host_in to
 // dev_in before the kernel, the output from out to host_out after it.
@@ -239,74 +192,30 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   // Pick the kernel (and make its dynamic shared memory allowance) before
   // anything is enqueued.
   const bool vk = a.state_layout == KDA_LAYOUT_VK;
-  const bool multi = T > 1;
-  const bool v128 = V == 128;
   const void* func = nullptr;
-  cudaError_t err = cudaSuccess;
-  // One instantiation per (K, V fixed at 128 or not, gated, state type, input
-  // form, state layout); T == 1 and T > 1 (chunked) kernels.
-#define KDA_PICK_ONE(KERNEL, KK, VV, GG, STT, RR, VKK)                                               \
-  do {                                                                                                \
-    constexpr auto kern = kda::KERNEL<KK, VV, GG, STT, RR, VKK>;                                      \
-    constexpr int smem = kda::KERNEL##_dyn_smem<KK, STT, VKK>;                                        \
-    cfg.dynamicSmemBytes = smem;                                                                      \
-    err = smem ? allow_dynamic_smem<kern>(smem) : cudaSuccess;                                        \
-    func = reinterpret_cast<const void*>(kern);                                                       \
-  } while (0)
-#define KDA_PICK_ST(KERNEL, KK, VV, GG, RR)                                                           \
-  do {                                                                                                \
-    if (vk) {                                                                                         \
-      if (bf16_state) KDA_PICK_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, true);                      \
-      else KDA_PICK_ONE(KERNEL, KK, VV, GG, float, RR, true);                                         \
-    } else {                                                                                          \
-      if (bf16_state) KDA_PICK_ONE(KERNEL, KK, VV, GG, __nv_bfloat16, RR, false);                     \
-      else KDA_PICK_ONE(KERNEL, KK, VV, GG, float, RR, false);                                        \
-    }                                                                                                 \
-  } while (0)
-#define KDA_PICK(KERNEL, KK, VV, GG)                                                  \
-  do {                                                                                \
-    if (form == kda::kInRaw) KDA_PICK_ST(KERNEL, KK, VV, GG, kda::kInRaw);            \
-    else if (form == kda::kInDense) KDA_PICK_ST(KERNEL, KK, VV, GG, kda::kInDense);   \
-    else KDA_PICK_ST(KERNEL, KK, VV, GG, kda::kInStrided);                            \
-  } while (0)
-#define KDA_PICK_V(KK, GG)                                                   \
-  do {                                                                       \
-    if (multi) {                                                             \
-      if (v128) KDA_PICK(kda_decode_chunked_kernel, KK, 128, GG);            \
-      else KDA_PICK(kda_decode_chunked_kernel, KK, 0, GG);                   \
-    } else {                                                                 \
-      if (v128) KDA_PICK(kda_decode_kernel, KK, 128, GG);                    \
-      else KDA_PICK(kda_decode_kernel, KK, 0, GG);                           \
-    }                                                                        \
-  } while (0)
-#define KDA_PICK_K(KK)                     \
-  do {                                     \
-    if (gated) KDA_PICK_V(KK, true);       \
-    else KDA_PICK_V(KK, false);            \
-  } while (0)
+  int smem = 0;
+  kda::KernelChoice choice;
+  choice.gated = gated;
+  choice.multi = T > 1;
+  choice.v128 = V == 128;
+  choice.vk = vk;
+  choice.bf16_state = bf16_state;
+  choice.form = form;
+  choice.tiles = static_cast<int>(tiles);
+  choice.check_launch = hc != nullptr;
+  cudaError_t err = cudaErrorInvalidValue;
   switch (K) {
-    case 64: KDA_PICK_K(64); break;
-    case 128: KDA_PICK_K(128); break;
-    case 256: KDA_PICK_K(256); break;
+    case 64: err = kda::pick_decode_kernel<64>(choice, &func, &smem); break;
+    case 128: err = kda::pick_decode_kernel<128>(choice, &func, &smem); break;
+    case 256: err = kda::pick_decode_kernel<256>(choice, &func, &smem); break;
     default: return KDA_ERR_UNSUPPORTED;
   }
-#undef KDA_PICK_K
-#undef KDA_PICK_V
-#undef KDA_PICK
-#undef KDA_PICK_ST
-#undef KDA_PICK_ONE
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   if (err != cudaSuccess || func == nullptr) return KDA_ERR_CUDA;
   if (hc) {
-    // With host copies around the step, check what can be checked about the
-    // launch before the copy in is enqueued: the kernel loads on this device
-    // and, for a cluster launch, at least one cluster fits.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, func) != cudaSuccess) return KDA_ERR_CUDA;
-    if (gated) {
-      int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, func, &cfg) != cudaSuccess || clusters < 1)
-        return KDA_ERR_CUDA;
-    }
+    // With host copies around the step, the launch was checked above (once per
+    // kernel and device: the kernel loads, a cluster fits) before the copy in
+    // is enqueued.
     if (hc->in_bytes > 0 &&
         cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
                         cfg.stream) != cudaSuccess)

@@ -1,0 +1,565 @@
+// kda_prefill_kernel.cuh -- sm_100a kernels of the chunked KDA prefill.
+//
+// The same recurrence as the decode step, taken over long token runs: per
+// sequence n and value head h, for t = 0 .. T-1,
+//   S <- Diag(exp(g_t)) S;  u_t = beta_t (v_t - S^T k_t);  S <- S + k_t u_t^T;
+//   o_t = scale S^T q_t.
+// Tokens are grouped in chunks of C = 64 and the recurrence is regrouped into
+// the WY / UT chunk form (vLLM #57585 "Tune recurrent KDA launch configuration
+// on SM90", Details: FlashInfer's fused KDA prefill path on Blackwell is the
+// related work the page names).  Inside a chunk, with Gamma_t = sum_{s<=t} g_s
+// (per key channel, the cumulative log-decay from the chunk start) and S0 the
+// state at the chunk start:
+//   Kt_t = k_t * exp(Gamma_t)            (decayed keys)
+//   Qt_t = q_t * exp(Gamma_t)            (decayed queries)
+//   Kh_t = k_t * exp(Gamma_C - Gamma_t)  (keys decayed to the chunk end)
+//   M[t][s] = sum_i k_t,i k_s,i exp(Gamma_t,i - Gamma_s,i)   (s < t)
+//   P[t][s] = sum_i q_t,i k_s,i exp(Gamma_t,i - Gamma_s,i)   (s <= t)
+// the corrections solve the unit lower-triangular system
+//   u_t + beta_t sum_{s<t} M[t][s] u_s = beta_t (v_t - S0^T Kt_t),
+// i.e. U = Ut - W S0 with [W | Ut] = (I + diag(beta) M)^-1 diag(beta) [Kt | V],
+// and then
+//   O   = scale (Qt S0 + P U),
+//   S_C = Diag(exp(Gamma_C)) S0 + Kh^T U.
+// This equals the token-by-token recurrence in exact arithmetic.
+//
+// Three kernels:
+//   1. kda_prefill_chunk_kernel (one CTA per (n, h, chunk), all chunks at
+//      once): Gamma in fp64, the decay factors, M and P, the substitution for
+//      W and Ut; writes them to the workspace.
+//   2. kda_prefill_state_kernel (one CTA per (n, h, 16-column value tile),
+//      chunks in order): the state chain U = Ut - W S0, S_C = D S0 + Kh^T U,
+//      keeping S in shared memory; writes each chunk's start state and U to the
+//      workspace and the final state back to the pool slot.
+//   3. kda_prefill_output_kernel (one CTA per (n, h, chunk)): O = scale (Qt S0
+//      + P U), bf16 output.
+//
+// Numerics.  exp(Gamma_t - Gamma_s) is never formed by dividing decays: the
+// chunk kernel factors it as exp(Gamma_t - Gamma_r) exp(Gamma_r - Gamma_s)
+// around the chunk's middle token r, which keeps both factors in fp32 range
+// whenever every key channel decays by at most e^80 between r and any token
+// of the chunk; a chunk outside that bound (a decay of more than e^-2.5 per
+// token on some channel, sustained over half a chunk) takes a slower exact
+// path that forms every pair's exponential directly.  Gamma is summed in fp64
+// and each exponential is taken from the fp64 difference, so the long-range
+// decays keep fp32 accuracy (a cumulative sum in fp32 would lose up to
+// 64 ulp of |Gamma|).  All other arithmetic is fp32.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kdap {
+
+constexpr int kC = 64;        // tokens per chunk
+constexpr int kK = 128;       // key dimension (the kernels are written for K = V = 128)
+constexpr int kV = 128;       // value dimension
+constexpr int kBV = 16;       // value columns per state-chain CTA
+constexpr float kSafeExp = 80.f;  // |Gamma_t - Gamma_r| bound of the factored path
+
+struct Params {
+  const __nv_bfloat16* q;  // [N, T, HV, K]
+  const __nv_bfloat16* k;  // [N, T, HV, K]
+  const __nv_bfloat16* v;  // [N, T, HV, V]
+  const float* g;          // [N, T, HV, K]
+  const float* beta;       // [N, T, HV]
+  float* state;            // [num_slots, HV, K, V]
+  const int32_t* slot_idx; // [N]
+  __nv_bfloat16* out;      // [N, T, HV, V]
+  float* ws;               // workspace (see Workspace)
+  int64_t T;
+  int64_t HV;
+  int32_t nchunks;         // ceil(T / C)
+  float scale;
+};
+
+// Workspace layout: one record per (n, h, chunk), fp32.
+struct Workspace {
+  static constexpr int64_t kWt = 0;                   // W^T  [K][C]
+  static constexpr int64_t kKh = kWt + kK * kC;       // Kh   [C][K]
+  static constexpr int64_t kUt = kKh + kC * kK;       // Ut   [C][V]   (the V part of the solve)
+  static constexpr int64_t kQt = kUt + kC * kV;       // Qt^T [K][C]
+  static constexpr int64_t kPt = kQt + kK * kC;       // P^T  [C][C]   (Pt[s][t] = P[t][s], zero for s > t)
+  static constexpr int64_t kDc = kPt + kC * kC;       // exp(Gamma_C) [K]
+  static constexpr int64_t kS0 = kDc + kK;            // chunk-start state [K][V]
+  static constexpr int64_t kU = kS0 + kK * kV;        // U [C][V]
+  static constexpr int64_t kFloats = kU + kC * kV;    // per record
+  static __host__ __device__ int64_t record(int64_t unit, int64_t chunk, int32_t nchunks) {
+    return (unit * nchunks + chunk) * kFloats;
+  }
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// exp(x) for an fp64 argument, to fp32 accuracy: expf of the fp32 part times
+// (1 + the remainder), the remainder being below half an fp32 ulp of x.
+__device__ __forceinline__ float exp_of(double x) {
+  const float hi = static_cast<float>(x);
+  const float lo = static_cast<float>(x - static_cast<double>(hi));
+  return expf(hi) * (1.0f + lo);
+}
+
+// ---------------------------------------------------------------- kernel 1
+// Shared memory of the chunk kernel (dynamic; about 200 KB).
+struct ChunkSmem {
+  double gam[kC][kK];               // Gamma_t - Gamma_r (fast path) or Gamma_t (exact path); 64 KB
+  float kt[kC][kK];                 // Kt = k exp(Gamma_t) [t][i]; the solve reads its columns
+  float at[kK][kC];                 // k_t exp(Gamma_t - Gamma_r) [i][t]
+  float aq[kK][kC];                 // q_t exp(Gamma_t - Gamma_r) [i][t]
+  float bk[kK][kC];                 // k_s exp(Gamma_r - Gamma_s) [i][s]
+  float L[kC][kC];                  // beta_t M[t][s] (s < t), zero elsewhere
+  float beta[kC];
+  int exact;                        // some channel is outside the factored path's range
+};
+// The raw bf16 inputs are staged over `at` .. `bk` before the factors are formed.
+struct ChunkRaw {
+  __nv_bfloat16 q[kC][kK];
+  __nv_bfloat16 k[kC][kK];
+  __nv_bfloat16 v[kC][kV];
+};
+static_assert(sizeof(ChunkRaw) <= 3 * kK * kC * sizeof(float), "raw inputs fit over the factor buffers");
+
+constexpr int kChunkThreads = 256;
+
+__global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(const Params p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ChunkSmem& sm = *reinterpret_cast<ChunkSmem*>(smem_raw);
+  ChunkRaw& raw = *reinterpret_cast<ChunkRaw*>(&sm.at[0][0]);
+
+  const int tid = threadIdx.x;
+  const int64_t unit = blockIdx.x / p.nchunks;  // n * HV + h
+  const int32_t chunk = static_cast<int32_t>(blockIdx.x - unit * p.nchunks);
+  const int64_t n = unit / p.HV;
+  const int64_t h = unit - n * p.HV;
+  const int64_t t0 = static_cast<int64_t>(chunk) * kC;
+  const int tc = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);  // tokens in this chunk
+  if (__ldg(p.slot_idx + n) < 0) return;  // inactive row: nothing to prepare
+
+  // ---- 1. stage q, k, v (bf16) and beta; g goes straight to fp64 cumulative sums
+  for (int c = tid; c < kC * (kK / 8); c += kChunkThreads) {  // q and k: 16 pieces of 16 B per row
+    const int t = c / (kK / 8), pc = c % (kK / 8);
+    if (t < tc) {
+      const int64_t row = ((n * p.T + t0 + t) * p.HV + h);
+      cp_async16(&raw.q[t][pc * 8], p.q + row * kK + pc * 8);
+      cp_async16(&raw.k[t][pc * 8], p.k + row * kK + pc * 8);
+      cp_async16(&raw.v[t][pc * 8], p.v + row * kV + pc * 8);
+    } else {
+      *reinterpret_cast<uint4*>(&raw.q[t][pc * 8]) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(&raw.k[t][pc * 8]) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(&raw.v[t][pc * 8]) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  cp_async_commit();
+  if (tid < kC) sm.beta[tid] = tid < tc ? __ldg(p.beta + (n * p.T + t0 + tid) * p.HV + h) : 0.f;
+  if (tid == 0) sm.exact = 0;
+
+  // Gamma per key channel (threads 0..127), summed in fp64; tokens past the
+  // chunk's end do not decay.  The reference token r is the chunk's middle.
+  constexpr int kRef = kC / 2 - 1;
+  if (tid < kK) {
+    const int i = tid;
+    double acc = 0.0;
+    for (int t = 0; t < kC; ++t) {
+      if (t < tc) acc += static_cast<double>(__ldg(p.g + ((n * p.T + t0 + t) * p.HV + h) * kK + i));
+      sm.gam[t][i] = acc;
+    }
+  }
+  __syncthreads();
+  double gam_end = 0.0, gam_ref = 0.0;  // per channel (threads 0..127)
+  if (tid < kK) {
+    gam_end = sm.gam[kC - 1][tid];
+    gam_ref = sm.gam[kRef][tid];
+    double worst = 0.0;
+    for (int t = 0; t < kC; ++t) {
+      const double d = sm.gam[t][tid] - gam_ref;
+      worst = fmax(worst, fabs(d));
+    }
+    if (worst > kSafeExp) atomicOr(&sm.exact, 1);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  const bool exact = sm.exact != 0;
+
+  // ---- 2. per-token decayed keys/queries (written straight to the workspace)
+  // and, on the factored path, the factors around the reference token.
+  float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
+  for (int e = tid; e < kC * kK; e += kChunkThreads) {
+    const int t = e / kK, i = e % kK;
+    const double gt = sm.gam[t][i];
+    const float kv = __bfloat162float(raw.k[t][i]);
+    const float qv = __bfloat162float(raw.q[t][i]);
+    const float d_t = exp_of(gt);                                    // exp(Gamma_t) <= 1
+    const float d_end = exp_of(sm.gam[kC - 1][i] - gt);              // exp(Gamma_C - Gamma_t) <= 1
+    sm.kt[t][i] = kv * d_t;
+    rec[Workspace::kKh + t * kK + i] = kv * d_end;
+    rec[Workspace::kQt + i * kC + t] = qv * d_t;
+  }
+  if (tid < kK) rec[Workspace::kDc + tid] = exp_of(gam_end);
+  __syncthreads();  // raw q/k still needed below; kt complete
+
+  // ---- 3. M and P
+  float* const Pt = rec + Workspace::kPt;  // Pt[s][t] = P[t][s]
+  if (!exact) {
+    // The factors go through registers: the raw inputs they are made from live
+    // in the buffers they are written to.
+    float fa[kC * kK / kChunkThreads], fq[kC * kK / kChunkThreads], fb[kC * kK / kChunkThreads];
+#pragma unroll
+    for (int j = 0; j < kC * kK / kChunkThreads; ++j) {
+      const int e = tid + j * kChunkThreads;
+      const int t = e / kK, i = e % kK;
+      const double d = sm.gam[t][i] - sm.gam[kRef][i];
+      const float kv = __bfloat162float(raw.k[t][i]);
+      fa[j] = kv * exp_of(d);
+      fq[j] = __bfloat162float(raw.q[t][i]) * exp_of(d);
+      fb[j] = kv * exp_of(-d);
+    }
+    __syncthreads();
+    // The solve needs v, which the factors overwrite: move it into the Gamma
+    // buffer (no longer needed on this path) as fp32 [t][j].
+    float* const vf = reinterpret_cast<float*>(&sm.gam[0][0]);
+    for (int e = tid; e < kC * kV; e += kChunkThreads) vf[e] = __bfloat162float(raw.v[e / kV][e % kV]);
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kC * kK / kChunkThreads; ++j) {
+      const int e = tid + j * kChunkThreads;
+      const int t = e / kK, i = e % kK;
+      sm.at[i][t] = fa[j];
+      sm.aq[i][t] = fq[j];
+      sm.bk[i][t] = fb[j];
+    }
+    __syncthreads();
+    // 4 x 4 tiles of (t, s); tiles above the diagonal are skipped
+    const int tb = tid / 16, sb = tid % 16;
+    float m[4][4], pp[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) m[a][b] = pp[a][b] = 0.f;
+    if (sb <= tb) {
+      for (int i = 0; i < kK; ++i) {
+        const float4 A = *reinterpret_cast<const float4*>(&sm.at[i][tb * 4]);
+        const float4 Q = *reinterpret_cast<const float4*>(&sm.aq[i][tb * 4]);
+        const float4 B = *reinterpret_cast<const float4*>(&sm.bk[i][sb * 4]);
+        const float av[4] = {A.x, A.y, A.z, A.w}, qv[4] = {Q.x, Q.y, Q.z, Q.w}, bv[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            m[a][b] = fmaf(av[a], bv[b], m[a][b]);
+            pp[a][b] = fmaf(qv[a], bv[b], pp[a][b]);
+          }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int t = tb * 4 + a;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int s = sb * 4 + b;
+        sm.L[t][s] = (s < t) ? sm.beta[t] * m[a][b] : 0.f;
+        Pt[s * kC + t] = (s <= t) ? pp[a][b] : 0.f;
+      }
+    }
+  } else {
+    // Exact path: every pair's exponential from the fp64 Gamma difference.
+    // One thread per (t, s) pair group; rare (decays beyond e^80 within half a chunk).
+    for (int e = tid; e < kC * kC; e += kChunkThreads) {
+      const int t = e / kC, s = e % kC;
+      float mv = 0.f, pv = 0.f;
+      if (s <= t) {
+        for (int i = 0; i < kK; ++i) {
+          const float w = __bfloat162float(raw.k[s][i]) * exp_of(sm.gam[t][i] - sm.gam[s][i]);
+          mv = fmaf(__bfloat162float(raw.k[t][i]), w, mv);
+          pv = fmaf(__bfloat162float(raw.q[t][i]), w, pv);
+        }
+      }
+      sm.L[t][s] = (s < t) ? sm.beta[t] * mv : 0.f;
+      Pt[s * kC + t] = (s <= t) ? pv : 0.f;
+    }
+    __syncthreads();
+    float* const vf = reinterpret_cast<float*>(&sm.gam[0][0]);
+    // gam is dead after the loop above; v moves there as on the fast path
+    float vtmp[kC * kV / kChunkThreads];
+#pragma unroll
+    for (int j = 0; j < kC * kV / kChunkThreads; ++j) {
+      const int e = tid + j * kChunkThreads;
+      vtmp[j] = __bfloat162float(raw.v[e / kV][e % kV]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kC * kV / kChunkThreads; ++j) vf[tid + j * kChunkThreads] = vtmp[j];
+  }
+  __syncthreads();
+
+  // ---- 4. forward substitution: X[t] = beta_t R[t] - sum_{s<t} L[t][s] X[s],
+  // R = [Kt | V]; thread j owns column j (j < K: W, else Ut).
+  {
+    const int j = tid;
+    const float* const vf = reinterpret_cast<const float*>(&sm.gam[0][0]);
+    float x[kC];
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      float acc = sm.beta[t] * (j < kK ? sm.kt[t][j] : vf[t * kV + (j - kK)]);
+#pragma unroll
+      for (int s = 0; s + 3 < t; s += 4) {
+        const float4 l = *reinterpret_cast<const float4*>(&sm.L[t][s]);
+        acc = fmaf(-l.x, x[s], acc);
+        acc = fmaf(-l.y, x[s + 1], acc);
+        acc = fmaf(-l.z, x[s + 2], acc);
+        acc = fmaf(-l.w, x[s + 3], acc);
+      }
+#pragma unroll
+      for (int s = t & ~3; s < t; ++s) acc = fmaf(-sm.L[t][s], x[s], acc);
+      x[t] = acc;
+    }
+    if (j < kK) {
+      float* const wt = rec + Workspace::kWt + j * kC;  // W^T row j
+#pragma unroll
+      for (int t = 0; t < kC; t += 4) *reinterpret_cast<float4*>(wt + t) = make_float4(x[t], x[t + 1], x[t + 2], x[t + 3]);
+    } else {
+      float* const ut = rec + Workspace::kUt + (j - kK);
+#pragma unroll
+      for (int t = 0; t < kC; ++t) ut[t * kV] = x[t];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- kernel 2
+constexpr int kStateThreads = 128;
+
+struct StateBuf {
+  float wt[kK][kC];   // W^T
+  float kh[kC][kK];   // Kh
+  float ut[kC][kBV];  // this tile's columns of Ut
+  float dc[kK];       // exp(Gamma_C)
+};
+struct StateSmem {
+  StateBuf buf[2];
+  float s[kK][kBV];   // state tile
+  float u[kC][kBV];   // corrections of the current chunk
+};
+
+__device__ __forceinline__ void stage_chunk(StateBuf& b, const float* rec, int col0, int tid) {
+  for (int c = tid; c < (kK * kC) / 4; c += kStateThreads) {
+    cp_async16(&b.wt[0][0] + 4 * c, rec + Workspace::kWt + 4 * c);
+    cp_async16(&b.kh[0][0] + 4 * c, rec + Workspace::kKh + 4 * c);
+  }
+  for (int c = tid; c < kC * (kBV / 4); c += kStateThreads) {
+    const int t = c / (kBV / 4), pc = c % (kBV / 4);
+    cp_async16(&b.ut[t][pc * 4], rec + Workspace::kUt + t * kV + col0 + pc * 4);
+  }
+  for (int c = tid; c < kK / 4; c += kStateThreads) cp_async16(&b.dc[4 * c], rec + Workspace::kDc + 4 * c);
+}
+
+__global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(const Params p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  StateSmem& sm = *reinterpret_cast<StateSmem*>(smem_raw);
+  constexpr int kTiles = kV / kBV;
+  const int tid = threadIdx.x;
+  const int64_t unit = blockIdx.x / kTiles;
+  const int tile = static_cast<int>(blockIdx.x - unit * kTiles);
+  const int col0 = tile * kBV;
+  const int64_t n = unit / p.HV;
+  const int64_t h = unit - n * p.HV;
+  const int32_t slot = __ldg(p.slot_idx + n);
+  if (slot < 0) return;
+
+  float* const blk = p.state + (static_cast<int64_t>(slot) * p.HV + h) * kK * kV;
+  // initial state tile
+  for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {
+    const int i = c / (kBV / 4), pc = c % (kBV / 4);
+    cp_async16(&sm.s[i][pc * 4], blk + i * kV + col0 + pc * 4);
+  }
+  stage_chunk(sm.buf[0], p.ws + Workspace::record(unit, 0, p.nchunks), col0, tid);
+  cp_async_commit();
+
+  // GEMM 1 tile: 4 tokens x 4 columns (16 x 4 threads... 128 threads: 16 token groups x 4 column groups x 2 halves of K)
+  const int g1_t = (tid % 16) * 4;      // tokens t0 .. t0+3
+  const int g1_j = ((tid / 16) % 4) * 4;  // columns j0 .. j0+3
+  const int g1_h = tid / 64;            // which half of K
+  // GEMM 2 tile: 4 key rows x 4 columns
+  const int g2_i = (tid % 32) * 4;
+  const int g2_j = (tid / 32) * 4;
+
+  for (int32_t c = 0; c < p.nchunks; ++c) {
+    const int cb = c & 1;
+    if (c + 1 < p.nchunks) {
+      stage_chunk(sm.buf[cb ^ 1], p.ws + Workspace::record(unit, c + 1, p.nchunks), col0, tid);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const StateBuf& b = sm.buf[cb];
+    float* const rec = p.ws + Workspace::record(unit, c, p.nchunks);
+
+    // chunk-start state to the workspace (the output kernel reads it)
+    for (int e = tid; e < kK * (kBV / 4); e += kStateThreads) {
+      const int i = e / (kBV / 4), pc = e % (kBV / 4);
+      *reinterpret_cast<float4*>(rec + Workspace::kS0 + i * kV + col0 + pc * 4) =
+          *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
+    }
+
+    // GEMM 1: partial (W S)[t][j] over half of K, the halves combined in smem
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
+    const int i_lo = g1_h * (kK / 2);
+#pragma unroll 8
+    for (int i = i_lo; i < i_lo + kK / 2; ++i) {
+      const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][g1_t]);
+      const float4 s = *reinterpret_cast<const float4*>(&sm.s[i][g1_j]);
+      const float wv[4] = {w.x, w.y, w.z, w.w}, sv[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(wv[a], sv[bb], acc[a][bb]);
+    }
+    if (g1_h == 1) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        *reinterpret_cast<float4*>(&sm.u[g1_t + a][g1_j]) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    }
+    __syncthreads();
+    if (g1_h == 0) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float4 o = *reinterpret_cast<const float4*>(&sm.u[g1_t + a][g1_j]);
+        const float4 ut = *reinterpret_cast<const float4*>(&b.ut[g1_t + a][g1_j]);
+        const float4 u = make_float4(ut.x - (acc[a][0] + o.x), ut.y - (acc[a][1] + o.y),
+                                     ut.z - (acc[a][2] + o.z), ut.w - (acc[a][3] + o.w));
+        *reinterpret_cast<float4*>(&sm.u[g1_t + a][g1_j]) = u;
+        *reinterpret_cast<float4*>(rec + Workspace::kU + (g1_t + a) * kV + col0 + g1_j) = u;
+      }
+    }
+    __syncthreads();
+
+    // GEMM 2: S = D S + Kh^T U
+    float sn[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float d = b.dc[g2_i + a];
+      const float4 s = *reinterpret_cast<const float4*>(&sm.s[g2_i + a][g2_j]);
+      sn[a][0] = d * s.x; sn[a][1] = d * s.y; sn[a][2] = d * s.z; sn[a][3] = d * s.w;
+    }
+#pragma unroll 8
+    for (int t = 0; t < kC; ++t) {
+      const float4 kh = *reinterpret_cast<const float4*>(&b.kh[t][g2_i]);
+      const float4 u = *reinterpret_cast<const float4*>(&sm.u[t][g2_j]);
+      const float kv[4] = {kh.x, kh.y, kh.z, kh.w}, uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) sn[a][bb] = fmaf(kv[a], uv[bb], sn[a][bb]);
+    }
+    __syncthreads();  // every thread is done reading s and the buffer
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+      *reinterpret_cast<float4*>(&sm.s[g2_i + a][g2_j]) = make_float4(sn[a][0], sn[a][1], sn[a][2], sn[a][3]);
+  }
+  __syncthreads();
+  for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {
+    const int i = c / (kBV / 4), pc = c % (kBV / 4);
+    *reinterpret_cast<float4*>(blk + i * kV + col0 + pc * 4) = *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
+  }
+}
+
+// ---------------------------------------------------------------- kernel 3
+constexpr int kOutThreads = 256;
+
+struct OutSmem {
+  float qt[kK][kC];   // Qt^T
+  float s0[kK][kV];   // chunk-start state
+  float pt[kC][kC];   // P^T
+  float u[kC][kV];    // U
+};
+
+__global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(const Params p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int64_t unit = blockIdx.x / p.nchunks;
+  const int32_t chunk = static_cast<int32_t>(blockIdx.x - unit * p.nchunks);
+  const int64_t n = unit / p.HV;
+  const int64_t h = unit - n * p.HV;
+  const int64_t t0 = static_cast<int64_t>(chunk) * kC;
+  const int tc = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
+  // thread tile: 4 tokens x 8 columns
+  const int ot = (tid % 16) * 4;
+  const int oj = (tid / 16) * 8;
+  if (__ldg(p.slot_idx + n) < 0) {  // inactive row: zero output
+    for (int a = 0; a < 4; ++a) {
+      if (ot + a < tc) {
+        __nv_bfloat16* o = p.out + ((n * p.T + t0 + ot + a) * p.HV + h) * kV + oj;
+        *reinterpret_cast<uint4*>(o) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    return;
+  }
+  const float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
+  for (int c = tid; c < (kK * kC) / 4; c += kOutThreads) cp_async16(&sm.qt[0][0] + 4 * c, rec + Workspace::kQt + 4 * c);
+  for (int c = tid; c < (kK * kV) / 4; c += kOutThreads) cp_async16(&sm.s0[0][0] + 4 * c, rec + Workspace::kS0 + 4 * c);
+  for (int c = tid; c < (kC * kC) / 4; c += kOutThreads) cp_async16(&sm.pt[0][0] + 4 * c, rec + Workspace::kPt + 4 * c);
+  for (int c = tid; c < (kC * kV) / 4; c += kOutThreads) cp_async16(&sm.u[0][0] + 4 * c, rec + Workspace::kU + 4 * c);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  float acc[4][8];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < kK; ++i) {
+    const float4 q = *reinterpret_cast<const float4*>(&sm.qt[i][ot]);
+    const float4 s0 = *reinterpret_cast<const float4*>(&sm.s0[i][oj]);
+    const float4 s1 = *reinterpret_cast<const float4*>(&sm.s0[i][oj + 4]);
+    const float qv[4] = {q.x, q.y, q.z, q.w}, sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(qv[a], sv[b], acc[a][b]);
+  }
+  const int s_end = ot + 4;  // P[t][s] = 0 for s > t
+  for (int s = 0; s < s_end; ++s) {
+    const float4 pq = *reinterpret_cast<const float4*>(&sm.pt[s][ot]);
+    const float4 u0 = *reinterpret_cast<const float4*>(&sm.u[s][oj]);
+    const float4 u1 = *reinterpret_cast<const float4*>(&sm.u[s][oj + 4]);
+    const float pv[4] = {pq.x, pq.y, pq.z, pq.w}, uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(pv[a], uv[b], acc[a][b]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    if (ot + a >= tc) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      __nv_bfloat162 x = __floats2bfloat162_rn(p.scale * acc[a][2 * b], p.scale * acc[a][2 * b + 1]);
+      w[b] = *reinterpret_cast<uint32_t*>(&x);
+    }
+    __nv_bfloat16* o = p.out + ((n * p.T + t0 + ot + a) * p.HV + h) * kV + oj;
+    *reinterpret_cast<uint4*>(o) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+constexpr int kChunkSmem = static_cast<int>(sizeof(ChunkSmem));
+constexpr int kStateSmem = static_cast<int>(sizeof(StateSmem));
+constexpr int kOutSmem = static_cast<int>(sizeof(OutSmem));
+
+}  // namespace kdap

@@ -196,9 +196,25 @@ CONFIGS = {
 }
 
 
+# Long token runs for the chunked prefill (kda_prefill): one prompt of 64, 1000
+# (a ragged last chunk) and 8192 tokens at 8 heads, and a batch of 8 prompts of
+# 1024 tokens.  The pages give no prefill shapes; these take the decode
+# serving shapes' 8 local heads and K = V = 128 (vLLM #57585, "Retained
+# baseline trace attribution") with prompt lengths of the long-context
+# serving runs it reports (2048-token and mixed 2048/32768-token inputs,
+# "Follow-up serving validation").
+PREFILL_CONFIGS = {
+    "prefill_n1_t64_hv8": dict(N=1, T=64, HV=8, num_slots=2),
+    "prefill_n1_t1000_hv8": dict(N=1, T=1000, HV=8, num_slots=2),
+    "prefill_n1_t8192_hv8": dict(N=1, T=8192, HV=8, num_slots=2),
+    "prefill_n8_t1024_hv8": dict(N=8, T=1024, HV=8, num_slots=16),
+}
+
+
 def config(name: str, seed: int = 0) -> Workload:
     """One of the named workloads (K = V = 128), drawn with ``seed``."""
-    return make(name=name, seed=seed, **CONFIGS[name])
+    kw = CONFIGS[name] if name in CONFIGS else PREFILL_CONFIGS[name]
+    return make(name=name, seed=seed, **kw)
 
 
 @dataclasses.dataclass

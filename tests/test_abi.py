@@ -21,6 +21,8 @@ from linear_attention_recurrent_decode_b200 import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kda_decode.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fabricated pointers: CPU-only check")
 
 
@@ -31,14 +33,19 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    return {re.findall(r"\w+", m)[-1] for m in re.findall(r"^KDA_API([^(;]*)\(", text, re.M)}
+    """Every function the headers under include/ declare."""
+    names = set()
+    for path in HEADERS:
+        text = open(path).read()
+        names |= {re.findall(r"\w+", m)[-1] for m in re.findall(r"^KDA_API([^(;]*)\(", text, re.M)}
+    return names
 
 
 def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
-                                    "kda_decode_host", "kda_status_string", "kda_abi_version"}
+                                    "kda_decode_host", "kda_status_string", "kda_abi_version",
+                                    "kda_prefill", "kda_prefill_workspace_bytes"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -235,6 +242,40 @@ def test_host_entry_point_validation(lib):
     assert call(hin=None, din=None, nbytes=0) == E.KDA_ERR_DEVICE  # nothing to copy in
     assert call(hout=None) == E.KDA_ERR_INVALID_ARG
     assert call(din=BASE + 5 * step - 64, nbytes=128) == E.KDA_ERR_ALIAS  # staging runs into the pool
+
+
+@no_gpu
+def test_prefill_validation(lib):
+    """kda_prefill's host checks, with fabricated addresses (rejected before any launch)."""
+    E = kda
+    step = 1 << 30
+    N, T, HV = 2, 100, 2
+    need = lib.kda_prefill_workspace_bytes(N, T, HV, 128, 128)
+    assert need == N * HV * 2 * 246272  # two chunks per (n, h) of 61,568 fp32 each
+    assert lib.kda_prefill_workspace_bytes(N, T, HV, 128, 64) == -1
+    assert lib.kda_prefill_workspace_bytes(-1, T, HV, 128, 128) == -1
+    assert lib.kda_prefill_workspace_bytes(N, 0, HV, 128, 128) == 0
+
+    def call(q=BASE, ws=BASE + 12 * step, wsb=None, out=BASE + 9 * step, K=128, V=128, n=N, t=T, g=BASE + 3 * step,
+             beta=BASE + 4 * step):
+        return lib.kda_prefill(q, BASE + step, BASE + 2 * step, g, beta, BASE + 5 * step, BASE + 8 * step, out,
+                               ws, need if wsb is None else wsb, n, t, HV, K, V, 0.1, None)
+
+    assert call() == E.KDA_ERR_DEVICE                         # valid, no device here
+    assert call(n=0, q=0, ws=0, out=0) == E.KDA_OK            # nothing to do
+    assert call(K=64) == E.KDA_ERR_UNSUPPORTED
+    assert call(V=256) == E.KDA_ERR_UNSUPPORTED
+    assert call(t=-1) == E.KDA_ERR_INVALID_ARG
+    assert call(q=0) == E.KDA_ERR_INVALID_ARG
+    assert call(ws=0) == E.KDA_ERR_INVALID_ARG
+    assert call(wsb=need - 1) == E.KDA_ERR_INVALID_ARG
+    assert call(q=BASE + 8) == E.KDA_ERR_MISALIGNED
+    assert call(ws=BASE + 12 * step + 4) == E.KDA_ERR_MISALIGNED
+    assert call(beta=BASE + 4 * step + 2) == E.KDA_ERR_MISALIGNED
+    assert call(out=BASE + 64) == E.KDA_ERR_ALIAS             # out over q
+    assert call(ws=BASE + 9 * step + 64) == E.KDA_ERR_ALIAS   # workspace over out
+    assert call(ws=BASE + 5 * step - 1024) == E.KDA_ERR_ALIAS # workspace runs into the pool
+    assert call(g=BASE + 5 * step + 4096) == E.KDA_ERR_ALIAS  # an input inside slot 0
 
 
 @pytest.mark.gpu
