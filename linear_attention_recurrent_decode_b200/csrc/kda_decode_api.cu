@@ -44,11 +44,16 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   if (gated && !(a.eps >= 0.0f && a.eps <= 3.0e38f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
   if (a.state_dtype != KDA_STATE_FP32 && a.state_dtype != KDA_STATE_BF16) return KDA_ERR_INVALID_ARG;
   if (a.state_layout != KDA_LAYOUT_KV && a.state_layout != KDA_LAYOUT_VK) return KDA_ERR_INVALID_ARG;
-  if (HV < 1) return KDA_ERR_UNSUPPORTED;
-  if (K != 64 && K != 128 && K != 256) return KDA_ERR_UNSUPPORTED;
-  if (V < kda::kBV || V % kda::kBV != 0) return KDA_ERR_UNSUPPORTED;
-  const int64_t tiles = V / kda::kBV;
+  if (HV < 1 || K < 1 || K > 256 || V < 1) return KDA_ERR_UNSUPPORTED;
+  // The vectorised kernels take K in {64, 128, 256} and V a multiple of 32;
+  // any other K <= 256 and V run the general (masked, element-wise) form of
+  // the same kernels on K padded to 64, 128 or 256 rows.
+  const bool general = !((K == 64 || K == 128 || K == 256) && V % kda::kBV == 0);
+  const int64_t K_pad = K <= 64 ? 64 : (K <= 128 ? 128 : 256);
+  const int64_t tiles = (V + kda::kBV - 1) / kda::kBV;
   if (gated && tiles > kda::kMaxClusterTiles) return KDA_ERR_UNSUPPORTED;
+  if (general && (a.state_layout != KDA_LAYOUT_KV || a.raw_gate != nullptr || a.raw_beta != nullptr))
+    return KDA_ERR_UNSUPPORTED;  // the general form takes [K][V] blocks and activated g, beta
   if (N == 0 || T == 0) return KDA_OK;  // nothing to do; no pointer is touched
 
   int64_t rows, hk, hvv, grid, out_elems;
@@ -71,21 +76,25 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   if (gated && (!a.gate || !a.norm_weight)) return KDA_ERR_INVALID_ARG;
   const void* gsrc = raw ? a.raw_gate : static_cast<const void*>(a.g);
   const void* bsrc = raw ? a.raw_beta : static_cast<const void*>(a.beta);
-  if (!aligned(a.q, 16) || !aligned(a.k, 16) || !aligned(a.v, 16) || !aligned(gsrc, 16) ||
-      !aligned(a.state_pool, 16) || !aligned(a.out, 16) || !aligned(bsrc, raw ? 2 : 4) ||
+  const bool bf16_pool = a.state_dtype == KDA_STATE_BF16;
+  // The vectorised kernels read 16-byte pieces; the general form reads element
+  // by element and needs only each element's own alignment.
+  const uintptr_t va = general ? 2 : 16, ga = general ? 4 : 16, sa = general ? (bf16_pool ? 2 : 4) : 16;
+  if (!aligned(a.q, va) || !aligned(a.k, va) || !aligned(a.v, va) || !aligned(gsrc, ga) ||
+      !aligned(a.state_pool, sa) || !aligned(a.out, va) || !aligned(bsrc, raw ? 2 : 4) ||
       !aligned(a.slot_idx, 4))
     return KDA_ERR_MISALIGNED;
   if (raw && (!aligned(a.dt_bias, 16) || !aligned(a.A_log, 4))) return KDA_ERR_MISALIGNED;
   if (a.status && !aligned(a.status, 4)) return KDA_ERR_MISALIGNED;
-  if (gated && (!aligned(a.gate, 16) || !aligned(a.norm_weight, 16))) return KDA_ERR_MISALIGNED;
+  if (gated && (!aligned(a.gate, va) || !aligned(a.norm_weight, va))) return KDA_ERR_MISALIGNED;
 
-  // ---- row strides: at least one row, and 16-byte aligned rows for the vector loads
+  // ---- row strides: at least one row, and (vectorised kernels) 16-byte aligned rows
   const int64_t g_elem = raw ? 2 : 4;
   if (a.q_row_stride < hk || a.k_row_stride < hk || a.v_row_stride < hvv || a.g_row_stride < hk ||
       a.beta_row_stride < HV || (gated && a.gate_row_stride < hvv))
     return KDA_ERR_INVALID_ARG;
-  if (a.q_row_stride % 8 || a.k_row_stride % 8 || a.v_row_stride % 8 ||
-      (a.g_row_stride * g_elem) % 16 || (gated && a.gate_row_stride % 8))
+  if (!general && (a.q_row_stride % 8 || a.k_row_stride % 8 || a.v_row_stride % 8 ||
+                   (a.g_row_stride * g_elem) % 16 || (gated && a.gate_row_stride % 8)))
     return KDA_ERR_MISALIGNED;
 
   // ---- aliasing: out must not overlap any input or the pool
@@ -158,6 +167,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   p.eps = a.eps;
   p.num_slots = a.num_slots;
   p.status = a.status;
+  p.k_rt = static_cast<int32_t>(K);
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -187,7 +197,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   const bool dense = a.q_row_stride == hk && a.k_row_stride == hk && a.v_row_stride == hvv &&
                      a.g_row_stride == hk && a.beta_row_stride == HV && (!gated || a.gate_row_stride == hvv) &&
                      a.num_slots == 0;
-  const int form = raw ? kda::kInRaw : dense ? kda::kInDense : kda::kInStrided;
+  const int form = general ? kda::kInGeneral : raw ? kda::kInRaw : dense ? kda::kInDense : kda::kInStrided;
 
   // Pick the kernel (and make its dynamic shared memory allowance) before
   // anything is enqueued.
@@ -204,7 +214,7 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
   choice.tiles = static_cast<int>(tiles);
   choice.check_launch = hc != nullptr;
   cudaError_t err = cudaErrorInvalidValue;
-  switch (K) {
+  switch (K_pad) {
     case 64: err = kda::pick_decode_kernel<64>(choice, &func, &smem); break;
     case 128: err = kda::pick_decode_kernel<128>(choice, &func, &smem); break;
     case 256: err = kda::pick_decode_kernel<256>(choice, &func, &smem); break;
@@ -327,8 +337,9 @@ const char* kda_status_string(kda_status status) {
     case KDA_OK: return "ok";
     case KDA_ERR_INVALID_ARG:
       return "invalid argument (null pointer, negative size, bad eps, short row stride or mixed input forms)";
-    case KDA_ERR_UNSUPPORTED: return "unsupported size (K must be 64/128/256, V a multiple of 32, "
-                                     "V <= 256 when gated, HV >= 1)";
+    case KDA_ERR_UNSUPPORTED: return "unsupported size or form (K in 1..256, V >= 1, V <= 256 when gated, "
+                                     "HV >= 1; K outside {64,128,256} or V not a multiple of 32 only with "
+                                     "[K][V] blocks and activated g, beta; prefill: K = V = 128)";
     case KDA_ERR_ALIAS: return "output overlaps an input or the state pool";
     case KDA_ERR_MISALIGNED: return "misaligned pointer or row stride";
     case KDA_ERR_DEVICE: return "current device is not compute capability 10.0 (sm_100a)";

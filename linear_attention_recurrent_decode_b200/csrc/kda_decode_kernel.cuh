@@ -127,6 +127,9 @@ struct ParamsEx : Params {
   // inactive row and stores 1 to *status (when not null).
   int64_t num_slots;
   int32_t* status;
+  // General form only: the run-time key width (the kernel's K is its padded
+  // row count).
+  int32_t k_rt;
 };
 
 // How a kernel addresses its per-token inputs and which decay/beta inputs it
@@ -136,6 +139,10 @@ enum InputForm : int {
   kInDense = 0,    // q, k, v, g, beta, gate dense [N, T, HV, ...]; activated g and beta
   kInStrided = 1,  // row-strided views; activated g and beta
   kInRaw = 2,      // row-strided views; raw gate and beta, activated in the kernel
+  // Any K <= the kernel's K and any V: row-strided views read element by
+  // element, key rows >= k_rt and value columns >= V masked to zero (never
+  // read or written).  [K][V] pool blocks, activated g and beta.
+  kInGeneral = 3,
 };
 template <int IN>
 using ParamsOf = typename std::conditional<IN == kInDense, Params, ParamsEx>::type;
@@ -240,6 +247,78 @@ __device__ __forceinline__ void ld_f32_rows(float (&d)[NF], const float* p) {
     d[4 * i + 0] = x.x; d[4 * i + 1] = x.y; d[4 * i + 2] = x.z; d[4 * i + 3] = x.w;
   }
 }
+
+// General form: RPT consecutive rows starting at key row r0, element by element,
+// zero for rows at or past k_rt.
+template <int RPT>
+__device__ __forceinline__ void ld_bf16_rows_masked(uint32_t (&w)[RPT / 2], const __nv_bfloat16* p, int r0,
+                                                    int k_rt) {
+  const unsigned short* u = reinterpret_cast<const unsigned short*>(p);
+#pragma unroll
+  for (int i = 0; i < RPT / 2; ++i) {
+    const uint32_t lo = r0 + 2 * i < k_rt ? __ldg(u + 2 * i) : 0u;
+    const uint32_t hi = r0 + 2 * i + 1 < k_rt ? __ldg(u + 2 * i + 1) : 0u;
+    w[i] = lo | (hi << 16);
+  }
+}
+template <int NF>
+__device__ __forceinline__ void ld_f32_rows_masked(float (&d)[NF], const float* p, int r0, int k_rt) {
+#pragma unroll
+  for (int i = 0; i < NF; ++i) d[i] = r0 + i < k_rt ? __ldg(p + i) : 0.f;
+}
+// Four consecutive bf16 values of a row, element by element, zero at or past
+// column `lim` (the row's value count) from column `c`.
+__device__ __forceinline__ void ld_bf16x4_masked(uint32_t (&w)[2], const __nv_bfloat16* p, int64_t c, int64_t lim) {
+  const unsigned short* u = reinterpret_cast<const unsigned short*>(p);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t lo = c + 2 * i < lim ? __ldg(u + 2 * i) : 0u;
+    const uint32_t hi = c + 2 * i + 1 < lim ? __ldg(u + 2 * i + 1) : 0u;
+    w[i] = lo | (hi << 16);
+  }
+}
+__device__ __forceinline__ void st_bf16x4_masked(__nv_bfloat16* p, const float (&y)[4], int64_t c, int64_t lim) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (c + j < lim) p[j] = __float2bfloat16_rn(y[j]);
+}
+
+// General form: a thread's state tile (rows r0 .. r0+RPT-1, columns c .. c+3)
+// element by element in a [K][V] block of run-time size, masked to the block.
+template <typename ST, int RPT>
+struct MaskedTile {
+  static __device__ __forceinline__ ST* base(void* pool, int64_t slot, int64_t HV, int64_t h, int64_t k_rt,
+                                             int64_t V, int r0, int64_t c) {
+    return static_cast<ST*>(pool) + (slot * HV + h) * k_rt * V + static_cast<int64_t>(r0) * V + c;
+  }
+  static __device__ __forceinline__ float rd(const float* p) { return *p; }
+  static __device__ __forceinline__ float rd(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ void wr(float* p, float x) { __stcs(p, x); }
+  static __device__ __forceinline__ void wr(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+  static __device__ __forceinline__ void load(float2 (&s)[RPT][2], const ST* b, int64_t V, int r0, int k_rt,
+                                              int64_t c) {
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      const bool row = r0 + i < k_rt;
+      float x[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[j] = (row && c + j < V) ? rd(b + i * V + j) : 0.f;
+      s[i][0] = make_float2(x[0], x[1]);
+      s[i][1] = make_float2(x[2], x[3]);
+    }
+  }
+  static __device__ __forceinline__ void store(ST* b, const float2 (&s)[RPT][2], int64_t V, int r0, int k_rt,
+                                               int64_t c) {
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      if (r0 + i >= k_rt) continue;
+      const float x[4] = {s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (c + j < V) wr(b + i * V + j, x[j]);
+    }
+  }
+};
 
 // Inputs of one token for one thread: its RPT key rows of q, k, g, its 4 value
 // columns of v (and of the gate z), and beta.
@@ -454,6 +533,37 @@ struct alignas(16) TokenSmem {
 template <int K, bool GATED, int IN>
 __device__ __forceinline__ void stage_tokens(TokenSmem<K>* buf, const ParamsOf<IN>& p, int64_t V, int64_t n,
                                              int64_t h, int64_t col0, int64_t t0, int cnt) {
+  if constexpr (IN == kInGeneral) {
+    // element by element (rows need not be 16-byte aligned), zero past k_rt
+    // and V; synchronous loads, so the caller's cp.async waits are no-ops here
+    const int k_rt = p.k_rt;
+    constexpr int kPer = 3 * K + 2 * kBV + 1;
+    for (int c = threadIdx.x; c < cnt * kPer; c += kThreads) {
+      const int j = c / kPer;
+      int r = c - j * kPer;
+      const int64_t nt = n * p.T + t0 + j;
+      const int64_t row = nt * p.HV + h;
+      TokenSmem<K>& s = buf[j];
+      if (r < K) { s.q[r] = r < k_rt ? p.q[in_off<IN, kRowQ>(p, row, nt, h, k_rt) + r] : __float2bfloat16(0.f); continue; }
+      r -= K;
+      if (r < K) { s.k[r] = r < k_rt ? p.k[in_off<IN, kRowK>(p, row, nt, h, k_rt) + r] : __float2bfloat16(0.f); continue; }
+      r -= K;
+      if (r < K) { s.g[r] = r < k_rt ? __ldg(p.g + in_off<IN, kRowG>(p, row, nt, h, k_rt) + r) : 0.f; continue; }
+      r -= K;
+      if (r < kBV) {
+        s.v[r] = col0 + r < V ? p.v[in_off<IN, kRowV>(p, row, nt, h, V) + col0 + r] : __float2bfloat16(0.f);
+        continue;
+      }
+      r -= kBV;
+      if (r < kBV) {
+        if constexpr (GATED)
+          s.z[r] = col0 + r < V ? p.gate[in_off<IN, kRowZ>(p, row, nt, h, V) + col0 + r] : __float2bfloat16(0.f);
+        continue;
+      }
+      s.beta[0] = __ldg(p.beta + in_off<IN, kRowB>(p, row, nt, h, 1));
+    }
+    return;
+  }
   constexpr bool RAW = IN == kInRaw;
   constexpr int kQ = K * 2 / 16;    // 16-byte chunks of q (and of k)
   constexpr int kG = (RAW ? K * 2 : K * 4) / 16;  // of g (fp32) or raw_gate (bf16, into the g slot)
@@ -603,6 +713,7 @@ template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
 __global__ void __launch_bounds__(kThreads, (MinBlocksT1<K, VS, GATED>::value))
 kda_decode_kernel(const ParamsOf<IN> p) {
   constexpr bool RAW = IN == kInRaw;
+  constexpr bool GEN = IN == kInGeneral;  // run-time K <= K, any V, masked element access
   constexpr int RPT = K / (kWarps * kRowGroups);
   static_assert(RPT * kWarps * kRowGroups == K && (RPT == 4 || RPT % 8 == 0), "K in {64,128,256}");
 
@@ -625,6 +736,8 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   const int64_t col = static_cast<int64_t>(tile) * kBV + cq * 4;
   const bool writer = (warp == 0) && (rg == 0);  // 8 lanes store the tile's 32 outputs
   const int64_t row = n * p.HV + h;              // (n, t = 0, h) of the dense output
+  int k_rt = K;                                   // key rows of the block (the general form's k_rt)
+  if constexpr (GEN) k_rt = p.k_rt;
 
   wait_prior_grids();
   const int32_t slot = __ldg(p.slot_idx + n);
@@ -634,8 +747,13 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   // code measured 1.5 % faster at the one-wave headline shape than the same
   // offsets taken through in_off.
   TokenIn<RPT> cur;
-  ld_bf16_rows<RPT>(cur.q, p.q + (IN == kInDense ? row * K : in_off<IN, kRowQ>(p, row, n, h, K)) + r0);
-  ld_bf16_rows<RPT>(cur.k, p.k + (IN == kInDense ? row * K : in_off<IN, kRowK>(p, row, n, h, K)) + r0);
+  if constexpr (GEN) {
+    ld_bf16_rows_masked<RPT>(cur.q, p.q + in_off<IN, kRowQ>(p, row, n, h, k_rt) + r0, r0, k_rt);
+    ld_bf16_rows_masked<RPT>(cur.k, p.k + in_off<IN, kRowK>(p, row, n, h, k_rt) + r0, r0, k_rt);
+  } else {
+    ld_bf16_rows<RPT>(cur.q, p.q + (IN == kInDense ? row * K : in_off<IN, kRowQ>(p, row, n, h, K)) + r0);
+    ld_bf16_rows<RPT>(cur.k, p.k + (IN == kInDense ? row * K : in_off<IN, kRowK>(p, row, n, h, K)) + r0);
+  }
   // Serving form: the 8 column-quad lanes of a row group share its RPT rows,
   // so each lane activates the rows i = cq (mod 8) and the decays travel by
   // shuffle; otherwise every thread reads its rows' log-decays.
@@ -648,14 +766,21 @@ kda_decode_kernel(const ParamsOf<IN> p) {
       graw[j] = __bfloat162float(p.raw_gate[in_off<IN, kRowG>(p, row, n, h, K) + r0 + i]);
       dtb[j] = __ldg(p.dt_bias + h * K + r0 + i);
     }
+  } else if constexpr (GEN) {
+    ld_f32_rows_masked<RPT>(cur.g, p.g + in_off<IN, kRowG>(p, row, n, h, k_rt) + r0, r0, k_rt);
   } else {
     ld_f32_rows<RPT>(cur.g, p.g + (IN == kInDense ? row * K : in_off<IN, kRowG>(p, row, n, h, K)) + r0);
   }
-  const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + (IN == kInDense ? row * V : in_off<IN, kRowV>(p, row, n, h, V)) + col));
-  cur.v[0] = vv_raw.x; cur.v[1] = vv_raw.y;
-  if constexpr (GATED) {
-    const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + col));
-    cur.z[0] = zz.x; cur.z[1] = zz.y;
+  if constexpr (GEN) {
+    ld_bf16x4_masked(cur.v, p.v + in_off<IN, kRowV>(p, row, n, h, V) + col, col, V);
+    if constexpr (GATED) ld_bf16x4_masked(cur.z, p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + col, col, V);
+  } else {
+    const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + (IN == kInDense ? row * V : in_off<IN, kRowV>(p, row, n, h, V)) + col));
+    cur.v[0] = vv_raw.x; cur.v[1] = vv_raw.y;
+    if constexpr (GATED) {
+      const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + col));
+      cur.z[0] = zz.x; cur.z[1] = zz.y;
+    }
   }
   if constexpr (RAW) {
     cur.beta = sigmoid_f(__bfloat162float(p.raw_beta[in_off<IN, kRowB>(p, row, n, h, 1)]));
@@ -672,24 +797,39 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   }
 
   if (!row_active<IN>(p, slot)) {  // inactive (padding) row: zero output, pool untouched
-    if (writer) *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(0u, 0u);
+    if (writer) {
+      if constexpr (GEN) {
+        const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+        st_bf16x4_masked(p.out + row * V + col, zero, col, V);
+      } else {
+        *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(0u, 0u);
+      }
+    }
     return;  // uniform over the cluster: every tile of this (n, h) sees the same slot
   }
 
   using Tile = TileIO<ST, VK, K, RPT>;
   extern __shared__ __align__(16) unsigned char dyn_smem[];  // [V][K] staging (VK kernels only)
   auto& stage = *reinterpret_cast<typename Tile::Stage*>(dyn_smem);
-  ST* const sp = Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
+  ST* const sp = GEN ? MaskedTile<ST, RPT>::base(p.state, slot, p.HV, h, k_rt, V, r0, col)
+                     : Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
   float2 s[RPT][2];
-  Tile::load(s, sp, V, stage, r0, cq);
+  if constexpr (GEN) MaskedTile<ST, RPT>::load(s, sp, V, r0, k_rt, col);
+  else Tile::load(s, sp, V, stage, r0, cq);
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
   float2 wgt[2] = {f2(0.f), f2(0.f)};
   if constexpr (GATED) {
-    const uint2 w = __ldg(reinterpret_cast<const uint2*>(p.norm_weight + col));
-    wgt[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
-    wgt[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+    uint32_t w[2];
+    if constexpr (GEN) {
+      ld_bf16x4_masked(w, p.norm_weight + col, col, V);
+    } else {
+      const uint2 x = __ldg(reinterpret_cast<const uint2*>(p.norm_weight + col));
+      w[0] = x.x; w[1] = x.y;
+    }
+    wgt[0] = make_float2(bf16lo(w[0]), bf16hi(w[0]));
+    wgt[1] = make_float2(bf16lo(w[1]), bf16hi(w[1]));
   }
 
   // decay and the partial reductions over this thread's rows
@@ -731,13 +871,20 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   }
 
   if constexpr (!GATED) {
-    if (writer)
-      *reinterpret_cast<uint2*>(p.out + row * V + col) =
-          make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
+    if (writer) {
+      if constexpr (GEN) {
+        const float y[4] = {o[0].x, o[0].y, o[1].x, o[1].y};
+        st_bf16x4_masked(p.out + row * V + col, y, col, V);
+      } else {
+        *reinterpret_cast<uint2*>(p.out + row * V + col) =
+            make_uint2(pack_bf16x2(o[0].x, o[0].y), pack_bf16x2(o[1].x, o[1].y));
+      }
+    }
   }
 
   allow_next_grid();
-  Tile::store(sp, s, V, stage, r0, cq);
+  if constexpr (GEN) MaskedTile<ST, RPT>::store(sp, s, V, r0, k_rt, col);
+  else Tile::store(sp, s, V, stage, r0, cq);
 
   if constexpr (GATED) {
     // The norm needs the whole head's o; the state does not, so it is
@@ -745,8 +892,10 @@ kda_decode_kernel(const ParamsOf<IN> p) {
     cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
     float y[4];
     gated_norm(y, o, wgt, cur.z, nrm, tile, tiles, V, p.eps, writer, lane);
-    if (writer)
-      *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+    if (writer) {
+      if constexpr (GEN) st_bf16x4_masked(p.out + row * V + col, y, col, V);
+      else *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+    }
   }
 }
 
@@ -904,6 +1053,7 @@ template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
 __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkBuffers<K, GATED>& b,
                                              typename TileIO<ST, VK, K, K / 16>::Stage& stage) {
   constexpr bool RAW = IN == kInRaw;
+  constexpr bool GEN = IN == kInGeneral;  // run-time K <= K, any V, masked element access
   constexpr int RPT = K / (kWarps * kRowGroups);
   using Tile = TileIO<ST, VK, K, RPT>;
   auto& tok = b.tok;
@@ -930,6 +1080,8 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
   const int64_t col0 = static_cast<int64_t>(tile) * kBV;
   const int64_t col = col0 + cq * 4;
   const bool writer = (warp == 0) && (rg == 0);
+  int k_rt = K;  // key rows of the block (the general form's k_rt)
+  if constexpr (GEN) k_rt = p.k_rt;
 
   wait_prior_grids();
   const int32_t slot = __ldg(p.slot_idx + n);
@@ -951,21 +1103,30 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
   // The norm weight, also ahead of the state loads.
   [[maybe_unused]] float wj = 0.f;  // gated: norm weight of this lane's solve column (warp 0)
   if constexpr (GATED) {
-    if (warp == 0) wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + rg]);
+    if (warp == 0 && (!GEN || col0 + 4 * cq + rg < V)) wj = __bfloat162float(p.norm_weight[col0 + 4 * cq + rg]);
   }
 
   if (!row_active<IN>(p, slot)) {  // inactive (padding) row: zero output, pool untouched
     cp_async_wait<0>();
     if (writer) {
-      for (int64_t t = 0; t < p.T; ++t)
-        *reinterpret_cast<uint2*>(p.out + ((n * p.T + t) * p.HV + h) * V + col) = make_uint2(0u, 0u);
+      for (int64_t t = 0; t < p.T; ++t) {
+        __nv_bfloat16* const o = p.out + ((n * p.T + t) * p.HV + h) * V + col;
+        if constexpr (GEN) {
+          const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+          st_bf16x4_masked(o, zero, col, V);
+        } else {
+          *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
+        }
+      }
     }
     return;
   }
 
-  ST* const sp = Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
+  ST* const sp = GEN ? MaskedTile<ST, RPT>::base(p.state, slot, p.HV, h, k_rt, V, r0, col)
+                     : Tile::base(p.state, slot, p.HV, h, V, r0, col - 4 * cq, cq);
   float2 s[RPT][2];
-  Tile::load(s, sp, V, stage, r0, cq);
+  if constexpr (GEN) MaskedTile<ST, RPT>::load(s, sp, V, r0, k_rt, col);
+  else Tile::load(s, sp, V, stage, r0, cq);
 
   if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
 
@@ -1047,7 +1208,7 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
             o *= p.scale;
             if constexpr (GATED) {
               osm[t][4 * cq + jc] = o;  // until the chunk's exchange
-            } else {
+            } else if (!GEN || col0 + 4 * cq + jc < V) {
               p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(o);
             }
           }
@@ -1106,7 +1267,8 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
               const float inv = rsqrtf(tot / static_cast<float>(V) + p.eps);
               const float z = __bfloat162float(tok[cb][t].z[4 * cq + jc]);
               const float y = osm[t][4 * cq + jc] * inv * wj * (1.0f / (1.0f + __expf(-z)));
-              p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(y);
+              if (!GEN || col0 + 4 * cq + jc < V)
+                p.out[((n * p.T + c0 + t) * p.HV + h) * V + col0 + 4 * cq + jc] = __float2bfloat16_rn(y);
             }
           }
         }
@@ -1118,7 +1280,8 @@ __device__ __forceinline__ void chunked_body(const ParamsOf<IN>& p, const ChunkB
   }
 
   allow_next_grid();
-  Tile::store(sp, s, V, stage, r0, cq);
+  if constexpr (GEN) MaskedTile<ST, RPT>::store(sp, s, V, r0, k_rt, col);
+  else Tile::store(sp, s, V, stage, r0, cq);
 }
 
 template <int K, int VS, bool GATED, typename ST, int IN, bool VK>

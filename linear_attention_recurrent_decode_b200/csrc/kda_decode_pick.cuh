@@ -111,7 +111,15 @@ cudaError_t pick_decode_kernel(const KernelChoice& c, const void** func, int* sm
   } while (0)
 #define KDA_PICK_V(KK, GG)                                              \
   do {                                                                  \
-    if (c.multi) {                                                      \
+    if (form == kInGeneral) {                                           \
+      if (c.multi) {                                                    \
+        if (bf16_state) KDA_PICK_ONE(kda_decode_chunked_kernel, KK, 0, GG, __nv_bfloat16, kInGeneral, false); \
+        else KDA_PICK_ONE(kda_decode_chunked_kernel, KK, 0, GG, float, kInGeneral, false);                     \
+      } else {                                                          \
+        if (bf16_state) KDA_PICK_ONE(kda_decode_kernel, KK, 0, GG, __nv_bfloat16, kInGeneral, false);         \
+        else KDA_PICK_ONE(kda_decode_kernel, KK, 0, GG, float, kInGeneral, false);                             \
+      }                                                                 \
+    } else if (c.multi) {                                               \
       if (c.v128) KDA_PICK(kda_decode_chunked_kernel, KK, 128, GG);     \
       else KDA_PICK(kda_decode_chunked_kernel, KK, 0, GG);              \
     } else {                                                            \

@@ -158,9 +158,16 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       *reinterpret_cast<uint4*>(&raw.v[t][pc * 8]) = make_uint4(0, 0, 0, 0);
     }
   }
+  // g goes through the kt buffer (free until step 2): 32 pieces of 16 B per row
+  for (int c = tid; c < tc * (kK / 4); c += kChunkThreads) {
+    const int t = c / (kK / 4), pc = c % (kK / 4);
+    cp_async16(&sm.kt[t][pc * 4], p.g + ((n * p.T + t0 + t) * p.HV + h) * kK + pc * 4);
+  }
   cp_async_commit();
   if (tid < kC) sm.beta[tid] = tid < tc ? __ldg(p.beta + (n * p.T + t0 + tid) * p.HV + h) : 0.f;
   if (tid == 0) sm.exact = 0;
+  cp_async_wait<0>();
+  __syncthreads();
 
   // Gamma per key channel (threads 0..127), summed in fp64; tokens past the
   // chunk's end do not decay.  The reference token r is the chunk's middle.
@@ -168,8 +175,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   if (tid < kK) {
     const int i = tid;
     double acc = 0.0;
+#pragma unroll 8
     for (int t = 0; t < kC; ++t) {
-      if (t < tc) acc += static_cast<double>(__ldg(p.g + ((n * p.T + t0 + t) * p.HV + h) * kK + i));
+      if (t < tc) acc += static_cast<double>(sm.kt[t][i]);
       sm.gam[t][i] = acc;
     }
   }
@@ -185,23 +193,22 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
     }
     if (worst > kSafeExp) atomicOr(&sm.exact, 1);
   }
-  cp_async_wait<0>();
   __syncthreads();
   const bool exact = sm.exact != 0;
 
   // ---- 2. per-token decayed keys/queries (written straight to the workspace)
   // and, on the factored path, the factors around the reference token.
   float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
-  for (int e = tid; e < kC * kK; e += kChunkThreads) {
+  for (int e = tid; e < kC * kK; e += kChunkThreads) {  // [t][i] order: consecutive threads, consecutive i
     const int t = e / kK, i = e % kK;
     const double gt = sm.gam[t][i];
     const float kv = __bfloat162float(raw.k[t][i]);
-    const float qv = __bfloat162float(raw.q[t][i]);
-    const float d_t = exp_of(gt);                                    // exp(Gamma_t) <= 1
-    const float d_end = exp_of(sm.gam[kC - 1][i] - gt);              // exp(Gamma_C - Gamma_t) <= 1
-    sm.kt[t][i] = kv * d_t;
-    rec[Workspace::kKh + t * kK + i] = kv * d_end;
-    rec[Workspace::kQt + i * kC + t] = qv * d_t;
+    sm.kt[t][i] = kv * exp_of(gt);                                   // k exp(Gamma_t)
+    rec[Workspace::kKh + t * kK + i] = kv * exp_of(sm.gam[kC - 1][i] - gt);  // k exp(Gamma_C - Gamma_t)
+  }
+  for (int e = tid; e < kC * kK; e += kChunkThreads) {  // [i][t] order for the transposed store
+    const int i = e / kC, t = e % kC;
+    rec[Workspace::kQt + i * kC + t] = __bfloat162float(raw.q[t][i]) * exp_of(sm.gam[t][i]);
   }
   if (tid < kK) rec[Workspace::kDc + tid] = exp_of(gam_end);
   __syncthreads();  // raw q/k still needed below; kt complete
@@ -334,7 +341,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
 }
 
 // ---------------------------------------------------------------- kernel 2
-constexpr int kStateThreads = 128;
+constexpr int kStateThreads = 256;
 
 struct StateBuf {
   float wt[kK][kC];   // W^T
@@ -344,8 +351,8 @@ struct StateBuf {
 };
 struct StateSmem {
   StateBuf buf[2];
-  float s[kK][kBV];   // state tile
-  float u[kC][kBV];   // corrections of the current chunk
+  float s[kK][kBV];      // state tile
+  float part[4][kC][kBV];  // (W S) partial sums over quarters of K; part[0] then holds U
 };
 
 __device__ __forceinline__ void stage_chunk(StateBuf& b, const float* rec, int col0, int tid) {
@@ -382,13 +389,15 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
   stage_chunk(sm.buf[0], p.ws + Workspace::record(unit, 0, p.nchunks), col0, tid);
   cp_async_commit();
 
-  // GEMM 1 tile: 4 tokens x 4 columns (16 x 4 threads... 128 threads: 16 token groups x 4 column groups x 2 halves of K)
-  const int g1_t = (tid % 16) * 4;      // tokens t0 .. t0+3
-  const int g1_j = ((tid / 16) % 4) * 4;  // columns j0 .. j0+3
-  const int g1_h = tid / 64;            // which half of K
-  // GEMM 2 tile: 4 key rows x 4 columns
-  const int g2_i = (tid % 32) * 4;
-  const int g2_j = (tid / 32) * 4;
+  // GEMM 1 (W S over a quarter of K): 4 tokens x 4 columns per thread
+  const int g1_t = (tid % 16) * 4;
+  const int g1_j = ((tid / 16) % 4) * 4;
+  const int g1_q = tid / 64;  // quarter of K
+  // U = Ut - sum of the quarters: 4 elements per thread
+  const int u_t = tid / 4, u_j = (tid % 4) * 4;
+  // GEMM 2 (Kh^T U): 2 key rows x 4 columns per thread
+  const int g2_i = (tid % 64) * 2;
+  const int g2_j = (tid / 64) * 4;
 
   for (int32_t c = 0; c < p.nchunks; ++c) {
     const int cb = c & 1;
@@ -410,63 +419,65 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
           *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
     }
 
-    // GEMM 1: partial (W S)[t][j] over half of K, the halves combined in smem
-    float acc[4][4];
+    // GEMM 1: partial (W S)[t][j] over one quarter of K
+    {
+      float acc[4][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
-    const int i_lo = g1_h * (kK / 2);
+        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
+      const int i_lo = g1_q * (kK / 4);
 #pragma unroll 8
-    for (int i = i_lo; i < i_lo + kK / 2; ++i) {
-      const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][g1_t]);
-      const float4 s = *reinterpret_cast<const float4*>(&sm.s[i][g1_j]);
-      const float wv[4] = {w.x, w.y, w.z, w.w}, sv[4] = {s.x, s.y, s.z, s.w};
+      for (int i = i_lo; i < i_lo + kK / 4; ++i) {
+        const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][g1_t]);
+        const float4 sv4 = *reinterpret_cast<const float4*>(&sm.s[i][g1_j]);
+        const float wv[4] = {w.x, w.y, w.z, w.w}, sv[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(wv[a], sv[bb], acc[a][bb]);
+      }
 #pragma unroll
       for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(wv[a], sv[bb], acc[a][bb]);
-    }
-    if (g1_h == 1) {
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-        *reinterpret_cast<float4*>(&sm.u[g1_t + a][g1_j]) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        *reinterpret_cast<float4*>(&sm.part[g1_q][g1_t + a][g1_j]) =
+            make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
     }
     __syncthreads();
-    if (g1_h == 0) {
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const float4 o = *reinterpret_cast<const float4*>(&sm.u[g1_t + a][g1_j]);
-        const float4 ut = *reinterpret_cast<const float4*>(&b.ut[g1_t + a][g1_j]);
-        const float4 u = make_float4(ut.x - (acc[a][0] + o.x), ut.y - (acc[a][1] + o.y),
-                                     ut.z - (acc[a][2] + o.z), ut.w - (acc[a][3] + o.w));
-        *reinterpret_cast<float4*>(&sm.u[g1_t + a][g1_j]) = u;
-        *reinterpret_cast<float4*>(rec + Workspace::kU + (g1_t + a) * kV + col0 + g1_j) = u;
-      }
+    {  // U = Ut - (W S), quarters summed in a fixed order
+      const float4 p0 = *reinterpret_cast<const float4*>(&sm.part[0][u_t][u_j]);
+      const float4 p1 = *reinterpret_cast<const float4*>(&sm.part[1][u_t][u_j]);
+      const float4 p2 = *reinterpret_cast<const float4*>(&sm.part[2][u_t][u_j]);
+      const float4 p3 = *reinterpret_cast<const float4*>(&sm.part[3][u_t][u_j]);
+      const float4 ut = *reinterpret_cast<const float4*>(&b.ut[u_t][u_j]);
+      const float4 u = make_float4(ut.x - ((p0.x + p1.x) + (p2.x + p3.x)), ut.y - ((p0.y + p1.y) + (p2.y + p3.y)),
+                                   ut.z - ((p0.z + p1.z) + (p2.z + p3.z)), ut.w - ((p0.w + p1.w) + (p2.w + p3.w)));
+      __syncthreads();  // every thread has read its partials before part[0] is overwritten
+      *reinterpret_cast<float4*>(&sm.part[0][u_t][u_j]) = u;
+      *reinterpret_cast<float4*>(rec + Workspace::kU + u_t * kV + col0 + u_j) = u;
     }
     __syncthreads();
 
     // GEMM 2: S = D S + Kh^T U
-    float sn[4][4];
+    float sn[2][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
+    for (int a = 0; a < 2; ++a) {
       const float d = b.dc[g2_i + a];
-      const float4 s = *reinterpret_cast<const float4*>(&sm.s[g2_i + a][g2_j]);
-      sn[a][0] = d * s.x; sn[a][1] = d * s.y; sn[a][2] = d * s.z; sn[a][3] = d * s.w;
+      const float4 sv4 = *reinterpret_cast<const float4*>(&sm.s[g2_i + a][g2_j]);
+      sn[a][0] = d * sv4.x; sn[a][1] = d * sv4.y; sn[a][2] = d * sv4.z; sn[a][3] = d * sv4.w;
     }
 #pragma unroll 8
     for (int t = 0; t < kC; ++t) {
-      const float4 kh = *reinterpret_cast<const float4*>(&b.kh[t][g2_i]);
-      const float4 u = *reinterpret_cast<const float4*>(&sm.u[t][g2_j]);
-      const float kv[4] = {kh.x, kh.y, kh.z, kh.w}, uv[4] = {u.x, u.y, u.z, u.w};
+      const float2 kh = *reinterpret_cast<const float2*>(&b.kh[t][g2_i]);
+      const float4 u = *reinterpret_cast<const float4*>(&sm.part[0][t][g2_j]);
+      const float kv[2] = {kh.x, kh.y}, uv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 2; ++a)
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) sn[a][bb] = fmaf(kv[a], uv[bb], sn[a][bb]);
     }
     __syncthreads();  // every thread is done reading s and the buffer
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 2; ++a)
       *reinterpret_cast<float4*>(&sm.s[g2_i + a][g2_j]) = make_float4(sn[a][0], sn[a][1], sn[a][2], sn[a][3]);
   }
   __syncthreads();

@@ -106,9 +106,9 @@ def test_rejections(lib, gated):
     assert call(lib, N=-1, gated=gated) == E.KDA_ERR_INVALID_ARG
     assert call(lib, T=-2, gated=gated) == E.KDA_ERR_INVALID_ARG
     assert call(lib, HV=0, gated=gated) == E.KDA_ERR_UNSUPPORTED
-    assert call(lib, K=96, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, K=0, gated=gated) == E.KDA_ERR_UNSUPPORTED
+    assert call(lib, K=257, gated=gated) == E.KDA_ERR_UNSUPPORTED
     assert call(lib, K=512, gated=gated) == E.KDA_ERR_UNSUPPORTED
-    assert call(lib, V=100, gated=gated) == E.KDA_ERR_UNSUPPORTED
     assert call(lib, V=0, gated=gated) == E.KDA_ERR_UNSUPPORTED
     assert call(lib, q=0, gated=gated) == E.KDA_ERR_INVALID_ARG
     assert call(lib, slot=0, gated=gated) == E.KDA_ERR_INVALID_ARG
@@ -134,6 +134,23 @@ def test_rejections(lib, gated):
 def test_valid_call_without_a_device_reports_device_error(lib):
     assert call(lib) == kda.KDA_ERR_DEVICE
     assert call(lib, gated=True) == kda.KDA_ERR_DEVICE
+
+
+@no_gpu
+@pytest.mark.parametrize("gated", [False, True])
+def test_general_shapes_pass_validation(lib, gated):
+    """K outside {64, 128, 256} and V not a multiple of 32 take the general
+    (masked, element-wise) form: valid, with element alignment only."""
+    E = kda
+    for K, V in [(96, 100), (192, 130), (1, 1), (256, 33), (48, 128), (128, 17)]:
+        assert call(lib, K=K, V=V, gated=gated) == E.KDA_ERR_DEVICE, (K, V)
+    # element alignment suffices for the general form, not for the vectorised one
+    assert call(lib, K=96, V=100, q=BASE + 2, gated=gated) == E.KDA_ERR_DEVICE
+    assert call(lib, K=96, V=100, q=BASE + 1, gated=gated) == E.KDA_ERR_MISALIGNED
+    assert call(lib, K=96, V=100, g=BASE + 3 * (1 << 30) + 2, gated=gated) == E.KDA_ERR_MISALIGNED
+    assert call(lib, K=128, V=128, q=BASE + 2, gated=gated) == E.KDA_ERR_MISALIGNED
+    if gated:
+        assert call(lib, K=96, V=257, gated=True) == E.KDA_ERR_UNSUPPORTED  # 9 tiles > one cluster
 
 
 def test_binding_refuses_cpu_tensors():
@@ -213,6 +230,11 @@ def test_ex_entry_point_validation(lib):
     assert args(g=BASE + 5 * step + 3 * block) == E.KDA_ERR_DEVICE            # slot 3: unseen unchecked
     assert args(g=BASE + 5 * step + 3 * block, num_slots=4) == E.KDA_ERR_ALIAS
     assert args(g=BASE + 5 * step + 4 * block, num_slots=4) == E.KDA_ERR_DEVICE  # just past the pool
+    # the general form takes [K][V] blocks and activated g, beta only
+    assert args(V=100, v_row_stride=2 * 100) == E.KDA_ERR_DEVICE
+    assert args(V=100, v_row_stride=2 * 100 + 3) == E.KDA_ERR_DEVICE  # any row stride
+    assert args(V=100, v_row_stride=200, state_layout=kda.KDA_LAYOUT_VK) == E.KDA_ERR_UNSUPPORTED
+    assert args(K=96, q_row_stride=192, k_row_stride=192, g_row_stride=192, **raw) == E.KDA_ERR_UNSUPPORTED
 
 
 @no_gpu

@@ -654,3 +654,50 @@ def test_checked_slots_equal_unchecked_when_in_range(cuda_device):
     o2 = kda.kda_decode_ex(d2.q, d2.k, d2.v, d2.state, d2.slot_idx, g=d2.g, beta=d2.beta, num_slots=12)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(d1.state, d2.state)
+
+
+# ---------------------------------------------------------------------------
+# general K and V (masked, element-wise form)
+# ---------------------------------------------------------------------------
+GENERAL_CASES = [
+    (3, 1, 2, 96, 100, False, "fp32", 1),
+    (3, 1, 2, 192, 130, True, "fp32", 1),
+    (2, 5, 2, 96, 130, False, "fp32", 0),
+    (3, 7, 3, 192, 100, True, "bf16", 1),
+    (2, 1, 2, 48, 17, False, "bf16", 0),
+    (3, 6, 1, 200, 33, True, "fp32", 1),
+    (3, 3, 2, 128, 100, False, "fp32", 1),   # K of the vectorised set, V ragged
+    (2, 1, 2, 80, 128, True, "fp32", 0),     # V of the vectorised set, K ragged
+    (2, 9, 2, 1, 1, False, "fp32", 0),       # one key channel, one value column
+    (2, 13, 2, 256, 250, True, "bf16", 1),   # eight value tiles, the last ragged
+]
+
+
+@pytest.mark.parametrize("N,T,HV,K,V,gated,state,inactive", GENERAL_CASES)
+def test_general_shapes_parity(N, T, HV, K, V, gated, state, inactive, cuda_device):
+    """K outside {64, 128, 256} (rows padded, masked) and V not a multiple of 32
+    (last value tile masked), through the fixed entry points, against the oracle;
+    padding rows included."""
+    w = workloads.make(N=N, T=T, HV=HV, K=K, V=V, num_slots=N + 2, gated=gated, seed=400 + K + V + T,
+                       state_dtype=state, inactive=inactive)
+    o, pool, before = run_gpu(w, cuda_device)
+    assert_parity(w, o, pool, before)
+
+
+@pytest.mark.parametrize("T,gated", [(1, False), (1, True), (6, False), (5, True)])
+def test_general_shapes_strided_rows(T, gated, cuda_device):
+    """The general form with q, k, v as slices of one packed row buffer whose
+    row stride is odd (rows of no particular alignment), bit-identical to the
+    dense call."""
+    w = workloads.make(N=3, T=T, HV=2, K=96, V=100, num_slots=5, gated=gated, seed=450 + T, inactive=1)
+    d1, d2 = w.to(cuda_device), w.to(cuda_device)
+    _, (q, k, v) = workloads.pack_rows([d2.q, d2.k, d2.v], pad=3)
+    assert q.stride(1) % 2 == 1
+    extra1 = dict(gate=d1.gate, norm_weight=d1.norm_weight, eps=w.eps) if gated else {}
+    extra2 = dict(gate=d2.gate, norm_weight=d2.norm_weight, eps=w.eps) if gated else {}
+    o1 = kda.kda_decode_ex(d1.q, d1.k, d1.v, d1.state, d1.slot_idx, g=d1.g, beta=d1.beta, **extra1)
+    o2 = kda.kda_decode_ex(q, k, v, d2.state, d2.slot_idx, g=d2.g, beta=d2.beta, **extra2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(d1.state, d2.state)
+    before = w.to(cuda_device).state
+    assert_parity(w, o2, d2.state, before)
