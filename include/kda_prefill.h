@@ -14,8 +14,9 @@
  * the decode step up to fp32 rounding; what differs is how it is computed: the
  * tokens are taken in chunks of 64 in the WY / UT chunk form (a triangular
  * solve inside each chunk, a short state recurrence across chunks and the
- * chunk outputs as dense products), which turns the work of a long run into
- * parallel per-chunk products instead of a token-by-token chain.
+ * chunk outputs as dense products on the tensor cores), which turns the work
+ * of a long run into parallel per-chunk products instead of a token-by-token
+ * chain.
  *
  * Source: vLLM #57585 "Tune recurrent KDA launch configuration on SM90",
  * Details: the related work it names (FlashInfer's fused KDA on Blackwell)
@@ -36,9 +37,14 @@
  * kda_prefill_workspace_bytes(N, T, HV, K, V) bytes (16-byte aligned); the
  * library allocates nothing.  Per (sequence, head, chunk of 64 tokens) it holds
  * about 240 KB of fp32 intermediates (the chunk's solve results, decayed keys
- * and queries, its start state and corrections).  Its contents are not
- * meaningful between calls; calls that share a workspace must not overlap on
- * the device (stream order is enough).
+ * and queries, its start state and corrections), after a 256-byte header.
+ * Its contents are not meaningful between calls; calls that share a workspace
+ * must not overlap on the device (stream order is enough).  The header's first
+ * int32 is an error word: the output kernel waits for its tensor-core results
+ * with a bounded poll, and if that wait ever gives up (it takes seconds; the
+ * products take microseconds) it leaves that chunk's outputs unwritten and
+ * stores 1 there.  The library never clears it: a caller that wants to watch
+ * it zeroes it before the call.
  *
  * Execution: three kernels enqueued on `stream` in order (chunk preparation,
  * the state recurrence across chunks, the chunk outputs); no host sync; can be

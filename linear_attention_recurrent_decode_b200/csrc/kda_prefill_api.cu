@@ -19,7 +19,8 @@ namespace kp = kdap;
 bool workspace_floats(int64_t N, int64_t T, int64_t HV, int64_t* nchunks, int64_t* floats) {
   *nchunks = (T + kp::kC - 1) / kp::kC;
   int64_t units;
-  return mul_ok(N, HV, &units) && mul_ok(units, *nchunks, floats) && mul_ok(*floats, kp::Workspace::kFloats, floats);
+  return mul_ok(N, HV, &units) && mul_ok(units, *nchunks, floats) && mul_ok(*floats, kp::Workspace::kFloats, floats) &&
+         !__builtin_add_overflow(*floats, kp::Workspace::kHeaderFloats, floats);
 }
 
 // Once per device: the three kernels' dynamic shared memory allowances.

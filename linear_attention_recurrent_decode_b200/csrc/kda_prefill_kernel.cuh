@@ -32,7 +32,7 @@
 //      keeping S in shared memory; writes each chunk's start state and U to the
 //      workspace and the final state back to the pool slot.
 //   3. kda_prefill_output_kernel (one CTA per (n, h, chunk)): O = scale (Qt S0
-//      + P U), bf16 output.
+//      + P U) on the tensor cores (tcgen05), bf16 output.
 //
 // Numerics.  exp(Gamma_t - Gamma_s) is never formed by dividing decays: the
 // chunk kernel factors it as exp(Gamma_t - Gamma_r) exp(Gamma_r - Gamma_s)
@@ -43,7 +43,8 @@
 // path that forms every pair's exponential directly.  Gamma is summed in fp64
 // and each exponential is taken from the fp64 difference, so the long-range
 // decays keep fp32 accuracy (a cumulative sum in fp32 would lose up to
-// 64 ulp of |Gamma|).  All other arithmetic is fp32.
+// 64 ulp of |Gamma|).  All other arithmetic is fp32, except the output
+// products, whose bf16-pair operands carry 16 significant bits (see kernel 3).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -74,19 +75,21 @@ struct Params {
   float scale;
 };
 
-// Workspace layout: one record per (n, h, chunk), fp32.
+// Workspace layout: a 256-byte header (word 0: the error word, see
+// wait_bounded), then one fp32 record per (n, h, chunk).
 struct Workspace {
+  static constexpr int64_t kHeaderFloats = 64;
   static constexpr int64_t kWt = 0;                   // W^T  [K][C]
   static constexpr int64_t kKh = kWt + kK * kC;       // Kh   [C][K]
   static constexpr int64_t kUt = kKh + kC * kK;       // Ut   [C][V]   (the V part of the solve)
-  static constexpr int64_t kQt = kUt + kC * kV;       // Qt^T [K][C]
-  static constexpr int64_t kPt = kQt + kK * kC;       // P^T  [C][C]   (Pt[s][t] = P[t][s], zero for s > t)
-  static constexpr int64_t kDc = kPt + kC * kC;       // exp(Gamma_C) [K]
+  static constexpr int64_t kQ = kUt + kC * kV;        // Qt   [C][K]   (decayed queries)
+  static constexpr int64_t kP = kQ + kC * kK;         // P    [C][C]   (zero for s > t)
+  static constexpr int64_t kDc = kP + kC * kC;        // exp(Gamma_C) [K]
   static constexpr int64_t kS0 = kDc + kK;            // chunk-start state [K][V]
   static constexpr int64_t kU = kS0 + kK * kV;        // U [C][V]
   static constexpr int64_t kFloats = kU + kC * kV;    // per record
   static __host__ __device__ int64_t record(int64_t unit, int64_t chunk, int32_t nchunks) {
-    return (unit * nchunks + chunk) * kFloats;
+    return kHeaderFloats + (unit * nchunks + chunk) * kFloats;
   }
 };
 
@@ -206,15 +209,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
     sm.kt[t][i] = kv * exp_of(gt);                                   // k exp(Gamma_t)
     rec[Workspace::kKh + t * kK + i] = kv * exp_of(sm.gam[kC - 1][i] - gt);  // k exp(Gamma_C - Gamma_t)
   }
-  for (int e = tid; e < kC * kK; e += kChunkThreads) {  // [i][t] order for the transposed store
-    const int i = e / kC, t = e % kC;
-    rec[Workspace::kQt + i * kC + t] = __bfloat162float(raw.q[t][i]) * exp_of(sm.gam[t][i]);
+  for (int e = tid; e < kC * kK; e += kChunkThreads) {
+    const int t = e / kK, i = e % kK;
+    rec[Workspace::kQ + t * kK + i] = __bfloat162float(raw.q[t][i]) * exp_of(sm.gam[t][i]);  // q exp(Gamma_t)
   }
   if (tid < kK) rec[Workspace::kDc + tid] = exp_of(gam_end);
   __syncthreads();  // raw q/k still needed below; kt complete
 
   // ---- 3. M and P
-  float* const Pt = rec + Workspace::kPt;  // Pt[s][t] = P[t][s]
+  float* const Pm = rec + Workspace::kP;  // P[t][s]
   if (!exact) {
     // The factors go through registers: the raw inputs they are made from live
     // in the buffers they are written to.
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       for (int b = 0; b < 4; ++b) {
         const int s = sb * 4 + b;
         sm.L[t][s] = (s < t) ? sm.beta[t] * m[a][b] : 0.f;
-        Pt[s * kC + t] = (s <= t) ? pp[a][b] : 0.f;
+        Pm[t * kC + s] = (s <= t) ? pp[a][b] : 0.f;
       }
     }
   } else {
@@ -290,7 +293,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
         }
       }
       sm.L[t][s] = (s < t) ? sm.beta[t] * mv : 0.f;
-      Pt[s * kC + t] = (s <= t) ? pv : 0.f;
+      Pm[t * kC + s] = (s <= t) ? pv : 0.f;
     }
     __syncthreads();
     float* const vf = reinterpret_cast<float*>(&sm.gam[0][0]);
@@ -488,85 +491,246 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
 }
 
 // ---------------------------------------------------------------- kernel 3
+// The chunk outputs on the tensor cores (tcgen05, kind::f16), transposed so
+// that the value index is the MMA's M = 128:
+//   O^T [V x C] = S0^T [V x K] . Qt^T [K x C]  +  U^T [V x C] . P^T [C x C].
+// fp32 operands are split into bf16 pairs x = hi + lo (hi = bf16(x),
+// lo = bf16(x - hi): 16 significant bits), and each product takes three MMAs
+// (hi.hi + hi.lo + lo.hi; the dropped lo.lo term is 2^-18 relative), so the
+// fp32 accumulation in tensor memory is accurate to about 2^-16 -- well inside
+// the bf16 output rounding.  Operand tiles sit in shared memory in the
+// canonical K-major layout without swizzle: 8-row x 16-byte core matrices, the
+// two core matrices of one 16-element K step 128 bytes apart (the leading byte
+// offset) and consecutive 8-row groups (K/8) * 128 bytes apart (the stride
+// byte offset).  One thread issues the 36 MMAs and commits them to an
+// mbarrier; every thread then reads its value column's 64 outputs back from
+// tensor memory (tcgen05.ld, lane = value column).
+namespace tc {
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  // start address, leading and stride byte offsets in 16-byte units; the
+  // SM100 descriptor version (1) at bit 46; no swizzle, base offset 0
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void commit(uint64_t* mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(mbar))
+               : "memory");
+}
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(mbar)), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Wait for phase `parity` of the mbarrier, giving up after `limit` polls
+// (returns false then): the kernels never wait without bound.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* mbar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_addr(mbar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// 16 consecutive fp32 columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Offset, in bytes, of element (row r, k) of a K-major bf16 tile with kd
+// elements along K (canonical layout, no swizzle).
+__host__ __device__ constexpr uint32_t kmajor_off(int r, int k, int kd) {
+  return static_cast<uint32_t>((r / 8) * (kd / 8) * 128 + (k / 8) * 128 + (r % 8) * 16 + (k % 8) * 2);
+}
+// The hi and lo bf16 halves of eight fp32 values, packed for one 16-byte store each.
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+    h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[i] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+}  // namespace tc
+
 constexpr int kOutThreads = 256;
+constexpr uint32_t kOutTmemCols = 64;  // the fp32 accumulator, 128 lanes x C columns
 
 struct OutSmem {
-  float qt[kK][kC];   // Qt^T
-  float s0[kK][kV];   // chunk-start state
-  float pt[kC][kC];   // P^T
-  float u[kC][kV];    // U
+  alignas(1024) unsigned char a1h[kV * kK * 2];  // S0^T  [V rows][K]  bf16 hi
+  alignas(1024) unsigned char a1l[kV * kK * 2];  //                      lo
+  alignas(1024) unsigned char b1h[kC * kK * 2];  // Qt    [C rows][K]
+  alignas(1024) unsigned char b1l[kC * kK * 2];
+  alignas(1024) unsigned char a2h[kV * kC * 2];  // U^T   [V rows][C]
+  alignas(1024) unsigned char a2l[kV * kC * 2];
+  alignas(1024) unsigned char b2h[kC * kC * 2];  // P     [C rows][C]
+  alignas(1024) unsigned char b2l[kC * kC * 2];
+  uint64_t mbar;
+  uint32_t tmem;
 };
 
 __global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(const Params p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int64_t unit = blockIdx.x / p.nchunks;
   const int32_t chunk = static_cast<int32_t>(blockIdx.x - unit * p.nchunks);
   const int64_t n = unit / p.HV;
   const int64_t h = unit - n * p.HV;
   const int64_t t0 = static_cast<int64_t>(chunk) * kC;
   const int tc = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
-  // thread tile: 4 tokens x 8 columns
-  const int ot = (tid % 16) * 4;
-  const int oj = (tid / 16) * 8;
+  // epilogue: value column j = 32 (warp % 4) + lane, tokens of half (warp / 4)
+  const int j = 32 * (warp % 4) + lane;
+  const int half = warp / 4;
   if (__ldg(p.slot_idx + n) < 0) {  // inactive row: zero output
-    for (int a = 0; a < 4; ++a) {
-      if (ot + a < tc) {
-        __nv_bfloat16* o = p.out + ((n * p.T + t0 + ot + a) * p.HV + h) * kV + oj;
-        *reinterpret_cast<uint4*>(o) = make_uint4(0, 0, 0, 0);
-      }
-    }
+    for (int t = half * 32; t < half * 32 + 32 && t < tc; ++t)
+      p.out[((n * p.T + t0 + t) * p.HV + h) * kV + j] = __float2bfloat16(0.f);
     return;
   }
-  const float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
-  for (int c = tid; c < (kK * kC) / 4; c += kOutThreads) cp_async16(&sm.qt[0][0] + 4 * c, rec + Workspace::kQt + 4 * c);
-  for (int c = tid; c < (kK * kV) / 4; c += kOutThreads) cp_async16(&sm.s0[0][0] + 4 * c, rec + Workspace::kS0 + 4 * c);
-  for (int c = tid; c < (kC * kC) / 4; c += kOutThreads) cp_async16(&sm.pt[0][0] + 4 * c, rec + Workspace::kPt + 4 * c);
-  for (int c = tid; c < (kC * kV) / 4; c += kOutThreads) cp_async16(&sm.u[0][0] + 4 * c, rec + Workspace::kU + 4 * c);
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
+  if (warp == 0) tc::tmem_alloc(&sm.tmem, kOutTmemCols);
+  if (tid == 0) tc::mbar_init(&sm.mbar, 1);
 
-  float acc[4][8];
+  // ---- operand tiles: fp32 from the workspace, split to bf16 hi/lo
+  const float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
+  // A1 = S0^T: item (value row j, key group of 8); loads are coalesced over j
+  for (int e = tid; e < kV * (kK / 8); e += kOutThreads) {
+    const int jj = e % kV, ig = e / kV;
+    float x[8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < kK; ++i) {
-    const float4 q = *reinterpret_cast<const float4*>(&sm.qt[i][ot]);
-    const float4 s0 = *reinterpret_cast<const float4*>(&sm.s0[i][oj]);
-    const float4 s1 = *reinterpret_cast<const float4*>(&sm.s0[i][oj + 4]);
-    const float qv[4] = {q.x, q.y, q.z, q.w}, sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(qv[a], sv[b], acc[a][b]);
+    for (int r = 0; r < 8; ++r) x[r] = rec[Workspace::kS0 + (ig * 8 + r) * kV + jj];
+    uint4 hi, lo;
+    tc::split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(sm.a1h + tc::kmajor_off(jj, ig * 8, kK)) = hi;
+    *reinterpret_cast<uint4*>(sm.a1l + tc::kmajor_off(jj, ig * 8, kK)) = lo;
   }
-  const int s_end = ot + 4;  // P[t][s] = 0 for s > t
-  for (int s = 0; s < s_end; ++s) {
-    const float4 pq = *reinterpret_cast<const float4*>(&sm.pt[s][ot]);
-    const float4 u0 = *reinterpret_cast<const float4*>(&sm.u[s][oj]);
-    const float4 u1 = *reinterpret_cast<const float4*>(&sm.u[s][oj + 4]);
-    const float pv[4] = {pq.x, pq.y, pq.z, pq.w}, uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(pv[a], uv[b], acc[a][b]);
+  // B1 = Qt: item (token row t, key group of 8): one 32-byte read
+  for (int e = tid; e < kC * (kK / 8); e += kOutThreads) {
+    const int t = e / (kK / 8), ig = e % (kK / 8);
+    const float4 u0 = *reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8);
+    const float4 u1 = *reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8 + 4);
+    const float x[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    uint4 hi, lo;
+    tc::split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(sm.b1h + tc::kmajor_off(t, ig * 8, kK)) = hi;
+    *reinterpret_cast<uint4*>(sm.b1l + tc::kmajor_off(t, ig * 8, kK)) = lo;
   }
+  // A2 = U^T: item (value row j, token group of 8); loads coalesced over j
+  for (int e = tid; e < kV * (kC / 8); e += kOutThreads) {
+    const int jj = e % kV, sg = e / kV;
+    float x[8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    if (ot + a >= tc) continue;
-    uint32_t w[4];
+    for (int r = 0; r < 8; ++r) x[r] = rec[Workspace::kU + (sg * 8 + r) * kV + jj];
+    uint4 hi, lo;
+    tc::split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(sm.a2h + tc::kmajor_off(jj, sg * 8, kC)) = hi;
+    *reinterpret_cast<uint4*>(sm.a2l + tc::kmajor_off(jj, sg * 8, kC)) = lo;
+  }
+  // B2 = P: item (token row t, token group of 8)
+  for (int e = tid; e < kC * (kC / 8); e += kOutThreads) {
+    const int t = e / (kC / 8), sg = e % (kC / 8);
+    const float4 u0 = *reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8);
+    const float4 u1 = *reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8 + 4);
+    const float x[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    uint4 hi, lo;
+    tc::split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(sm.b2h + tc::kmajor_off(t, sg * 8, kC)) = hi;
+    *reinterpret_cast<uint4*>(sm.b2l + tc::kmajor_off(t, sg * 8, kC)) = lo;
+  }
+  tc::fence_proxy_async();  // the tiles, written by threads, are read by the tensor cores
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm.tmem;
+
+  if (tid == 0) {
+    constexpr uint32_t idesc = tc::idesc_bf16(128, kC);
+    const uint32_t a1h = smem_addr(sm.a1h), a1l = smem_addr(sm.a1l), b1h = smem_addr(sm.b1h),
+                   b1l = smem_addr(sm.b1l), a2h = smem_addr(sm.a2h), a2l = smem_addr(sm.a2l),
+                   b2h = smem_addr(sm.b2h), b2l = smem_addr(sm.b2l);
+    constexpr uint32_t kLbo = 128;
+    constexpr uint32_t kSbo1 = (kK / 8) * 128;  // K = 128 along the K dimension
+    constexpr uint32_t kSbo2 = (kC / 8) * 128;  // K = 64
+    uint32_t acc = 0;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      __nv_bfloat162 x = __floats2bfloat162_rn(p.scale * acc[a][2 * b], p.scale * acc[a][2 * b + 1]);
-      w[b] = *reinterpret_cast<uint32_t*>(&x);
+    for (int st = 0; st < kK / 16; ++st) {
+      const uint32_t off = st * 256;  // two core matrices per 16-element K step
+      tc::mma_bf16(tmem, tc::smem_desc(a1h + off, kLbo, kSbo1), tc::smem_desc(b1h + off, kLbo, kSbo1), idesc, acc);
+      acc = 1;
+      tc::mma_bf16(tmem, tc::smem_desc(a1h + off, kLbo, kSbo1), tc::smem_desc(b1l + off, kLbo, kSbo1), idesc, 1);
+      tc::mma_bf16(tmem, tc::smem_desc(a1l + off, kLbo, kSbo1), tc::smem_desc(b1h + off, kLbo, kSbo1), idesc, 1);
     }
-    __nv_bfloat16* o = p.out + ((n * p.T + t0 + ot + a) * p.HV + h) * kV + oj;
-    *reinterpret_cast<uint4*>(o) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+    for (int st = 0; st < kC / 16; ++st) {
+      const uint32_t off = st * 256;
+      tc::mma_bf16(tmem, tc::smem_desc(a2h + off, kLbo, kSbo2), tc::smem_desc(b2h + off, kLbo, kSbo2), idesc, 1);
+      tc::mma_bf16(tmem, tc::smem_desc(a2h + off, kLbo, kSbo2), tc::smem_desc(b2l + off, kLbo, kSbo2), idesc, 1);
+      tc::mma_bf16(tmem, tc::smem_desc(a2l + off, kLbo, kSbo2), tc::smem_desc(b2h + off, kLbo, kSbo2), idesc, 1);
+    }
+    tc::commit(&sm.mbar);
   }
+  // about 2^26 polls: seconds, against microseconds for the MMAs
+  const bool ok = tc::mbar_wait_bounded(&sm.mbar, 0, 1u << 26);
+  tc::fence_after_sync();
+  if (ok) {
+    // lane j of this warp's 32-lane slice; columns (tokens) of this warp's half
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp % 4)) << 16) + static_cast<uint32_t>(half * 32);
+    float o[32];
+    tc::tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&o[0]));
+    tc::tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&o[16]));
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int t = half * 32 + c;
+      if (t < tc) p.out[((n * p.T + t0 + t) * p.HV + h) * kV + j] = __float2bfloat16_rn(p.scale * o[c]);
+    }
+  } else if (tid == 0) {
+    atomicExch(reinterpret_cast<int*>(p.ws), 1);  // the workspace header's error word
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, kOutTmemCols);
 }
 
 constexpr int kChunkSmem = static_cast<int>(sizeof(ChunkSmem));

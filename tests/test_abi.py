@@ -273,7 +273,7 @@ def test_prefill_validation(lib):
     step = 1 << 30
     N, T, HV = 2, 100, 2
     need = lib.kda_prefill_workspace_bytes(N, T, HV, 128, 128)
-    assert need == N * HV * 2 * 246272  # two chunks per (n, h) of 61,568 fp32 each
+    assert need == 256 + N * HV * 2 * 246272  # a header, then two chunks per (n, h) of 61,568 fp32 each
     assert lib.kda_prefill_workspace_bytes(N, T, HV, 128, 64) == -1
     assert lib.kda_prefill_workspace_bytes(-1, T, HV, 128, 128) == -1
     assert lib.kda_prefill_workspace_bytes(N, 0, HV, 128, 128) == 0

@@ -257,7 +257,7 @@ def test_rejections_with_real_buffers(cuda_device):
     assert call() == kda.KDA_ERR_ALIAS                             # out inside q
     assert call(out=d.state.data_ptr()) == kda.KDA_ERR_ALIAS       # out = pool
     assert call(out=out.data_ptr() + 2) == kda.KDA_ERR_MISALIGNED
-    assert call(out=out.data_ptr(), K=96) == kda.KDA_ERR_UNSUPPORTED
+    assert call(out=out.data_ptr(), K=300) == kda.KDA_ERR_UNSUPPORTED
     assert call(out=out.data_ptr(), q=d.q.data_ptr() + 8) == kda.KDA_ERR_MISALIGNED
     torch.cuda.synchronize()
     assert torch.equal(d.state, before)
@@ -692,7 +692,7 @@ def test_general_shapes_strided_rows(T, gated, cuda_device):
     w = workloads.make(N=3, T=T, HV=2, K=96, V=100, num_slots=5, gated=gated, seed=450 + T, inactive=1)
     d1, d2 = w.to(cuda_device), w.to(cuda_device)
     _, (q, k, v) = workloads.pack_rows([d2.q, d2.k, d2.v], pad=3)
-    assert q.stride(1) % 2 == 1
+    assert (q.stride(1) if T > 1 else q.stride(0)) % 2 == 1  # rows two bytes apart from alignment
     extra1 = dict(gate=d1.gate, norm_weight=d1.norm_weight, eps=w.eps) if gated else {}
     extra2 = dict(gate=d2.gate, norm_weight=d2.norm_weight, eps=w.eps) if gated else {}
     o1 = kda.kda_decode_ex(d1.q, d1.k, d1.v, d1.state, d1.slot_idx, g=d1.g, beta=d1.beta, **extra1)
