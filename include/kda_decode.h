@@ -99,7 +99,8 @@ typedef enum {
     KDA_ERR_ALIAS = 3,       /* out overlaps an input or the pool */
     KDA_ERR_MISALIGNED = 4,  /* a pointer breaks the alignment rule above */
     KDA_ERR_DEVICE = 5,      /* current device is not compute capability 10.0 */
-    KDA_ERR_CUDA = 6         /* the CUDA runtime refused the launch */
+    KDA_ERR_CUDA = 6,        /* the CUDA runtime refused the launch */
+    KDA_ERR_SCRATCH_LIMIT = 7 /* kda_prefill_no_alloc: the sizes need more than its fixed scratch */
 } kda_status;
 
 /*

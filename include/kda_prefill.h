@@ -80,6 +80,43 @@ KDA_API kda_status kda_prefill(const void *q, const void *k, const void *v, cons
                                int64_t T, int64_t HV, int64_t K, int64_t V, float scale,
                                kda_stream_t stream);
 
+/*
+ * The same chunked prefill for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it is this library's own.
+ *
+ * Some callers of an attention library may not call cudaMalloc at all: an
+ * inference server that hands nearly all of the GPU's memory to its own
+ * caching allocator at start-up (a later cudaMalloc then fails or fragments
+ * that pool), a framework plugin whose host forbids allocations outside the
+ * framework's allocator, or a runtime that records its work into CUDA graphs
+ * and has no allocation step between captures.  kda_prefill needs a workspace
+ * those callers cannot provide; this entry point takes none.  Instead it uses
+ * a fixed scratch array of KDA_PREFILL_NO_ALLOC_SCRATCH_BYTES (32 MiB) that
+ * the library declares in device memory: every GPU that loads the library
+ * holds those 32 MiB until the process exits, whether or not it calls this.
+ *
+ * Arguments, layouts, results and errors are those of kda_prefill without the
+ * workspace.  Sizes whose workspace (kda_prefill_workspace_bytes) exceeds the
+ * scratch return KDA_ERR_SCRATCH_LIMIT before anything is enqueued: with
+ * K = V = 128 that is N * HV * ceil(T / 64) <= 136 chunks (for example one
+ * sequence of up to 1088 tokens at HV = 8).
+ *
+ * The first call on each device looks the scratch array's device address up
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ * first call before capturing any stream into a CUDA graph.  Every call on a
+ * device uses the same array, and the array keeps whatever the last call left
+ * in it (nothing in it needs to start at zero: each call writes every part it
+ * reads), so two calls whose kernels overlap on the GPU -- on different
+ * streams without an ordering between them -- race on it and give wrong
+ * results.  Calls in one stream, or otherwise ordered, are safe.
+ */
+#define KDA_PREFILL_NO_ALLOC_SCRATCH_BYTES (32LL << 20)
+
+KDA_API kda_status kda_prefill_no_alloc(const void *q, const void *k, const void *v, const float *g,
+                                        const float *beta, float *state_pool, const int32_t *slot_idx,
+                                        void *out, int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
+                                        float scale, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,7 +27,8 @@ import torch
 __all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "kda_prefill",
            "prefill_workspace_bytes", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
-           "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_STATE_FP32", "KDA_STATE_BF16",
+           "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_ERR_SCRATCH_LIMIT", "KDA_STATE_FP32",
+           "KDA_STATE_BF16",
            "KDA_LAYOUT_KV", "KDA_LAYOUT_VK", "LIBRARY_PATH", "EXPORTED_SYMBOLS"]
 
 LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda_decode.so")
@@ -39,6 +40,7 @@ KDA_ERR_ALIAS = 3
 KDA_ERR_MISALIGNED = 4
 KDA_ERR_DEVICE = 5
 KDA_ERR_CUDA = 6
+KDA_ERR_SCRATCH_LIMIT = 7
 
 _P, _I, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
 
@@ -82,6 +84,7 @@ EXPORTED_SYMBOLS = {
     # include/kda_prefill.h
     "kda_prefill_workspace_bytes": ([_I] * 5, ctypes.c_int64),
     "kda_prefill": ([_P] * 9 + [_I] * 6 + [_F, _P], ctypes.c_int),
+    "kda_prefill_no_alloc": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
 }
 
 _lock = threading.Lock()

@@ -344,10 +344,12 @@ const char* kda_status_string(kda_status status) {
     case KDA_ERR_MISALIGNED: return "misaligned pointer or row stride";
     case KDA_ERR_DEVICE: return "current device is not compute capability 10.0 (sm_100a)";
     case KDA_ERR_CUDA: return "CUDA launch failed";
+    case KDA_ERR_SCRATCH_LIMIT:
+      return "sizes need more scratch than kda_prefill_no_alloc's fixed array holds (use kda_prefill)";
   }
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 5; }
+int32_t kda_abi_version(void) { return (1 << 16) | 6; }
 
 }  // extern "C"

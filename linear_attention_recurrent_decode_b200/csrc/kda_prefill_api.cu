@@ -125,3 +125,49 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- kda_prefill_no_alloc
+// Scratch for callers that cannot allocate (see include/kda_prefill.h): a
+// file-scope device array, 256-byte aligned like a cudaMalloc block.  In host
+// code its name stands for the variable, not for a device address: the
+// address comes from cudaGetSymbolAddress, once per device, below.
+static __device__ __align__(256) unsigned char g_prefill_scratch[KDA_PREFILL_NO_ALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::atomic<void*> g_scratch_addr[kMaxDevices];  // per device, found on its first call
+
+// The scratch array's address on the current device (nullptr if the lookup fails).
+void* scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  if (dev < kMaxDevices) {
+    void* known = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (known != nullptr) return known;
+  }
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_prefill_scratch) != cudaSuccess) return nullptr;
+  if (dev < kMaxDevices) g_scratch_addr[dev].store(addr, std::memory_order_release);
+  return addr;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_prefill_no_alloc(const void* q, const void* k, const void* v, const float* g,
+                                           const float* beta, float* state_pool, const int32_t* slot_idx,
+                                           void* out, int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
+                                           float scale, kda_stream_t stream) {
+  const int64_t need = kda_prefill_workspace_bytes(N, T, HV, K, V);
+  if (need < 0) {  // the sizes kda_prefill would refuse: let it give the reason
+    return kda_prefill(q, k, v, g, beta, state_pool, slot_idx, out, nullptr, 0, N, T, HV, K, V, scale, stream);
+  }
+  if (need > KDA_PREFILL_NO_ALLOC_SCRATCH_BYTES) return KDA_ERR_SCRATCH_LIMIT;
+  if (N == 0 || T == 0 || HV == 0)  // nothing to do; no pointer (and no scratch) is touched
+    return kda_prefill(q, k, v, g, beta, state_pool, slot_idx, out, nullptr, 0, N, T, HV, K, V, scale, stream);
+  const kda_status dev = check_device();
+  if (dev != KDA_OK) return dev;
+  void* const scratch = scratch_on_current_device();
+  if (scratch == nullptr) return KDA_ERR_CUDA;
+  return kda_prefill(q, k, v, g, beta, state_pool, slot_idx, out, scratch, KDA_PREFILL_NO_ALLOC_SCRATCH_BYTES, N, T,
+                     HV, K, V, scale, stream);
+}

@@ -45,7 +45,7 @@ def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
                                     "kda_decode_host", "kda_status_string", "kda_abi_version",
-                                    "kda_prefill", "kda_prefill_workspace_bytes"}
+                                    "kda_prefill", "kda_prefill_workspace_bytes", "kda_prefill_no_alloc"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -62,10 +62,10 @@ def test_library_exports_nothing_else(lib):
 
 def test_status_strings_and_version(lib):
     assert kda.status_string(kda.KDA_OK) == "ok"
-    for s in range(1, 7):
+    for s in range(1, 8):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 5
+    assert lib.kda_abi_version() == (1 << 16) | 6
 
 
 # ----------------------------------------------------------------- validation
@@ -298,6 +298,28 @@ def test_prefill_validation(lib):
     assert call(ws=BASE + 9 * step + 64) == E.KDA_ERR_ALIAS   # workspace over out
     assert call(ws=BASE + 5 * step - 1024) == E.KDA_ERR_ALIAS # workspace runs into the pool
     assert call(g=BASE + 5 * step + 4096) == E.KDA_ERR_ALIAS  # an input inside slot 0
+
+
+@no_gpu
+def test_prefill_no_alloc_validation(lib):
+    """kda_prefill_no_alloc: sizes beyond its fixed scratch are refused before
+    any device work; other sizes are validated as kda_prefill validates them."""
+    E = kda
+    step = 1 << 30
+
+    def call(N=1, T=1000, HV=8, K=128, V=128, q=BASE):
+        return lib.kda_prefill_no_alloc(q, BASE + step, BASE + 2 * step, BASE + 3 * step, BASE + 4 * step,
+                                        BASE + 5 * step, BASE + 8 * step, BASE + 9 * step, N, T, HV, K, V, 0.1,
+                                        None)
+
+    assert call() == E.KDA_ERR_DEVICE                      # 128 chunks fit: valid, no device here
+    assert call(T=1088) == E.KDA_ERR_DEVICE                # 136 chunks: the most that fit
+    assert call(T=1089) == E.KDA_ERR_SCRATCH_LIMIT         # 144 chunks
+    assert call(N=2, T=8192) == E.KDA_ERR_SCRATCH_LIMIT
+    assert call(K=64) == E.KDA_ERR_UNSUPPORTED
+    assert call(T=-1) == E.KDA_ERR_INVALID_ARG
+    assert call(N=0, q=0) == E.KDA_OK
+    assert kda.status_string(E.KDA_ERR_SCRATCH_LIMIT).startswith("sizes need more scratch")
 
 
 @pytest.mark.gpu
