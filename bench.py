@@ -484,14 +484,10 @@ def copy_floor(w, dev, stream, R, steps, preroll_s):
             "bytes_per_call": 2 * n * 4, "gbs": round(2 * n * 4 / (us * 1e-6) / 1e9, 1)}
 
 
-def run_e2e(kda, w, dev, stream, steps, world):
-    """µs per call with each step's inputs copied from pinned host memory and its
-    output read back, through the public API (``HostStep``, the C ABI's
-    ``kda_decode_host``), eager launches.  A step's inputs live in one packed
-    pinned buffer (as a serving host would stage them), so each step is one
-    host-to-device copy, the decode kernel and one device-to-host copy of the
-    output, enqueued by one library call; the state pool stays resident on the
-    GPU."""
+def _host_step(kda, w, dev, stream, pool):
+    """One staging set: the step's inputs packed in one pinned host buffer (as a
+    serving host would stage them), its device copy, and a HostStep bound to
+    them and to ``pool``."""
     import torch
 
     inputs = {k: t for k, t in w.tensors().items() if k != "state"}
@@ -499,43 +495,94 @@ def run_e2e(kda, w, dev, stream, steps, world):
     for k, t in inputs.items():
         host[k].copy_(t)
     dev_buf, devv = _packed(inputs, lambda n: torch.empty(n, dtype=torch.uint8, device=dev))
-    pool = w.state.to(dev)
     out_d = torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=dev)
     out_h = torch.empty(out_d.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = host_buf.numel()  # the packed buffer each step copies (inputs and their 16-byte alignment)
-    d2h = out_h.numel() * out_h.element_size()
-
     extra = dict(gate=devv["gate"], norm_weight=devv["norm_weight"], eps=w.eps) if w.gated else {}
     if w.raw is not None:
         extra.update(raw_gate=devv["raw_gate"], A_log=devv["A_log"], dt_bias=devv["dt_bias"],
                      raw_beta=devv["raw_beta"])
     else:
         extra.update(g=devv["g"], beta=devv["beta"])
-    # One library call per step: it enqueues the copy of the packed inputs, the
-    # decode step and the copy of the output back.
     step = kda.HostStep(devv["q"], devv["k"], devv["v"], pool, devv["slot_idx"], host_in=host_buf,
                         dev_in=dev_buf, host_out=out_h, out=out_d, stream=stream, scale=w.scale,
                         state_layout=w.state_layout, **extra)
+    return step, host_buf, dev_buf, out_h
 
-    with torch.cuda.stream(stream):
-        for _ in range(10):
-            step()
-    torch.cuda.synchronize()
+
+def _timed_steps(fn, steps, stream, lead_in, copy_stream=None):
+    """Device time of ``steps`` calls of fn between events on ``stream``, after
+    ``lead_in`` untimed calls enqueued without a host sync (the first event is
+    recorded on a busy stream); a copy stream waits for the first event, so no
+    copy of the timed steps starts before it."""
+    import torch
+
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        for _ in range(4):  # untimed lead-in: the first event is recorded on a busy stream
-            step()
+        for _ in range(lead_in):
+            fn()
         e0.record(stream)
+        if copy_stream is not None:
+            copy_stream.wait_event(e0)
         for _ in range(steps):
-            step()
+            fn()
         e1.record(stream)
     torch.cuda.synchronize()
-    ms = reduce_max(e0.elapsed_time(e1), dev)
-    return {"value": round(ms * 1e3 / (steps * world), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps,
-            "how": "one kda_decode_host call per step (HostStep): copy of the packed inputs from pinned host "
-                   "memory, the decode kernel, copy of the output back; the state pool stays resident on the GPU"}
+    return e0.elapsed_time(e1)
+
+
+def run_e2e(kda, w, dev, stream, steps, world):
+    """µs per step with each step's inputs copied from pinned host memory and
+    its output copied back, through the public API; the state pool stays
+    resident on the GPU.  The value is the pipelined form (``HostPipeline``,
+    the C ABI's ``kda_decode_host_pipelined``): two staging sets used in turn,
+    each step's copy in on a second stream so that it overlaps the previous
+    step's kernel and copy out.  Also reported: the same steps one after
+    another on one stream (``HostStep``, ``kda_decode_host``), and the copy in
+    alone."""
+    import torch
+
+    pool = w.state.to(dev)
+    copy_stream = torch.cuda.Stream(device=dev)
+    sets = [_host_step(kda, w, dev, stream, pool) for _ in range(2)]
+    pipe = kda.HostPipeline([s[0] for s in sets], copy_stream)
+    h2d = sets[0][1].numel()  # the packed buffer each step copies (inputs and their 16-byte alignment)
+    d2h = sets[0][3].numel() * sets[0][3].element_size()
+
+    for _ in range(10):
+        pipe()
+    torch.cuda.synchronize()
+    ms_eager = reduce_max(_timed_steps(pipe, steps, stream, lead_in=4, copy_stream=copy_stream), dev)
+    # The same calls captured once into a CUDA graph (as a serving loop replays
+    # its decode steps): each replay runs `per_graph` steps, copies included.
+    per_graph = 2 * max(1, min(steps, 64) // 2)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        copy_stream.wait_stream(stream)  # fork the copy stream into the capture
+        pipe.rearm()
+        for _ in range(per_graph):
+            pipe()
+        stream.wait_stream(copy_stream)  # and join it back
+    torch.cuda.synchronize()
+    reps = max(1, -(-steps // per_graph))
+    ms_graph = reduce_max(_timed_steps(graph.replay, reps, stream, lead_in=2), dev)
+    del graph
+    serial = sets[0][0]
+    ms_serial = reduce_max(_timed_steps(serial, steps, stream, lead_in=4), dev)
+    host_buf, dev_buf = sets[0][1], sets[0][2]
+    ms_copy = reduce_max(_timed_steps(lambda: dev_buf.copy_(host_buf, non_blocking=True), steps, stream,
+                                      lead_in=4), dev)
+    return {"value": round(ms_graph * 1e3 / (reps * per_graph * world), 3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": reps * per_graph,
+            "eager_us": round(ms_eager * 1e3 / (steps * world), 3),
+            "serial_us": round(ms_serial * 1e3 / (steps * world), 3),
+            "h2d_copy_us": round(ms_copy * 1e3 / steps, 3),
+            "how": f"kda_decode_host_pipelined through HostPipeline, {per_graph} steps captured in a CUDA graph "
+                   "and replayed: per step the copy of the packed inputs from pinned host memory (on a copy "
+                   "stream, overlapping the previous step), the decode kernel and the copy of the output back; "
+                   "two staging sets in turn; the state pool stays resident on the GPU.  eager_us: the same "
+                   "calls issued one by one from Python; serial_us: the steps one after another on one stream "
+                   "(kda_decode_host, eager); h2d_copy_us: the copy in alone"}
 
 
 def run_e2e_prefill(kda, w, dev, stream, steps, world):

@@ -91,6 +91,9 @@ extern "C" {
 /* Same type as cudaStream_t. */
 struct CUstream_st;
 typedef struct CUstream_st *kda_stream_t;
+/* Same type as cudaEvent_t. */
+struct CUevent_st;
+typedef struct CUevent_st *kda_event_t;
 
 typedef enum {
     KDA_OK = 0,
@@ -259,6 +262,40 @@ KDA_API kda_status kda_decode_ex(const kda_decode_args *args, kda_stream_t strea
  */
 KDA_API kda_status kda_decode_host(const kda_decode_args *args, const void *host_in, void *dev_in,
                                    int64_t in_bytes, void *host_out, kda_stream_t stream);
+
+/*
+ * kda_decode_host with the copy in on a second stream, so that consecutive
+ * steps overlap: one step's copy in runs while the previous step computes and
+ * copies its output out.  Like kda_decode_host, none of the pages describes
+ * such an entry point: it is this library's own, for callers that feed the
+ * step from host memory step after step (FlashInfer #4562's PR description
+ * names caller-stream execution and caller-owned buffers, which this keeps).
+ *
+ * It enqueues, in order:
+ *   on copy_stream: a wait for staging_free, the copy of in_bytes bytes from
+ *                   host_in to dev_in, a record of staging_ready;
+ *   on stream:      a wait for staging_ready, the step of kda_decode_ex(args),
+ *                   a record of staging_free, the copy of the output
+ *                   (N*T*HV*V bf16 from args->out) to host_out.
+ * A "staging set" is (host_in, dev_in, host_out, staging_ready, staging_free)
+ * with args pointing into dev_in.  The caller cycles two (or more) sets: the
+ * wait on staging_free keeps a copy in from overwriting dev_in while the step
+ * that reads it may still run (an event never recorded counts as complete).
+ * Steps run in the order of the calls on `stream`, so the state pool is
+ * updated step after step exactly as with kda_decode_host.  The caller owns
+ * both streams (distinct, on the current device) and both events (created
+ * once, e.g. cudaEventCreateWithFlags(..., cudaEventDisableTiming)); host_in
+ * and host_out must be page-locked, and host_out holds the step's output once
+ * `stream` has passed it.  The library allocates nothing.
+ *
+ * Errors: those of kda_decode_host; KDA_ERR_INVALID_ARG also for a NULL
+ * stream, copy_stream, staging_ready or staging_free, or stream ==
+ * copy_stream.  Nothing is enqueued unless validation passes.
+ */
+KDA_API kda_status kda_decode_host_pipelined(const kda_decode_args *args, const void *host_in, void *dev_in,
+                                             int64_t in_bytes, void *host_out, kda_stream_t stream,
+                                             kda_stream_t copy_stream, kda_event_t staging_ready,
+                                             kda_event_t staging_free);
 
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);

@@ -24,7 +24,7 @@ import threading
 
 import torch
 
-__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "kda_prefill",
+__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "HostPipeline", "kda_prefill",
            "prefill_workspace_bytes", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_ERR_SCRATCH_LIMIT", "KDA_STATE_FP32",
@@ -79,6 +79,7 @@ EXPORTED_SYMBOLS = {
     "kda_decode_gated_rmsnorm_bf16_state": ([_P] * 9 + [_F, _P] + [_I] * 5 + [_F, _P], ctypes.c_int),
     "kda_decode_ex": ([ctypes.POINTER(DecodeArgs), _P], ctypes.c_int),
     "kda_decode_host": ([ctypes.POINTER(DecodeArgs), _P, _P, _I, _P, _P], ctypes.c_int),
+    "kda_decode_host_pipelined": ([ctypes.POINTER(DecodeArgs), _P, _P, _I, _P, _P, _P, _P, _P], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_abi_version": ([], ctypes.c_int32),
     # include/kda_prefill.h
@@ -375,6 +376,59 @@ class HostStep:
         st = self._fn(self._ref, *self._ptrs, self._stream)
         if st != KDA_OK:
             raise KdaError(st, "kda_decode_host")
+
+
+class HostPipeline:
+    """Steps run from host memory with each step's copy in overlapping the
+    previous step's kernel and copy out (``kda_decode_host_pipelined`` of the C
+    ABI).
+
+    ``steps`` are :class:`HostStep` objects bound to the same ``stream`` and
+    state pool, each with its own staging buffers (``host_in``, ``dev_in``,
+    ``host_out``); calling the pipeline runs the next one in turn, its copy in
+    enqueued on ``copy_stream``.  Two staging sets let step i+1's inputs travel
+    while step i computes; the events that order a set's reuse are made here,
+    once.  A step's output is in its ``host_out`` once ``stream`` has passed it.
+    """
+
+    def __init__(self, steps, copy_stream):
+        if len(steps) < 1 or len({id(s._torch_stream) for s in steps}) != 1:
+            raise ValueError("steps must share one stream")
+        self._steps = list(steps)
+        self._copy = copy_stream
+        self._copy_handle = _stream_handle(copy_stream)
+        stream = steps[0]._torch_stream
+        if copy_stream.cuda_stream == stream.cuda_stream:
+            raise ValueError("copy_stream must differ from the steps' stream")
+        self._events = []
+        for _ in self._steps:  # torch creates an event's handle on its first record
+            ready, free = torch.cuda.Event(), torch.cuda.Event()
+            ready.record(copy_stream)
+            free.record(stream)
+            self._events.append((ready, free))
+        torch.cuda.synchronize()
+        self._handles = [(ctypes.c_void_p(r.cuda_event), ctypes.c_void_p(f.cuda_event)) for r, f in self._events]
+        self._fn = library().kda_decode_host_pipelined
+        self._next = 0
+
+    def rearm(self):
+        """Record every staging set's "free" event on the steps' stream now, so
+        that the next wait on it refers to this point.  Call it first when
+        capturing steps into a CUDA graph (inside the capture, after forking the
+        copy stream from the steps' stream): a captured wait must refer to a
+        record made inside the same capture."""
+        stream = self._steps[0]._torch_stream
+        for _, free in self._events:
+            free.record(stream)
+
+    def __call__(self):
+        i = self._next
+        st = self._steps[i]
+        rc = self._fn(st._ref, *st._ptrs, st._stream, self._copy_handle, *self._handles[i])
+        if rc != KDA_OK:
+            raise KdaError(rc, "kda_decode_host_pipelined")
+        self._next = (i + 1) % len(self._steps)
+        return st
 
 
 # ---------------------------------------------------------------- chunked prefill

@@ -27,12 +27,18 @@ namespace {
 using namespace kda_host;
 
 // Host staging of kda_decode_host: the step's inputs are copied from host_in to
-// dev_in before the kernel, the output from out to host_out after it.
+// dev_in before the kernel, the output from out to host_out after it.  With a
+// copy stream (kda_decode_host_pipelined) the copy in runs there, between a
+// wait for `free_ev` and a record of `ready_ev`; the kernel waits for
+// `ready_ev` and is followed by a record of `free_ev`.
 struct HostCopies {
   const void* host_in;
   void* dev_in;
   int64_t in_bytes;
   void* host_out;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ready_ev = nullptr;
+  cudaEvent_t free_ev = nullptr;
 };
 
 kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, const HostCopies* hc = nullptr) {
@@ -226,16 +232,27 @@ kda_status launch(const kda_decode_args& a, bool gated, kda_stream_t stream, con
     // With host copies around the step, the launch was checked above (once per
     // kernel and device: the kernel loads, a cluster fits) before the copy in
     // is enqueued.
-    if (hc->in_bytes > 0 &&
-        cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
-                        cfg.stream) != cudaSuccess)
+    if (hc->copy_stream) {
+      if (cudaStreamWaitEvent(hc->copy_stream, hc->free_ev, 0) != cudaSuccess) return KDA_ERR_CUDA;
+      if (hc->in_bytes > 0 &&
+          cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
+                          hc->copy_stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+      if (cudaEventRecord(hc->ready_ev, hc->copy_stream) != cudaSuccess ||
+          cudaStreamWaitEvent(cfg.stream, hc->ready_ev, 0) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    } else if (hc->in_bytes > 0 &&
+               cudaMemcpyAsync(hc->dev_in, hc->host_in, static_cast<size_t>(hc->in_bytes), cudaMemcpyHostToDevice,
+                               cfg.stream) != cudaSuccess) {
       return KDA_ERR_CUDA;
+    }
   }
   // The dense form's kernels take the smaller parameter block, which is the
   // leading part of p.
   void* kargs[] = {&p};
   err = cudaLaunchKernelExC(&cfg, func, kargs);
   if (err != cudaSuccess) return KDA_ERR_CUDA;
+  if (hc && hc->copy_stream && cudaEventRecord(hc->free_ev, cfg.stream) != cudaSuccess) return KDA_ERR_CUDA;
   if (hc && cudaMemcpyAsync(hc->host_out, a.out, static_cast<size_t>(out_elems) * 2, cudaMemcpyDeviceToHost,
                             cfg.stream) != cudaSuccess)
     return KDA_ERR_CUDA;
@@ -332,6 +349,21 @@ kda_status kda_decode_host(const kda_decode_args* args, const void* host_in, voi
   return launch(*args, /*gated=*/args->gate != nullptr, stream, &hc);
 }
 
+kda_status kda_decode_host_pipelined(const kda_decode_args* args, const void* host_in, void* dev_in,
+                                     int64_t in_bytes, void* host_out, kda_stream_t stream,
+                                     kda_stream_t copy_stream, kda_event_t staging_ready,
+                                     kda_event_t staging_free) {
+  if (args == nullptr || stream == nullptr || copy_stream == nullptr || stream == copy_stream ||
+      staging_ready == nullptr || staging_free == nullptr)
+    return KDA_ERR_INVALID_ARG;
+  if ((args->gate == nullptr) != (args->norm_weight == nullptr)) return KDA_ERR_INVALID_ARG;
+  HostCopies hc{host_in, dev_in, in_bytes, host_out};
+  hc.copy_stream = reinterpret_cast<cudaStream_t>(copy_stream);
+  hc.ready_ev = reinterpret_cast<cudaEvent_t>(staging_ready);
+  hc.free_ev = reinterpret_cast<cudaEvent_t>(staging_free);
+  return launch(*args, /*gated=*/args->gate != nullptr, stream, &hc);
+}
+
 const char* kda_status_string(kda_status status) {
   switch (status) {
     case KDA_OK: return "ok";
@@ -350,6 +382,6 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 6; }
+int32_t kda_abi_version(void) { return (1 << 16) | 7; }
 
 }  // extern "C"

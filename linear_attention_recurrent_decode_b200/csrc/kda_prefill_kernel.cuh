@@ -27,7 +27,7 @@
 //   1. kda_prefill_chunk_kernel (one CTA per (n, h, chunk), all chunks at
 //      once): Gamma in fp64, the decay factors, M and P, the substitution for
 //      W and Ut; writes them to the workspace.
-//   2. kda_prefill_state_kernel (one CTA per (n, h, 16-column value tile),
+//   2. kda_prefill_state_kernel (one CTA per (n, h, 8-column value tile),
 //      chunks in order): the state chain U = Ut - W S0, S_C = D S0 + Kh^T U,
 //      keeping S in shared memory; writes each chunk's start state and U to the
 //      workspace and the final state back to the pool slot.
@@ -56,7 +56,7 @@ namespace kdap {
 constexpr int kC = 64;        // tokens per chunk
 constexpr int kK = 128;       // key dimension (the kernels are written for K = V = 128)
 constexpr int kV = 128;       // value dimension
-constexpr int kBV = 16;       // value columns per state-chain CTA
+constexpr int kBV = 8;        // value columns per state-chain CTA
 constexpr float kSafeExp = 80.f;  // |Gamma_t - Gamma_r| bound of the factored path
 
 struct Params {
@@ -113,13 +113,20 @@ __device__ __forceinline__ float exp_of(double x) {
 
 // ---------------------------------------------------------------- kernel 1
 // Shared memory of the chunk kernel (dynamic; about 200 KB).
+// Rows of the transposed factor buffers are padded to 68 floats: the stores
+// from consecutive key channels then spread over the banks (4-way instead of
+// 32-way), and every row still starts on a 16-byte boundary for the float4
+// reads of the Gram products.
+constexpr int kCP = kC + 4;
 struct ChunkSmem {
-  double gam[kC][kK];               // Gamma_t - Gamma_r (fast path) or Gamma_t (exact path); 64 KB
+  double gam[kC][kK];               // Gamma_t, the cumulative log-decay from the chunk start; 64 KB
   float kt[kC][kK];                 // Kt = k exp(Gamma_t) [t][i]; the solve reads its columns
-  float at[kK][kC];                 // k_t exp(Gamma_t - Gamma_r) [i][t]
-  float aq[kK][kC];                 // q_t exp(Gamma_t - Gamma_r) [i][t]
-  float bk[kK][kC];                 // k_s exp(Gamma_r - Gamma_s) [i][s]
+  float at[kK][kCP];                // k_t exp(Gamma_t - Gamma_r) [i][t]
+  float aq[kK][kCP];                // q_t exp(Gamma_t - Gamma_r) [i][t]
+  float bk[kK][kCP];                // k_s exp(Gamma_r - Gamma_s) [i][s]
   float L[kC][kC];                  // beta_t M[t][s] (s < t), zero elsewhere
+  float e_ref[kK];                  // exp(Gamma_r) per channel (factored path)
+  float e_end_ref[kK];              // exp(Gamma_C - Gamma_r) per channel (factored path)
   float beta[kC];
   int exact;                        // some channel is outside the factored path's range
 };
@@ -129,7 +136,7 @@ struct ChunkRaw {
   __nv_bfloat16 k[kC][kK];
   __nv_bfloat16 v[kC][kV];
 };
-static_assert(sizeof(ChunkRaw) <= 3 * kK * kC * sizeof(float), "raw inputs fit over the factor buffers");
+static_assert(sizeof(ChunkRaw) <= 3 * kK * kCP * sizeof(float), "raw inputs fit over the factor buffers");
 
 constexpr int kChunkThreads = 256;
 
@@ -194,43 +201,42 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       const double d = sm.gam[t][tid] - gam_ref;
       worst = fmax(worst, fabs(d));
     }
-    if (worst > kSafeExp) atomicOr(&sm.exact, 1);
+    // the factored path also forms exp(Gamma_r) and exp(Gamma_C - Gamma_r): keep
+    // them normal fp32 numbers
+    if (worst > kSafeExp || gam_ref < -kSafeExp) atomicOr(&sm.exact, 1);
+    sm.e_ref[tid] = exp_of(gam_ref);
+    sm.e_end_ref[tid] = exp_of(gam_end - gam_ref);
   }
   __syncthreads();
   const bool exact = sm.exact != 0;
 
-  // ---- 2. per-token decayed keys/queries (written straight to the workspace)
-  // and, on the factored path, the factors around the reference token.
+  // ---- 2. per-token decays: the workspace's Kh and Qt, the solve's Kt, and on
+  // the factored path the factors around the reference token r, from two
+  // exponentials per element (exp(+-(Gamma_t - Gamma_r))) and the channel's
+  // exp(Gamma_r), exp(Gamma_C - Gamma_r).
   float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
-  for (int e = tid; e < kC * kK; e += kChunkThreads) {  // [t][i] order: consecutive threads, consecutive i
-    const int t = e / kK, i = e % kK;
-    const double gt = sm.gam[t][i];
-    const float kv = __bfloat162float(raw.k[t][i]);
-    sm.kt[t][i] = kv * exp_of(gt);                                   // k exp(Gamma_t)
-    rec[Workspace::kKh + t * kK + i] = kv * exp_of(sm.gam[kC - 1][i] - gt);  // k exp(Gamma_C - Gamma_t)
-  }
-  for (int e = tid; e < kC * kK; e += kChunkThreads) {
-    const int t = e / kK, i = e % kK;
-    rec[Workspace::kQ + t * kK + i] = __bfloat162float(raw.q[t][i]) * exp_of(sm.gam[t][i]);  // q exp(Gamma_t)
-  }
-  if (tid < kK) rec[Workspace::kDc + tid] = exp_of(gam_end);
-  __syncthreads();  // raw q/k still needed below; kt complete
-
-  // ---- 3. M and P
   float* const Pm = rec + Workspace::kP;  // P[t][s]
+  if (tid < kK) rec[Workspace::kDc + tid] = exp_of(gam_end);
+  constexpr int kPer = kC * kK / kChunkThreads;  // elements per thread
   if (!exact) {
     // The factors go through registers: the raw inputs they are made from live
     // in the buffers they are written to.
-    float fa[kC * kK / kChunkThreads], fq[kC * kK / kChunkThreads], fb[kC * kK / kChunkThreads];
+    float fa[kPer], fq[kPer], fb[kPer];
 #pragma unroll
-    for (int j = 0; j < kC * kK / kChunkThreads; ++j) {
-      const int e = tid + j * kChunkThreads;
+    for (int j = 0; j < kPer; ++j) {
+      const int e = tid + j * kChunkThreads;  // consecutive threads, consecutive channels
       const int t = e / kK, i = e % kK;
       const double d = sm.gam[t][i] - sm.gam[kRef][i];
+      const float up = exp_of(d);      // exp(Gamma_t - Gamma_r), in [e^-80, e^80] on this path
+      const float down = __frcp_rn(up);  // exp(Gamma_r - Gamma_t), correctly rounded reciprocal
       const float kv = __bfloat162float(raw.k[t][i]);
-      fa[j] = kv * exp_of(d);
-      fq[j] = __bfloat162float(raw.q[t][i]) * exp_of(d);
-      fb[j] = kv * exp_of(-d);
+      const float qv = __bfloat162float(raw.q[t][i]);
+      fa[j] = kv * up;
+      fq[j] = qv * up;
+      fb[j] = kv * down;
+      sm.kt[t][i] = fa[j] * sm.e_ref[i];                                // k exp(Gamma_t)
+      rec[Workspace::kKh + t * kK + i] = fb[j] * sm.e_end_ref[i];       // k exp(Gamma_C - Gamma_t)
+      rec[Workspace::kQ + t * kK + i] = fq[j] * sm.e_ref[i];            // q exp(Gamma_t)
     }
     __syncthreads();
     // The solve needs v, which the factors overwrite: move it into the Gamma
@@ -239,7 +245,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
     for (int e = tid; e < kC * kV; e += kChunkThreads) vf[e] = __bfloat162float(raw.v[e / kV][e % kV]);
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kC * kK / kChunkThreads; ++j) {
+    for (int j = 0; j < kPer; ++j) {
       const int e = tid + j * kChunkThreads;
       const int t = e / kK, i = e % kK;
       sm.at[i][t] = fa[j];
@@ -247,41 +253,75 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       sm.bk[i][t] = fb[j];
     }
     __syncthreads();
-    // 4 x 4 tiles of (t, s); tiles above the diagonal are skipped
-    const int tb = tid / 16, sb = tid % 16;
-    float m[4][4], pp[4][4];
+    // ---- 3. M and P in 4 x 4 tiles of (t, s): the 136 tiles on or below the
+    // diagonal go to the first 136 threads (whole warps past them skip the
+    // loop), the tiles above it are zeros written by the rest.
+    constexpr int kTb = kC / 4;                           // tile rows (16)
+    constexpr int kLower = kTb * (kTb + 1) / 2;          // 136
+    int tb, sb;
+    if (tid < kLower) {  // tid -> (tb, sb) with sb <= tb, row by row
+      tb = static_cast<int>((sqrtf(8.f * tid + 1.f) - 1.f) * 0.5f);
+      while ((tb + 1) * (tb + 2) / 2 <= tid) ++tb;
+      while (tb * (tb + 1) / 2 > tid) --tb;
+      sb = tid - tb * (tb + 1) / 2;
+      float2 m[4][2], pp[4][2];  // pairs of s
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) m[a][b] = pp[a][b] = 0.f;
-    if (sb <= tb) {
+      for (int a = 0; a < 4; ++a) m[a][0] = m[a][1] = pp[a][0] = pp[a][1] = make_float2(0.f, 0.f);
+#pragma unroll 4
       for (int i = 0; i < kK; ++i) {
         const float4 A = *reinterpret_cast<const float4*>(&sm.at[i][tb * 4]);
         const float4 Q = *reinterpret_cast<const float4*>(&sm.aq[i][tb * 4]);
         const float4 B = *reinterpret_cast<const float4*>(&sm.bk[i][sb * 4]);
-        const float av[4] = {A.x, A.y, A.z, A.w}, qv[4] = {Q.x, Q.y, Q.z, Q.w}, bv[4] = {B.x, B.y, B.z, B.w};
+        const float av[4] = {A.x, A.y, A.z, A.w}, qv[4] = {Q.x, Q.y, Q.z, Q.w};
+        const float2 b01 = make_float2(B.x, B.y), b23 = make_float2(B.z, B.w);
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            m[a][b] = fmaf(av[a], bv[b], m[a][b]);
-            pp[a][b] = fmaf(qv[a], bv[b], pp[a][b]);
-          }
+        for (int a = 0; a < 4; ++a) {
+          m[a][0] = __ffma2_rn(make_float2(av[a], av[a]), b01, m[a][0]);
+          m[a][1] = __ffma2_rn(make_float2(av[a], av[a]), b23, m[a][1]);
+          pp[a][0] = __ffma2_rn(make_float2(qv[a], qv[a]), b01, pp[a][0]);
+          pp[a][1] = __ffma2_rn(make_float2(qv[a], qv[a]), b23, pp[a][1]);
+        }
       }
-    }
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int t = tb * 4 + a;
+      for (int a = 0; a < 4; ++a) {
+        const int t = tb * 4 + a;
+        const float mv[4] = {m[a][0].x, m[a][0].y, m[a][1].x, m[a][1].y};
+        const float pv[4] = {pp[a][0].x, pp[a][0].y, pp[a][1].x, pp[a][1].y};
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int s = sb * 4 + b;
-        sm.L[t][s] = (s < t) ? sm.beta[t] * m[a][b] : 0.f;
-        Pm[t * kC + s] = (s <= t) ? pp[a][b] : 0.f;
+        for (int b = 0; b < 4; ++b) {
+          const int s = sb * 4 + b;
+          sm.L[t][s] = (s < t) ? sm.beta[t] * mv[b] : 0.f;
+          Pm[t * kC + s] = (s <= t) ? pv[b] : 0.f;
+        }
       }
+    } else {  // the 120 tiles above the diagonal: zeros
+      // k -> (r, c) with c < r in the strict lower triangle, mirrored to (tb, sb) = (c, r)
+      const int k = tid - kLower;
+      int r = static_cast<int>((sqrtf(8.f * k + 1.f) + 1.f) * 0.5f);
+      while (r * (r - 1) / 2 > k) --r;
+      while ((r + 1) * r / 2 <= k) ++r;
+      tb = k - r * (r - 1) / 2;
+      sb = r;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          sm.L[tb * 4 + a][sb * 4 + b] = 0.f;
+          Pm[(tb * 4 + a) * kC + sb * 4 + b] = 0.f;
+        }
     }
   } else {
-    // Exact path: every pair's exponential from the fp64 Gamma difference.
-    // One thread per (t, s) pair group; rare (decays beyond e^80 within half a chunk).
+    // Exact path (rare: decays beyond e^80 within half a chunk): every
+    // exponential from its own fp64 Gamma difference.
+    for (int e = tid; e < kC * kK; e += kChunkThreads) {
+      const int t = e / kK, i = e % kK;
+      const double gt = sm.gam[t][i];
+      const float kv = __bfloat162float(raw.k[t][i]);
+      const float dt = exp_of(gt);
+      sm.kt[t][i] = kv * dt;                                                   // k exp(Gamma_t)
+      rec[Workspace::kKh + t * kK + i] = kv * exp_of(sm.gam[kC - 1][i] - gt);  // k exp(Gamma_C - Gamma_t)
+      rec[Workspace::kQ + t * kK + i] = __bfloat162float(raw.q[t][i]) * dt;    // q exp(Gamma_t)
+    }
     for (int e = tid; e < kC * kC; e += kChunkThreads) {
       const int t = e / kC, s = e % kC;
       float mv = 0.f, pv = 0.f;
@@ -315,22 +355,28 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   {
     const int j = tid;
     const float* const vf = reinterpret_cast<const float*>(&sm.gam[0][0]);
-    float x[kC];
+    // x kept as pairs for packed fp32x2 FMAs; two pair accumulators (four
+    // partial sums) per row keep the dependent chain short
+    float2 x2[kC / 2];
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
-      float acc = sm.beta[t] * (j < kK ? sm.kt[t][j] : vf[t * kV + (j - kK)]);
+      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int s = 0; s + 3 < t; s += 4) {
         const float4 l = *reinterpret_cast<const float4*>(&sm.L[t][s]);
-        acc = fmaf(-l.x, x[s], acc);
-        acc = fmaf(-l.y, x[s + 1], acc);
-        acc = fmaf(-l.z, x[s + 2], acc);
-        acc = fmaf(-l.w, x[s + 3], acc);
+        a01 = __ffma2_rn(make_float2(-l.x, -l.y), x2[s / 2], a01);
+        a23 = __ffma2_rn(make_float2(-l.z, -l.w), x2[s / 2 + 1], a23);
       }
+      float a = sm.beta[t] * (j < kK ? sm.kt[t][j] : vf[t * kV + (j - kK)]);
 #pragma unroll
-      for (int s = t & ~3; s < t; ++s) acc = fmaf(-sm.L[t][s], x[s], acc);
-      x[t] = acc;
+      for (int s = t & ~3; s < t; ++s) a = fmaf(-sm.L[t][s], (s & 1) ? x2[s / 2].y : x2[s / 2].x, a);
+      const float xt = a + ((a01.x + a01.y) + (a23.x + a23.y));
+      if (t & 1) x2[t / 2].y = xt;
+      else x2[t / 2].x = xt;
     }
+    float x[kC];
+#pragma unroll
+    for (int t = 0; t < kC; ++t) x[t] = (t & 1) ? x2[t / 2].y : x2[t / 2].x;
     if (j < kK) {
       float* const wt = rec + Workspace::kWt + j * kC;  // W^T row j
 #pragma unroll
@@ -344,7 +390,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
 }
 
 // ---------------------------------------------------------------- kernel 2
+// One CTA per (n, h, 8-column value tile) walks the chunks in order with its
+// K x 8 state tile in shared memory; the next chunk's W^T, Kh, Ut and exp(Gamma_C)
+// are staged with cp.async while the current one is processed.  Both products
+// split their reduction over the CTA (W S over quarters of K, Kh^T U over halves
+// of the chunk), use packed fp32x2 FMAs, and sum the partials in a fixed order.
 constexpr int kStateThreads = 256;
+constexpr int kCU = kC + 4;  // padded rows of the transposed partial buffers
 
 struct StateBuf {
   float wt[kK][kC];   // W^T
@@ -354,8 +406,10 @@ struct StateBuf {
 };
 struct StateSmem {
   StateBuf buf[2];
-  float s[kK][kBV];      // state tile
-  float part[4][kC][kBV];  // (W S) partial sums over quarters of K; part[0] then holds U
+  float s[kK][kBV];             // state tile
+  float pw[4][kBV][kCU];        // (W S) partial sums per quarter of K, [j][t]
+  float u[kC][kBV + 2];         // U of the current chunk, [t][j] (rows padded to 10 floats)
+  float ps[2][kBV][kK + 4];      // (Kh^T U) partial sums per half of the chunk, [j][i]
 };
 
 __device__ __forceinline__ void stage_chunk(StateBuf& b, const float* rec, int col0, int tid) {
@@ -369,6 +423,9 @@ __device__ __forceinline__ void stage_chunk(StateBuf& b, const float* rec, int c
   }
   for (int c = tid; c < kK / 4; c += kStateThreads) cp_async16(&b.dc[4 * c], rec + Workspace::kDc + 4 * c);
 }
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 splat(float x) { return make_float2(x, x); }
 
 __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(const Params p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -384,23 +441,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
   if (slot < 0) return;
 
   float* const blk = p.state + (static_cast<int64_t>(slot) * p.HV + h) * kK * kV;
-  // initial state tile
-  for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {
+  for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {  // initial state tile
     const int i = c / (kBV / 4), pc = c % (kBV / 4);
     cp_async16(&sm.s[i][pc * 4], blk + i * kV + col0 + pc * 4);
   }
   stage_chunk(sm.buf[0], p.ws + Workspace::record(unit, 0, p.nchunks), col0, tid);
   cp_async_commit();
 
-  // GEMM 1 (W S over a quarter of K): 4 tokens x 4 columns per thread
-  const int g1_t = (tid % 16) * 4;
-  const int g1_j = ((tid / 16) % 4) * 4;
-  const int g1_q = tid / 64;  // quarter of K
-  // U = Ut - sum of the quarters: 4 elements per thread
-  const int u_t = tid / 4, u_j = (tid % 4) * 4;
-  // GEMM 2 (Kh^T U): 2 key rows x 4 columns per thread
-  const int g2_i = (tid % 64) * 2;
-  const int g2_j = (tid / 64) * 4;
+  // W S: thread (quarter of K, 4 tokens, 2 columns)
+  const int a_t = (tid % 16) * 4, a_j = ((tid / 16) % 4) * 2, a_q = tid / 64;
+  // U: thread (token, column pair)
+  const int u_t = tid % 64, u_j = (tid / 64) * 2;
+  // Kh^T U: thread (2 key rows, 4 columns, half of the chunk)
+  const int b_i = (tid % 64) * 2, b_j = ((tid / 64) % 2) * 4, b_h = tid / 128;
 
   for (int32_t c = 0; c < p.nchunks; ++c) {
     const int cb = c & 1;
@@ -422,66 +475,72 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
           *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
     }
 
-    // GEMM 1: partial (W S)[t][j] over one quarter of K
-    {
-      float acc[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
-      const int i_lo = g1_q * (kK / 4);
+    {  // W S over one quarter of K
+      float2 acc[4] = {splat(0.f), splat(0.f), splat(0.f), splat(0.f)};
+      const int i_lo = a_q * (kK / 4);
 #pragma unroll 8
       for (int i = i_lo; i < i_lo + kK / 4; ++i) {
-        const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][g1_t]);
-        const float4 sv4 = *reinterpret_cast<const float4*>(&sm.s[i][g1_j]);
-        const float wv[4] = {w.x, w.y, w.z, w.w}, sv[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
+        const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][a_t]);
+        const float2 sv = *reinterpret_cast<const float2*>(&sm.s[i][a_j]);
+        acc[0] = ffma2(splat(w.x), sv, acc[0]);
+        acc[1] = ffma2(splat(w.y), sv, acc[1]);
+        acc[2] = ffma2(splat(w.z), sv, acc[2]);
+        acc[3] = ffma2(splat(w.w), sv, acc[3]);
+      }
+      *reinterpret_cast<float4*>(&sm.pw[a_q][a_j][a_t]) = make_float4(acc[0].x, acc[1].x, acc[2].x, acc[3].x);
+      *reinterpret_cast<float4*>(&sm.pw[a_q][a_j + 1][a_t]) = make_float4(acc[0].y, acc[1].y, acc[2].y, acc[3].y);
+    }
+    __syncthreads();
+    {  // U = Ut - W S, the quarters summed in a fixed order
+      float uo[2];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(wv[a], sv[bb], acc[a][bb]);
+      for (int jj = 0; jj < 2; ++jj) {
+        const int j = u_j + jj;
+        const float ws = (sm.pw[0][j][u_t] + sm.pw[1][j][u_t]) + (sm.pw[2][j][u_t] + sm.pw[3][j][u_t]);
+        uo[jj] = b.ut[u_t][j] - ws;
+      }
+      *reinterpret_cast<float2*>(&sm.u[u_t][u_j]) = make_float2(uo[0], uo[1]);
+      *reinterpret_cast<float2*>(rec + Workspace::kU + u_t * kV + col0 + u_j) = make_float2(uo[0], uo[1]);
+    }
+    __syncthreads();
+    {  // Kh^T U over one half of the chunk
+      float2 acc[2][2] = {{splat(0.f), splat(0.f)}, {splat(0.f), splat(0.f)}};
+      const int t_lo = b_h * (kC / 2);
+#pragma unroll 8
+      for (int t = t_lo; t < t_lo + kC / 2; ++t) {
+        const float2 kh = *reinterpret_cast<const float2*>(&b.kh[t][b_i]);
+        const float2 u0 = *reinterpret_cast<const float2*>(&sm.u[t][b_j]);
+        const float2 u1 = *reinterpret_cast<const float2*>(&sm.u[t][b_j + 2]);
+        acc[0][0] = ffma2(splat(kh.x), u0, acc[0][0]);
+        acc[0][1] = ffma2(splat(kh.x), u1, acc[0][1]);
+        acc[1][0] = ffma2(splat(kh.y), u0, acc[1][0]);
+        acc[1][1] = ffma2(splat(kh.y), u1, acc[1][1]);
       }
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-        *reinterpret_cast<float4*>(&sm.part[g1_q][g1_t + a][g1_j]) =
-            make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+      for (int a = 0; a < 2; ++a) {
+        sm.ps[b_h][b_j][b_i + a] = acc[a][0].x;
+        sm.ps[b_h][b_j + 1][b_i + a] = acc[a][0].y;
+        sm.ps[b_h][b_j + 2][b_i + a] = acc[a][1].x;
+        sm.ps[b_h][b_j + 3][b_i + a] = acc[a][1].y;
+      }
     }
+    // S = D S + Kh^T U: thread (key row, 4 columns).  The decay is read before
+    // the barrier: after it no thread touches this chunk's stage buffer, which
+    // the next iteration's prefetch then refills.
+    const int s_i = tid / 2, s_j = (tid % 2) * 4;
+    const float d = b.dc[s_i];
     __syncthreads();
-    {  // U = Ut - (W S), quarters summed in a fixed order
-      const float4 p0 = *reinterpret_cast<const float4*>(&sm.part[0][u_t][u_j]);
-      const float4 p1 = *reinterpret_cast<const float4*>(&sm.part[1][u_t][u_j]);
-      const float4 p2 = *reinterpret_cast<const float4*>(&sm.part[2][u_t][u_j]);
-      const float4 p3 = *reinterpret_cast<const float4*>(&sm.part[3][u_t][u_j]);
-      const float4 ut = *reinterpret_cast<const float4*>(&b.ut[u_t][u_j]);
-      const float4 u = make_float4(ut.x - ((p0.x + p1.x) + (p2.x + p3.x)), ut.y - ((p0.y + p1.y) + (p2.y + p3.y)),
-                                   ut.z - ((p0.z + p1.z) + (p2.z + p3.z)), ut.w - ((p0.w + p1.w) + (p2.w + p3.w)));
-      __syncthreads();  // every thread has read its partials before part[0] is overwritten
-      *reinterpret_cast<float4*>(&sm.part[0][u_t][u_j]) = u;
-      *reinterpret_cast<float4*>(rec + Workspace::kU + u_t * kV + col0 + u_j) = u;
+    {
+      const float4 s0 = *reinterpret_cast<const float4*>(&sm.s[s_i][s_j]);
+      float hs[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) hs[jj] = sm.ps[0][s_j + jj][s_i] + sm.ps[1][s_j + jj][s_i];
+      *reinterpret_cast<float4*>(&sm.s[s_i][s_j]) =
+          make_float4(fmaf(d, s0.x, hs[0]), fmaf(d, s0.y, hs[1]), fmaf(d, s0.z, hs[2]), fmaf(d, s0.w, hs[3]));
     }
-    __syncthreads();
-
-    // GEMM 2: S = D S + Kh^T U
-    float sn[2][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      const float d = b.dc[g2_i + a];
-      const float4 sv4 = *reinterpret_cast<const float4*>(&sm.s[g2_i + a][g2_j]);
-      sn[a][0] = d * sv4.x; sn[a][1] = d * sv4.y; sn[a][2] = d * sv4.z; sn[a][3] = d * sv4.w;
-    }
-#pragma unroll 8
-    for (int t = 0; t < kC; ++t) {
-      const float2 kh = *reinterpret_cast<const float2*>(&b.kh[t][g2_i]);
-      const float4 u = *reinterpret_cast<const float4*>(&sm.part[0][t][g2_j]);
-      const float kv[2] = {kh.x, kh.y}, uv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) sn[a][bb] = fmaf(kv[a], uv[bb], sn[a][bb]);
-    }
-    __syncthreads();  // every thread is done reading s and the buffer
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-      *reinterpret_cast<float4*>(&sm.s[g2_i + a][g2_j]) = make_float4(sn[a][0], sn[a][1], sn[a][2], sn[a][3]);
+    // The next iteration's prefetch refills this chunk's stage buffer, which no
+    // thread reads after the barrier above; its first barrier orders these
+    // writes of s before any read.
   }
   __syncthreads();
   for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {
@@ -633,51 +692,83 @@ __global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(cons
   if (warp == 0) tc::tmem_alloc(&sm.tmem, kOutTmemCols);
   if (tid == 0) tc::mbar_init(&sm.mbar, 1);
 
-  // ---- operand tiles: fp32 from the workspace, split to bf16 hi/lo
+  // ---- operand tiles: fp32 from the workspace, split to bf16 hi/lo.  Each
+  // phase issues all of a thread's (read-only) loads before any split or
+  // store, so the 144 KB a CTA reads are in flight together.
   const float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
-  // A1 = S0^T: item (value row j, key group of 8); loads are coalesced over j
-  for (int e = tid; e < kV * (kK / 8); e += kOutThreads) {
-    const int jj = e % kV, ig = e / kV;
-    float x[8];
+  {  // A1 = S0^T: items (value row j, key group of 8), loads coalesced over j
+    constexpr int kItems = kV * (kK / 8) / kOutThreads;  // 8
+    float x[kItems][8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) x[r] = rec[Workspace::kS0 + (ig * 8 + r) * kV + jj];
-    uint4 hi, lo;
-    tc::split8(x, hi, lo);
-    *reinterpret_cast<uint4*>(sm.a1h + tc::kmajor_off(jj, ig * 8, kK)) = hi;
-    *reinterpret_cast<uint4*>(sm.a1l + tc::kmajor_off(jj, ig * 8, kK)) = lo;
-  }
-  // B1 = Qt: item (token row t, key group of 8): one 32-byte read
-  for (int e = tid; e < kC * (kK / 8); e += kOutThreads) {
-    const int t = e / (kK / 8), ig = e % (kK / 8);
-    const float4 u0 = *reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8);
-    const float4 u1 = *reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8 + 4);
-    const float x[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    uint4 hi, lo;
-    tc::split8(x, hi, lo);
-    *reinterpret_cast<uint4*>(sm.b1h + tc::kmajor_off(t, ig * 8, kK)) = hi;
-    *reinterpret_cast<uint4*>(sm.b1l + tc::kmajor_off(t, ig * 8, kK)) = lo;
-  }
-  // A2 = U^T: item (value row j, token group of 8); loads coalesced over j
-  for (int e = tid; e < kV * (kC / 8); e += kOutThreads) {
-    const int jj = e % kV, sg = e / kV;
-    float x[8];
+    for (int it = 0; it < kItems; ++it) {
+      const int e = tid + it * kOutThreads, jj = e % kV, ig = e / kV;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) x[r] = rec[Workspace::kU + (sg * 8 + r) * kV + jj];
-    uint4 hi, lo;
-    tc::split8(x, hi, lo);
-    *reinterpret_cast<uint4*>(sm.a2h + tc::kmajor_off(jj, sg * 8, kC)) = hi;
-    *reinterpret_cast<uint4*>(sm.a2l + tc::kmajor_off(jj, sg * 8, kC)) = lo;
+      for (int r = 0; r < 8; ++r) x[it][r] = __ldg(rec + Workspace::kS0 + (ig * 8 + r) * kV + jj);
+    }
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int e = tid + it * kOutThreads, jj = e % kV, ig = e / kV;
+      uint4 hi, lo;
+      tc::split8(x[it], hi, lo);
+      *reinterpret_cast<uint4*>(sm.a1h + tc::kmajor_off(jj, ig * 8, kK)) = hi;
+      *reinterpret_cast<uint4*>(sm.a1l + tc::kmajor_off(jj, ig * 8, kK)) = lo;
+    }
   }
-  // B2 = P: item (token row t, token group of 8)
-  for (int e = tid; e < kC * (kC / 8); e += kOutThreads) {
-    const int t = e / (kC / 8), sg = e % (kC / 8);
-    const float4 u0 = *reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8);
-    const float4 u1 = *reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8 + 4);
-    const float x[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    uint4 hi, lo;
-    tc::split8(x, hi, lo);
-    *reinterpret_cast<uint4*>(sm.b2h + tc::kmajor_off(t, sg * 8, kC)) = hi;
-    *reinterpret_cast<uint4*>(sm.b2l + tc::kmajor_off(t, sg * 8, kC)) = lo;
+  {  // A2 = U^T (items (j, token group of 8)) and B2 = P (items (t, token group of 8))
+    constexpr int kItemsA = kV * (kC / 8) / kOutThreads;  // 4
+    constexpr int kItemsB = kC * (kC / 8) / kOutThreads;  // 2
+    float x[kItemsA][8];
+    float4 y[kItemsB][2];
+#pragma unroll
+    for (int it = 0; it < kItemsA; ++it) {
+      const int e = tid + it * kOutThreads, jj = e % kV, sg = e / kV;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) x[it][r] = __ldg(rec + Workspace::kU + (sg * 8 + r) * kV + jj);
+    }
+#pragma unroll
+    for (int it = 0; it < kItemsB; ++it) {
+      const int e = tid + it * kOutThreads, t = e / (kC / 8), sg = e % (kC / 8);
+      y[it][0] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8));
+      y[it][1] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8 + 4));
+    }
+#pragma unroll
+    for (int it = 0; it < kItemsA; ++it) {
+      const int e = tid + it * kOutThreads, jj = e % kV, sg = e / kV;
+      uint4 hi, lo;
+      tc::split8(x[it], hi, lo);
+      *reinterpret_cast<uint4*>(sm.a2h + tc::kmajor_off(jj, sg * 8, kC)) = hi;
+      *reinterpret_cast<uint4*>(sm.a2l + tc::kmajor_off(jj, sg * 8, kC)) = lo;
+    }
+#pragma unroll
+    for (int it = 0; it < kItemsB; ++it) {
+      const int e = tid + it * kOutThreads, t = e / (kC / 8), sg = e % (kC / 8);
+      const float v8[8] = {y[it][0].x, y[it][0].y, y[it][0].z, y[it][0].w,
+                           y[it][1].x, y[it][1].y, y[it][1].z, y[it][1].w};
+      uint4 hi, lo;
+      tc::split8(v8, hi, lo);
+      *reinterpret_cast<uint4*>(sm.b2h + tc::kmajor_off(t, sg * 8, kC)) = hi;
+      *reinterpret_cast<uint4*>(sm.b2l + tc::kmajor_off(t, sg * 8, kC)) = lo;
+    }
+  }
+  {  // B1 = Qt: items (token row t, key group of 8), one 32-byte read each
+    constexpr int kItems = kC * (kK / 8) / kOutThreads;  // 4
+    float4 y[kItems][2];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int e = tid + it * kOutThreads, t = e / (kK / 8), ig = e % (kK / 8);
+      y[it][0] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8));
+      y[it][1] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8 + 4));
+    }
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int e = tid + it * kOutThreads, t = e / (kK / 8), ig = e % (kK / 8);
+      const float v8[8] = {y[it][0].x, y[it][0].y, y[it][0].z, y[it][0].w,
+                           y[it][1].x, y[it][1].y, y[it][1].z, y[it][1].w};
+      uint4 hi, lo;
+      tc::split8(v8, hi, lo);
+      *reinterpret_cast<uint4*>(sm.b1h + tc::kmajor_off(t, ig * 8, kK)) = hi;
+      *reinterpret_cast<uint4*>(sm.b1l + tc::kmajor_off(t, ig * 8, kK)) = lo;
+    }
   }
   tc::fence_proxy_async();  // the tiles, written by threads, are read by the tensor cores
   tc::fence_before_sync();

@@ -44,7 +44,8 @@ def declared_functions():
 def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
-                                    "kda_decode_host", "kda_status_string", "kda_abi_version",
+                                    "kda_decode_host", "kda_decode_host_pipelined", "kda_status_string",
+                                    "kda_abi_version",
                                     "kda_prefill", "kda_prefill_workspace_bytes", "kda_prefill_no_alloc"}
 
 
@@ -65,7 +66,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 8):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 6
+    assert lib.kda_abi_version() == (1 << 16) | 7
 
 
 # ----------------------------------------------------------------- validation
@@ -264,6 +265,20 @@ def test_host_entry_point_validation(lib):
     assert call(hin=None, din=None, nbytes=0) == E.KDA_ERR_DEVICE  # nothing to copy in
     assert call(hout=None) == E.KDA_ERR_INVALID_ARG
     assert call(din=BASE + 5 * step - 64, nbytes=128) == E.KDA_ERR_ALIAS  # staging runs into the pool
+
+    # the pipelined form: two distinct streams and both events are required
+    s1, s2, ev1, ev2 = BASE + 30 * step, BASE + 31 * step, BASE + 32 * step, BASE + 33 * step
+
+    def pcall(st=s1, cs=s2, r=ev1, f=ev2, nbytes=4096):
+        return lib.kda_decode_host_pipelined(ctypes.byref(a), host_in, dev_in, nbytes, host_out, st, cs, r, f)
+
+    assert pcall(st=None) == E.KDA_ERR_INVALID_ARG
+    assert pcall(cs=None) == E.KDA_ERR_INVALID_ARG
+    assert pcall(cs=s1) == E.KDA_ERR_INVALID_ARG
+    assert pcall(r=None) == E.KDA_ERR_INVALID_ARG
+    assert pcall(f=None) == E.KDA_ERR_INVALID_ARG
+    assert pcall(nbytes=-1) == E.KDA_ERR_INVALID_ARG
+    assert pcall() == E.KDA_ERR_DEVICE                     # valid, no device here
 
 
 @no_gpu

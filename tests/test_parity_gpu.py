@@ -701,3 +701,64 @@ def test_general_shapes_strided_rows(T, gated, cuda_device):
     assert torch.equal(o1, o2) and torch.equal(d1.state, d2.state)
     before = w.to(cuda_device).state
     assert_parity(w, o2, d2.state, before)
+
+
+# ---------------------------------------------------------------------------
+# pipelined host steps (kda_decode_host_pipelined)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["n32_t1_hv8", "n32_t1_hv16_gated", "n8_t4_hv8"])
+def test_host_pipeline_equals_device_calls(name, cuda_device):
+    """Four steps through two alternating staging sets, copies in on a second
+    stream, equal four device calls on the same inputs bit for bit (outputs read
+    from pinned host memory, final state)."""
+    w = workloads.config(name)
+    steps_in = [workloads.config(name, seed=60 + i) for i in range(4)]
+    for x in steps_in:
+        x.slot_idx.copy_(w.slot_idx)
+    d_ref = w.to(cuda_device)
+    pool = d_ref.state.clone()
+    stream = torch.cuda.Stream(device=cuda_device)
+    copy_stream = torch.cuda.Stream(device=cuda_device)
+    sets = []
+    for _ in range(2):
+        inputs = {k: t for k, t in w.tensors().items() if k != "state"}
+        nbytes = sum((t.numel() * t.element_size() + 15) // 16 * 16 for t in inputs.values())
+        host_in = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        dev_in = torch.empty(nbytes, dtype=torch.uint8, device=cuda_device)
+        host_views, dev_views, off = {}, {}, 0
+        for k, t in inputs.items():
+            n = t.numel() * t.element_size()
+            host_views[k] = host_in[off:off + n].view(t.dtype).view(t.shape)
+            dev_views[k] = dev_in[off:off + n].view(t.dtype).view(t.shape)
+            off += (n + 15) // 16 * 16
+        out_d = torch.empty(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16, device=cuda_device)
+        host_out = torch.empty(out_d.shape, dtype=torch.bfloat16).pin_memory()
+        extra = dict(gate=dev_views["gate"], norm_weight=dev_views["norm_weight"], eps=w.eps) if w.gated else {}
+        step = kda.HostStep(dev_views["q"], dev_views["k"], dev_views["v"], pool, dev_views["slot_idx"],
+                            host_in=host_in, dev_in=dev_in, host_out=host_out, out=out_d, stream=stream,
+                            g=dev_views["g"], beta=dev_views["beta"], scale=w.scale, **extra)
+        sets.append((step, host_views, host_out))
+    pipe = kda.HostPipeline([s[0] for s in sets], copy_stream)
+    got = []
+    for i, x in enumerate(steps_in):
+        step, host_views, host_out = sets[i % 2]
+        if i >= 2:  # the set's previous output must be read before it is reused
+            stream.synchronize()
+            got.append(host_out.clone())
+        for k, t in x.tensors().items():
+            if k != "state":
+                host_views[k].copy_(t)
+        pipe()
+    stream.synchronize()
+    got += [sets[0][2].clone(), sets[1][2].clone()]
+    # reference: the same four steps as device calls
+    for i, x in enumerate(steps_in):
+        d = x.to(cuda_device)
+        if w.gated:
+            ref = kda.kda_decode_gated_rmsnorm(d.q, d.k, d.v, d.g, d.beta, d_ref.state, d.slot_idx, d.gate,
+                                               d.norm_weight, eps=w.eps, scale=w.scale)
+        else:
+            ref = kda.kda_decode(d.q, d.k, d.v, d.g, d.beta, d_ref.state, d.slot_idx, scale=w.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(got[i], ref.cpu()), f"step {i}: output differs"
+    assert torch.equal(pool, d_ref.state)
