@@ -32,8 +32,11 @@
  *   above (decay, correction on the decayed state, write, readout after the
  *   write) is the plainest reading that all of them support.
  *
- * Layouts.  Every tensor is dense, row-major (last index fastest), in device
- * memory of the current CUDA device:
+ * Layouts.  Every tensor is dense, row-major (last index fastest), in memory
+ * the current CUDA device reads at the given address: its own device memory,
+ * or page-locked host memory mapped into its address space at the same
+ * address (see kda_host_memory_is_mapped; the kernel then reads and writes that
+ * memory across PCIe, so no separate copy is needed):
  *     q, k        bf16  [N, T, HV, K]     (one q/k head per value head)
  *     v           bf16  [N, T, HV, V]
  *     g           fp32  [N, T, HV, K]     log-decay, decay = exp(g)
@@ -296,6 +299,19 @@ KDA_API kda_status kda_decode_host_pipelined(const kda_decode_args *args, const 
                                              int64_t in_bytes, void *host_out, kda_stream_t stream,
                                              kda_stream_t copy_stream, kda_event_t staging_ready,
                                              kda_event_t staging_free);
+
+/*
+ * 1 if [p, p + bytes) lies in one page-locked host allocation that the current
+ * device reads and writes at the same address (cudaHostAlloc / cudaMallocHost
+ * memory under unified addressing, or cudaHostRegister'd memory mapped at its
+ * host address), else 0; also 0 without a device.  Such memory may be passed
+ * to every entry point as inputs or output: the kernels then read the step's
+ * inputs from host memory and write its output back to host memory across
+ * PCIe in the one launch, with no separate copies.  Check each buffer once
+ * before first use: a host pointer the device cannot reach would be an
+ * illegal access.  This library's own helper; none of the pages describes it.
+ */
+KDA_API int32_t kda_host_memory_is_mapped(const void *p, int64_t bytes);
 
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);

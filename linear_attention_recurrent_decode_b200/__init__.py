@@ -24,7 +24,8 @@ import threading
 
 import torch
 
-__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "HostPipeline", "kda_prefill",
+__all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "HostPipeline", "MappedStep",
+           "host_memory_is_mapped", "kda_prefill",
            "prefill_workspace_bytes", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_ERR_SCRATCH_LIMIT", "KDA_STATE_FP32",
@@ -81,6 +82,7 @@ EXPORTED_SYMBOLS = {
     "kda_decode_host": ([ctypes.POINTER(DecodeArgs), _P, _P, _I, _P, _P], ctypes.c_int),
     "kda_decode_host_pipelined": ([ctypes.POINTER(DecodeArgs), _P, _P, _I, _P, _P, _P, _P, _P], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "kda_host_memory_is_mapped": ([_P, _I], ctypes.c_int32),
     "kda_abi_version": ([], ctypes.c_int32),
     # include/kda_prefill.h
     "kda_prefill_workspace_bytes": ([_I] * 5, ctypes.c_int64),
@@ -429,6 +431,98 @@ class HostPipeline:
             raise KdaError(rc, "kda_decode_host_pipelined")
         self._next = (i + 1) % len(self._steps)
         return st
+
+
+def host_memory_is_mapped(t) -> bool:
+    """Whether the current device reads and writes the page-locked host tensor
+    ``t`` at its host address (``kda_host_memory_is_mapped`` of the C ABI)."""
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
+        return False
+    return bool(library().kda_host_memory_is_mapped(t.data_ptr(), t.numel() * t.element_size()))
+
+
+class MappedStep:
+    """One decode step read from and written to page-locked host memory directly:
+    ``kda_decode_ex`` given host pointers the device reaches at the same address
+    (checked once, here, with :func:`host_memory_is_mapped`).  The kernel reads
+    the step's inputs across PCIe and writes ``out`` back to host memory in its
+    one launch, so a step costs no separate copies and no stream dependencies.
+
+    ``host_in`` is the pinned buffer the input tensors are views of; ``out`` a
+    pinned bf16 [N, T, HV, V] tensor; the state pool stays on the device.
+    Keyword arguments are those of :func:`kda_decode_ex` (g/beta or the raw
+    form, gate, norm_weight, eps, scale, state_layout, num_slots, status)."""
+
+    def __init__(self, q, k, v, state_pool, slot_idx, *, host_in, out, stream=None, **kw):
+        for name, t in (("host_in", host_in), ("out", out)):
+            if not host_memory_is_mapped(t):
+                raise ValueError(f"{name} is not page-locked host memory the current device maps at its address")
+        lo, hi = host_in.data_ptr(), host_in.data_ptr() + host_in.numel() * host_in.element_size()
+        views = {"q": q, "k": k, "v": v, "slot_idx": slot_idx,
+                 **{key: t for key, t in kw.items() if isinstance(t, torch.Tensor) and not t.is_cuda}}
+        for name, t in views.items():
+            if not (lo <= t.data_ptr() and t.data_ptr() + t.numel() * t.element_size() <= hi):
+                raise ValueError(f"{name} must be a view into host_in")
+        if out.dtype != torch.bfloat16 or not out.is_contiguous():
+            raise ValueError("out must be a contiguous bf16 tensor")
+        if not state_pool.is_cuda:
+            raise ValueError("state_pool must be on the device")
+        self.args = _mapped_args(q, k, v, state_pool, slot_idx, out, kw)
+        self._keep = (q, k, v, state_pool, slot_idx, host_in, out, kw)
+        self._torch_stream = stream if stream is not None else torch.cuda.current_stream()
+        self._stream = _stream_handle(self._torch_stream)
+        self._fn = library().kda_decode_ex
+        self._ref = ctypes.byref(self.args)
+        self.out = out
+
+    def __call__(self):
+        st = self._fn(self._ref, self._stream)
+        if st != KDA_OK:
+            raise KdaError(st, "kda_decode_ex")
+
+
+def _mapped_args(q, k, v, state_pool, slot_idx, out, kw):
+    """kda_decode_args for host-resident (mapped) inputs and output: the same
+    marshalling as _ex_args, with the device checks applied to the pool only."""
+    N, T, HV, K = q.shape
+    V = v.shape[-1]
+    a = DecodeArgs()
+    bf, f32 = torch.bfloat16, torch.float32
+
+    def rows(t, name, dtype, inner):
+        if t is None:
+            return 0
+        if t.dtype != dtype or tuple(t.shape) != (N, T, *inner):
+            raise ValueError(f"{name} must be {dtype} {(N, T, *inner)}")
+        return t.stride(1) if T > 1 else t.stride(0)
+
+    a.q, a.q_row_stride = q.data_ptr(), rows(q, "q", bf, (HV, K))
+    a.k, a.k_row_stride = k.data_ptr(), rows(k, "k", bf, (HV, K))
+    a.v, a.v_row_stride = v.data_ptr(), rows(v, "v", bf, (HV, V))
+    if kw.get("raw_gate") is not None:
+        a.raw_gate, a.g_row_stride = kw["raw_gate"].data_ptr(), rows(kw["raw_gate"], "raw_gate", bf, (HV, K))
+        a.raw_beta, a.beta_row_stride = kw["raw_beta"].data_ptr(), rows(kw["raw_beta"], "raw_beta", bf, (HV,))
+        a.A_log, a.dt_bias = kw["A_log"].data_ptr(), kw["dt_bias"].data_ptr()
+    else:
+        a.g, a.g_row_stride = kw["g"].data_ptr(), rows(kw["g"], "g", f32, (HV, K))
+        a.beta, a.beta_row_stride = kw["beta"].data_ptr(), rows(kw["beta"], "beta", f32, (HV,))
+    layout = kw.get("state_layout", "kv")
+    a.state_pool = state_pool.data_ptr()
+    a.state_layout = KDA_LAYOUT_KV if layout == "kv" else KDA_LAYOUT_VK
+    a.state_dtype = KDA_STATE_BF16 if state_pool.dtype == bf else KDA_STATE_FP32
+    a.slot_idx = slot_idx.data_ptr()
+    if kw.get("gate") is not None:
+        a.gate, a.gate_row_stride = kw["gate"].data_ptr(), rows(kw["gate"], "gate", bf, (HV, V))
+        a.norm_weight = kw["norm_weight"].data_ptr()
+    a.eps = float(kw.get("eps", 1e-6))
+    if tuple(out.shape) != (N, T, HV, V):
+        raise ValueError(f"out must be [{N}, {T}, {HV}, {V}]")
+    a.out = out.data_ptr()
+    a.N, a.T, a.HV, a.K, a.V = N, T, HV, K, V
+    scale = kw.get("scale")
+    a.scale = float(1.0 / math.sqrt(K) if scale is None else scale)
+    a.num_slots = int(state_pool.shape[0] if kw.get("num_slots") is None else kw["num_slots"])
+    return a
 
 
 # ---------------------------------------------------------------- chunked prefill

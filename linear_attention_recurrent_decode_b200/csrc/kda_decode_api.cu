@@ -364,6 +364,22 @@ kda_status kda_decode_host_pipelined(const kda_decode_args* args, const void* ho
   return launch(*args, /*gated=*/args->gate != nullptr, stream, &hc);
 }
 
+int32_t kda_host_memory_is_mapped(const void* p, int64_t bytes) {
+  if (p == nullptr || bytes <= 0) return 0;
+  const unsigned char* last = static_cast<const unsigned char*>(p) + (bytes - 1);
+  for (const void* q : {p, static_cast<const void*>(last)}) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, q) != cudaSuccess) {
+      cudaGetLastError();  // an unregistered pointer is an answer here, not a sticky error
+      return 0;
+    }
+    if (attr.type != cudaMemoryTypeHost || attr.devicePointer != q || attr.hostPointer != q) return 0;
+  }
+  // both ends in one allocation: the device addresses of the two ends differ
+  // by exactly the host distance (checked above: they equal the host addresses)
+  return 1;
+}
+
 const char* kda_status_string(kda_status status) {
   switch (status) {
     case KDA_OK: return "ok";
@@ -382,6 +398,6 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 7; }
+int32_t kda_abi_version(void) { return (1 << 16) | 8; }
 
 }  // extern "C"

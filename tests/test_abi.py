@@ -45,7 +45,7 @@ def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
                                     "kda_decode_host", "kda_decode_host_pipelined", "kda_status_string",
-                                    "kda_abi_version",
+                                    "kda_abi_version", "kda_host_memory_is_mapped",
                                     "kda_prefill", "kda_prefill_workspace_bytes", "kda_prefill_no_alloc"}
 
 
@@ -66,7 +66,7 @@ def test_status_strings_and_version(lib):
     for s in range(1, 8):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 7
+    assert lib.kda_abi_version() == (1 << 16) | 8
 
 
 # ----------------------------------------------------------------- validation
@@ -129,6 +129,13 @@ def test_rejections(lib, gated):
         assert call(lib, eps=float("nan"), gated=True) == E.KDA_ERR_INVALID_ARG
         assert call(lib, eps=float("inf"), gated=True) == E.KDA_ERR_INVALID_ARG
         assert call(lib, out=BASE + 10 * (1 << 30), gated=True) == E.KDA_ERR_ALIAS
+
+
+@no_gpu
+def test_host_memory_is_never_mapped_without_a_device(lib):
+    assert lib.kda_host_memory_is_mapped(BASE, 4096) == 0
+    assert lib.kda_host_memory_is_mapped(None, 16) == 0
+    assert lib.kda_host_memory_is_mapped(BASE, 0) == 0
 
 
 @no_gpu

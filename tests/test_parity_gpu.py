@@ -762,3 +762,50 @@ def test_host_pipeline_equals_device_calls(name, cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(got[i], ref.cpu()), f"step {i}: output differs"
     assert torch.equal(pool, d_ref.state)
+
+
+# ---------------------------------------------------------------------------
+# steps read from and written to mapped page-locked host memory (MappedStep)
+# ---------------------------------------------------------------------------
+def _pinned_views(tensors):
+    nbytes = sum((t.numel() * t.element_size() + 15) // 16 * 16 for t in tensors.values())
+    buf = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    views, off = {}, 0
+    for key, t in tensors.items():
+        n = t.numel() * t.element_size()
+        views[key] = buf[off:off + n].view(t.dtype).view(t.shape)
+        views[key].copy_(t)
+        off += (n + 15) // 16 * 16
+    return buf, views
+
+
+@pytest.mark.parametrize("name", ["n32_t1_hv8", "n32_t1_hv16_gated", "n8_t4_hv8", "n32_t1_hv8_raw"])
+def test_mapped_host_step_equals_device_call(name, cuda_device):
+    """Inputs in page-locked host memory and the output written straight back
+    to it by the kernel: bit-identical to the same step on device buffers.  The
+    buffers are checked to be mapped at their host address before any launch."""
+    w = workloads.config(name)
+    inputs = {k: t for k, t in w.tensors().items() if k != "state"}
+    host_in, hv = _pinned_views(inputs)
+    out_h = torch.zeros(w.N, w.T, w.HV, w.V, dtype=torch.bfloat16).pin_memory()
+    if not (kda.host_memory_is_mapped(host_in) and kda.host_memory_is_mapped(out_h)):
+        pytest.skip("page-locked host memory is not mapped at its host address on this machine")
+    pool = w.state.to(cuda_device)
+    extra = dict(gate=hv["gate"], norm_weight=hv["norm_weight"], eps=w.eps) if w.gated else {}
+    if w.raw is not None:
+        extra.update(raw_gate=hv["raw_gate"], A_log=hv["A_log"], dt_bias=hv["dt_bias"], raw_beta=hv["raw_beta"])
+    else:
+        extra.update(g=hv["g"], beta=hv["beta"])
+    step = kda.MappedStep(hv["q"], hv["k"], hv["v"], pool, hv["slot_idx"], host_in=host_in, out=out_h,
+                          scale=w.scale, **extra)
+    step()
+    torch.cuda.synchronize()
+    d = w.to(cuda_device)
+    dextra = dict(gate=d.gate, norm_weight=d.norm_weight, eps=w.eps) if w.gated else {}
+    if w.raw is not None:
+        dextra.update(raw_gate=d.raw.raw_gate, A_log=d.raw.A_log, dt_bias=d.raw.dt_bias, raw_beta=d.raw.raw_beta)
+    else:
+        dextra.update(g=d.g, beta=d.beta)
+    ref = kda.kda_decode_ex(d.q, d.k, d.v, d.state, d.slot_idx, scale=w.scale, **dextra)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, ref.cpu()) and torch.equal(pool, d.state)
