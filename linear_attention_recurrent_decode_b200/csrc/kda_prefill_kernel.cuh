@@ -351,40 +351,57 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   __syncthreads();
 
   // ---- 4. forward substitution: X[t] = beta_t R[t] - sum_{s<t} L[t][s] X[s],
-  // R = [Kt | V]; thread j owns column j (j < K: W, else Ut).
+  // R = [Kt | V]; thread j owns column j (j < K: W, else Ut).  Blocks of 16
+  // tokens: the earlier blocks' contribution is a small product over solved
+  // rows kept in shared memory (rolled over the blocks), the in-block
+  // triangle is unrolled; the same arithmetic as a row-by-row solve with a
+  // quarter of the code (the kernel was stalling on instruction fetch).
   {
+    constexpr int kB = 16;                                   // tokens per block
+    constexpr int kCols = kK + kV;                           // solve columns
     const int j = tid;
     const float* const vf = reinterpret_cast<const float*>(&sm.gam[0][0]);
-    // x kept as pairs for packed fp32x2 FMAs; two pair accumulators (four
-    // partial sums) per row keep the dependent chain short
-    float2 x2[kC / 2];
+    float* const X = &sm.at[0][0];                           // [kC][kCols] solved rows (the factors are dead)
+    static_assert(kC * kCols <= 3 * kK * kCP, "solved rows fit over the factor buffers");
+    for (int b = 0; b < kC / kB; ++b) {
+      const int t0b = b * kB;
+      float xb[kB];
 #pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+      for (int t = 0; t < kB; ++t)
+        xb[t] = sm.beta[t0b + t] * (j < kK ? sm.kt[t0b + t][j] : vf[(t0b + t) * kV + (j - kK)]);
+      for (int pb = 0; pb < b; ++pb) {  // earlier blocks
+        const int s0 = pb * kB;
+        float2 xs[kB / 2];
 #pragma unroll
-      for (int s = 0; s + 3 < t; s += 4) {
-        const float4 l = *reinterpret_cast<const float4*>(&sm.L[t][s]);
-        a01 = __ffma2_rn(make_float2(-l.x, -l.y), x2[s / 2], a01);
-        a23 = __ffma2_rn(make_float2(-l.z, -l.w), x2[s / 2 + 1], a23);
+        for (int u = 0; u < kB / 2; ++u) xs[u] = make_float2(X[(s0 + 2 * u) * kCols + j], X[(s0 + 2 * u + 1) * kCols + j]);
+#pragma unroll
+        for (int t = 0; t < kB; ++t) {
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int q4 = 0; q4 < kB / 4; ++q4) {
+            const float4 l = *reinterpret_cast<const float4*>(&sm.L[t0b + t][s0 + 4 * q4]);
+            acc = __ffma2_rn(make_float2(l.x, l.y), xs[2 * q4], acc);
+            acc = __ffma2_rn(make_float2(l.z, l.w), xs[2 * q4 + 1], acc);
+          }
+          xb[t] -= acc.x + acc.y;
+        }
       }
-      float a = sm.beta[t] * (j < kK ? sm.kt[t][j] : vf[t * kV + (j - kK)]);
 #pragma unroll
-      for (int s = t & ~3; s < t; ++s) a = fmaf(-sm.L[t][s], (s & 1) ? x2[s / 2].y : x2[s / 2].x, a);
-      const float xt = a + ((a01.x + a01.y) + (a23.x + a23.y));
-      if (t & 1) x2[t / 2].y = xt;
-      else x2[t / 2].x = xt;
-    }
-    float x[kC];
+      for (int t = 1; t < kB; ++t) {  // in-block triangle
 #pragma unroll
-    for (int t = 0; t < kC; ++t) x[t] = (t & 1) ? x2[t / 2].y : x2[t / 2].x;
-    if (j < kK) {
-      float* const wt = rec + Workspace::kWt + j * kC;  // W^T row j
+        for (int s2 = 0; s2 < t; ++s2) xb[t] = fmaf(-sm.L[t0b + t][t0b + s2], xb[s2], xb[t]);
+      }
 #pragma unroll
-      for (int t = 0; t < kC; t += 4) *reinterpret_cast<float4*>(wt + t) = make_float4(x[t], x[t + 1], x[t + 2], x[t + 3]);
-    } else {
-      float* const ut = rec + Workspace::kUt + (j - kK);
+      for (int t = 0; t < kB; ++t) X[(t0b + t) * kCols + j] = xb[t];
+      if (j < kK) {
+        float* const wt = rec + Workspace::kWt + j * kC + t0b;  // W^T row j
 #pragma unroll
-      for (int t = 0; t < kC; ++t) ut[t * kV] = x[t];
+        for (int t = 0; t < kB; t += 4) *reinterpret_cast<float4*>(wt + t) = make_float4(xb[t], xb[t + 1], xb[t + 2], xb[t + 3]);
+      } else {
+        float* const ut = rec + Workspace::kUt + (j - kK);
+#pragma unroll
+        for (int t = 0; t < kB; ++t) ut[(t0b + t) * kV] = xb[t];
+      }
     }
   }
 }

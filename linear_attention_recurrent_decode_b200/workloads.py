@@ -193,6 +193,9 @@ CONFIGS = {
     "n32_t1_hv8_vk": dict(N=32, T=1, HV=8, num_slots=64, state_layout="vk"),
     "n32_t1_hv8_bf16state_vk": dict(N=32, T=1, HV=8, num_slots=64, state_dtype="bf16", state_layout="vk"),
     "n32_t4_hv8_vk": dict(N=32, T=4, HV=8, num_slots=64, state_layout="vk"),
+    # general shapes: K outside {64, 128, 256}, V not a multiple of 32 (masked form)
+    "n32_t1_hv8_k192_v130": dict(N=32, T=1, HV=8, K=192, V=130, num_slots=64),
+    "n32_t4_hv8_k96_v100": dict(N=32, T=4, HV=8, K=96, V=100, num_slots=64),
 }
 
 
@@ -212,7 +215,7 @@ PREFILL_CONFIGS = {
 
 
 def config(name: str, seed: int = 0) -> Workload:
-    """One of the named workloads (K = V = 128), drawn with ``seed``."""
+    """One of the named workloads (K = V = 128 unless the name says), drawn with ``seed``."""
     kw = CONFIGS[name] if name in CONFIGS else PREFILL_CONFIGS[name]
     return make(name=name, seed=seed, **kw)
 

@@ -76,6 +76,7 @@ def assert_parity(w, o_gpu, pool_gpu, pool_before, rows=None):
 
 
 SMALL_CONFIGS = ["n1_t1_hv8", "n32_t1_hv8", "n32_t1_hv16_gated", "n1_t4_hv8", "n8_t4_hv8", "n32_t4_hv8",
+                 "n32_t1_hv8_k192_v130", "n32_t4_hv8_k96_v100",
                  "n32_t1_hv8_bf16state", "n32_t1_hv16_gated_bf16state", "n32_t4_hv8_bf16state"]
 
 
