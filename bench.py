@@ -446,7 +446,7 @@ def run_ours(args):
                          "Python (no CUDA graph)"},
         "clocks": clocks,
         "floor": floor,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (3 if args.config.startswith("prefill_") else 1),
         "wall_s_timed": round(t_wall, 3),
     }
     print(json.dumps(line), flush=True)

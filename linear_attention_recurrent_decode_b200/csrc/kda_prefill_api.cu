@@ -33,13 +33,32 @@ cudaError_t prepare_kernels() {
   cudaError_t e = cudaFuncSetAttribute(kp::kda_prefill_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kp::kChunkSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kp::kStateSmem);
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<8>);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<16>);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<32>);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kp::kda_prefill_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kp::kOutSmem);
   if (e == cudaSuccess && bit) ready.fetch_or(bit, std::memory_order_relaxed);
   return e;
+}
+
+// The current device's SM count, once per device.
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int v = dev < kMaxDevices ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    if (dev < kMaxDevices) cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
 }
 
 }  // namespace
@@ -67,7 +86,7 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
   if (!workspace_floats(N, T, HV, &nchunks, &floats) || !mul_ok(N, T, &rows) || !mul_ok(HV, K, &hk) ||
       !mul_ok(HV, V, &hv_v) || !mul_ok(rows, hv_v, &out_elems) || out_elems > INT64_MAX / 8 ||
       !mul_ok(N * HV, nchunks, &grid_chunks) || grid_chunks > 0x7fffffffLL ||
-      !mul_ok(N * HV, kp::kV / kp::kBV, &grid_state) || grid_state > 0x7fffffffLL || floats > INT64_MAX / 4 ||
+      !mul_ok(N * HV, kp::kV / 8, &grid_state) || grid_state > 0x7fffffffLL || floats > INT64_MAX / 4 ||
       nchunks > 0x7fffffffLL)
     return KDA_ERR_UNSUPPORTED;
 
@@ -117,9 +136,15 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     return cudaLaunchKernelEx(&cfg, kernel, p);
   };
-  if (run(kp::kda_prefill_chunk_kernel, grid_chunks, kp::kChunkThreads, kp::kChunkSmem) != cudaSuccess ||
-      run(kp::kda_prefill_state_kernel, grid_state, kp::kStateThreads, kp::kStateSmem) != cudaSuccess ||
-      run(kp::kda_prefill_output_kernel, grid_chunks, kp::kOutThreads, kp::kOutSmem) != cudaSuccess)
+  const int bv = kp::state_tile_width(N * HV, sm_count());
+  const int64_t grid_tiles = N * HV * (kp::kV / bv);
+  cudaError_t e_state = cudaSuccess;
+  if (run(kp::kda_prefill_chunk_kernel, grid_chunks, kp::kChunkThreads, kp::kChunkSmem) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (bv == 8) e_state = run(kp::kda_prefill_state_kernel<8>, grid_tiles, kp::kStateThreads, kp::kStateSmem<8>);
+  else if (bv == 16) e_state = run(kp::kda_prefill_state_kernel<16>, grid_tiles, kp::kStateThreads, kp::kStateSmem<16>);
+  else e_state = run(kp::kda_prefill_state_kernel<32>, grid_tiles, kp::kStateThreads, kp::kStateSmem<32>);
+  if (e_state != cudaSuccess || run(kp::kda_prefill_output_kernel, grid_chunks, kp::kOutThreads, kp::kOutSmem) != cudaSuccess)
     return KDA_ERR_CUDA;
   return KDA_OK;
 }

@@ -27,7 +27,7 @@
 //   1. kda_prefill_chunk_kernel (one CTA per (n, h, chunk), all chunks at
 //      once): Gamma in fp64, the decay factors, M and P, the substitution for
 //      W and Ut; writes them to the workspace.
-//   2. kda_prefill_state_kernel (one CTA per (n, h, 8-column value tile),
+//   2. kda_prefill_state_kernel (one CTA per (n, h, 8/16/32-column value tile),
 //      chunks in order): the state chain U = Ut - W S0, S_C = D S0 + Kh^T U,
 //      keeping S in shared memory; writes each chunk's start state and U to the
 //      workspace and the final state back to the pool slot.
@@ -56,7 +56,6 @@ namespace kdap {
 constexpr int kC = 64;        // tokens per chunk
 constexpr int kK = 128;       // key dimension (the kernels are written for K = V = 128)
 constexpr int kV = 128;       // value dimension
-constexpr int kBV = 8;        // value columns per state-chain CTA
 constexpr float kSafeExp = 80.f;  // |Gamma_t - Gamma_r| bound of the factored path
 
 struct Params {
@@ -407,35 +406,51 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
 }
 
 // ---------------------------------------------------------------- kernel 2
-// One CTA per (n, h, 8-column value tile) walks the chunks in order with its
-// K x 8 state tile in shared memory; the next chunk's W^T, Kh, Ut and exp(Gamma_C)
-// are staged with cp.async while the current one is processed.  Both products
-// split their reduction over the CTA (W S over quarters of K, Kh^T U over halves
-// of the chunk), use packed fp32x2 FMAs, and sum the partials in a fixed order.
+// One CTA per (n, h, BV-column value tile) walks the chunks in order with its
+// K x BV state tile in shared memory; the next chunk's W^T, Kh, Ut and
+// exp(Gamma_C) are staged with cp.async while the current one is processed.
+// Both products split their reduction over the CTA (W S over quarters of K,
+// Kh^T U over halves of the chunk for narrow tiles), use packed fp32x2 FMAs,
+// and sum the partials in a fixed order.  Every CTA reads the chunk's 64 KB
+// of W^T and Kh whatever its width, so the launch takes the widest tile that
+// still keeps one CTA on every SM it can: BV = 8 for a few heads (one 8192-
+// token prompt at 8 heads: 128 CTAs), 16 or 32 for batches of prompts.
 constexpr int kStateThreads = 256;
 constexpr int kCU = kC + 4;  // padded rows of the transposed partial buffers
 
-struct StateBuf {
-  float wt[kK][kC];   // W^T
-  float kh[kC][kK];   // Kh
-  float ut[kC][kBV];  // this tile's columns of Ut
-  float dc[kK];       // exp(Gamma_C)
-};
-struct StateSmem {
-  StateBuf buf[2];
-  float s[kK][kBV];             // state tile
-  float pw[4][kBV][kCU];        // (W S) partial sums per quarter of K, [j][t]
-  float u[kC][kBV + 2];         // U of the current chunk, [t][j] (rows padded to 10 floats)
-  float ps[2][kBV][kK + 4];      // (Kh^T U) partial sums per half of the chunk, [j][i]
+template <int BV>
+struct StateCfg {
+  static_assert(BV == 8 || BV == 16 || BV == 32, "value tile of 8, 16 or 32 columns");
+  static constexpr int kJW = BV / 4;                 // W S: columns per thread (4 column groups)
+  static constexpr int kCS = BV == 32 ? 1 : 2;       // Kh^T U: splits of the chunk
+  static constexpr int kJW2 = BV == 8 ? 4 : 8;       // Kh^T U: columns per thread
+  static constexpr int kNG2 = BV / kJW2;             // Kh^T U: column groups
+  static_assert(64 * kNG2 * kCS == kStateThreads, "Kh^T U covers the tile once");
+  static constexpr int kUW = BV / 4;                 // U: columns per thread
+  static constexpr int kSW = BV / 2;                 // S update: columns per thread
+  struct Buf {
+    float wt[kK][kC];   // W^T
+    float kh[kC][kK];   // Kh
+    float ut[kC][BV];   // this tile's columns of Ut
+    float dc[kK];       // exp(Gamma_C)
+  };
+  struct Smem {
+    Buf buf[2];
+    float s[kK][BV];              // state tile
+    float pw[4][BV][kCU];         // (W S) partial sums per quarter of K, [j][t]
+    float u[kC][BV + 4];          // U of the current chunk, [t][j]
+    float ps[kCS][BV][kK + 4];    // (Kh^T U) partial sums per split of the chunk, [j][i]
+  };
 };
 
-__device__ __forceinline__ void stage_chunk(StateBuf& b, const float* rec, int col0, int tid) {
+template <int BV>
+__device__ __forceinline__ void stage_chunk(typename StateCfg<BV>::Buf& b, const float* rec, int col0, int tid) {
   for (int c = tid; c < (kK * kC) / 4; c += kStateThreads) {
     cp_async16(&b.wt[0][0] + 4 * c, rec + Workspace::kWt + 4 * c);
     cp_async16(&b.kh[0][0] + 4 * c, rec + Workspace::kKh + 4 * c);
   }
-  for (int c = tid; c < kC * (kBV / 4); c += kStateThreads) {
-    const int t = c / (kBV / 4), pc = c % (kBV / 4);
+  for (int c = tid; c < kC * (BV / 4); c += kStateThreads) {
+    const int t = c / (BV / 4), pc = c % (BV / 4);
     cp_async16(&b.ut[t][pc * 4], rec + Workspace::kUt + t * kV + col0 + pc * 4);
   }
   for (int c = tid; c < kK / 4; c += kStateThreads) cp_async16(&b.dc[4 * c], rec + Workspace::kDc + 4 * c);
@@ -444,115 +459,146 @@ __device__ __forceinline__ void stage_chunk(StateBuf& b, const float* rec, int c
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 splat(float x) { return make_float2(x, x); }
 
+template <int BV>
 __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(const Params p) {
+  using Cfg = StateCfg<BV>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  StateSmem& sm = *reinterpret_cast<StateSmem*>(smem_raw);
-  constexpr int kTiles = kV / kBV;
+  typename Cfg::Smem& sm = *reinterpret_cast<typename Cfg::Smem*>(smem_raw);
+  constexpr int kTiles = kV / BV;
   const int tid = threadIdx.x;
   const int64_t unit = blockIdx.x / kTiles;
   const int tile = static_cast<int>(blockIdx.x - unit * kTiles);
-  const int col0 = tile * kBV;
+  const int col0 = tile * BV;
   const int64_t n = unit / p.HV;
   const int64_t h = unit - n * p.HV;
   const int32_t slot = __ldg(p.slot_idx + n);
   if (slot < 0) return;
 
   float* const blk = p.state + (static_cast<int64_t>(slot) * p.HV + h) * kK * kV;
-  for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {  // initial state tile
-    const int i = c / (kBV / 4), pc = c % (kBV / 4);
+  for (int c = tid; c < kK * (BV / 4); c += kStateThreads) {  // initial state tile
+    const int i = c / (BV / 4), pc = c % (BV / 4);
     cp_async16(&sm.s[i][pc * 4], blk + i * kV + col0 + pc * 4);
   }
-  stage_chunk(sm.buf[0], p.ws + Workspace::record(unit, 0, p.nchunks), col0, tid);
+  stage_chunk<BV>(sm.buf[0], p.ws + Workspace::record(unit, 0, p.nchunks), col0, tid);
   cp_async_commit();
 
-  // W S: thread (quarter of K, 4 tokens, 2 columns)
-  const int a_t = (tid % 16) * 4, a_j = ((tid / 16) % 4) * 2, a_q = tid / 64;
-  // U: thread (token, column pair)
-  const int u_t = tid % 64, u_j = (tid / 64) * 2;
-  // Kh^T U: thread (2 key rows, 4 columns, half of the chunk)
-  const int b_i = (tid % 64) * 2, b_j = ((tid / 64) % 2) * 4, b_h = tid / 128;
+  // W S: thread (quarter of K, 4 tokens, kJW columns)
+  const int a_t = (tid % 16) * 4, a_j = ((tid / 16) % 4) * Cfg::kJW, a_q = tid / 64;
+  // U: thread (token, kUW columns)
+  const int u_t = tid % 64, u_j = (tid / 64) * Cfg::kUW;
+  // Kh^T U: thread (2 key rows, kJW2 columns, split of the chunk)
+  const int b_i = (tid % 64) * 2, b_j = ((tid / 64) % Cfg::kNG2) * Cfg::kJW2, b_h = tid / (64 * Cfg::kNG2);
+  // S update: thread (key row, kSW columns)
+  const int s_i = tid / 2, s_j = (tid % 2) * Cfg::kSW;
 
   for (int32_t c = 0; c < p.nchunks; ++c) {
     const int cb = c & 1;
     if (c + 1 < p.nchunks) {
-      stage_chunk(sm.buf[cb ^ 1], p.ws + Workspace::record(unit, c + 1, p.nchunks), col0, tid);
+      stage_chunk<BV>(sm.buf[cb ^ 1], p.ws + Workspace::record(unit, c + 1, p.nchunks), col0, tid);
       cp_async_commit();
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();
-    const StateBuf& b = sm.buf[cb];
+    const typename Cfg::Buf& b = sm.buf[cb];
     float* const rec = p.ws + Workspace::record(unit, c, p.nchunks);
 
     // chunk-start state to the workspace (the output kernel reads it)
-    for (int e = tid; e < kK * (kBV / 4); e += kStateThreads) {
-      const int i = e / (kBV / 4), pc = e % (kBV / 4);
+    for (int e = tid; e < kK * (BV / 4); e += kStateThreads) {
+      const int i = e / (BV / 4), pc = e % (BV / 4);
       *reinterpret_cast<float4*>(rec + Workspace::kS0 + i * kV + col0 + pc * 4) =
           *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
     }
 
     {  // W S over one quarter of K
-      float2 acc[4] = {splat(0.f), splat(0.f), splat(0.f), splat(0.f)};
+      float2 acc[4][Cfg::kJW / 2];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int jj = 0; jj < Cfg::kJW / 2; ++jj) acc[a][jj] = splat(0.f);
       const int i_lo = a_q * (kK / 4);
-#pragma unroll 8
+#pragma unroll 4
       for (int i = i_lo; i < i_lo + kK / 4; ++i) {
         const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][a_t]);
-        const float2 sv = *reinterpret_cast<const float2*>(&sm.s[i][a_j]);
-        acc[0] = ffma2(splat(w.x), sv, acc[0]);
-        acc[1] = ffma2(splat(w.y), sv, acc[1]);
-        acc[2] = ffma2(splat(w.z), sv, acc[2]);
-        acc[3] = ffma2(splat(w.w), sv, acc[3]);
+        float2 sv[Cfg::kJW / 2];
+#pragma unroll
+        for (int jj = 0; jj < Cfg::kJW / 2; ++jj) sv[jj] = *reinterpret_cast<const float2*>(&sm.s[i][a_j + 2 * jj]);
+        const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int jj = 0; jj < Cfg::kJW / 2; ++jj) acc[a][jj] = ffma2(splat(wv[a]), sv[jj], acc[a][jj]);
       }
-      *reinterpret_cast<float4*>(&sm.pw[a_q][a_j][a_t]) = make_float4(acc[0].x, acc[1].x, acc[2].x, acc[3].x);
-      *reinterpret_cast<float4*>(&sm.pw[a_q][a_j + 1][a_t]) = make_float4(acc[0].y, acc[1].y, acc[2].y, acc[3].y);
+#pragma unroll
+      for (int jj = 0; jj < Cfg::kJW / 2; ++jj) {
+        *reinterpret_cast<float4*>(&sm.pw[a_q][a_j + 2 * jj][a_t]) =
+            make_float4(acc[0][jj].x, acc[1][jj].x, acc[2][jj].x, acc[3][jj].x);
+        *reinterpret_cast<float4*>(&sm.pw[a_q][a_j + 2 * jj + 1][a_t]) =
+            make_float4(acc[0][jj].y, acc[1][jj].y, acc[2][jj].y, acc[3][jj].y);
+      }
     }
     __syncthreads();
     {  // U = Ut - W S, the quarters summed in a fixed order
-      float uo[2];
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
+      for (int jj = 0; jj < Cfg::kUW; ++jj) {
         const int j = u_j + jj;
         const float ws = (sm.pw[0][j][u_t] + sm.pw[1][j][u_t]) + (sm.pw[2][j][u_t] + sm.pw[3][j][u_t]);
-        uo[jj] = b.ut[u_t][j] - ws;
+        const float uo = b.ut[u_t][j] - ws;
+        sm.u[u_t][j] = uo;
+        rec[Workspace::kU + u_t * kV + col0 + j] = uo;
       }
-      *reinterpret_cast<float2*>(&sm.u[u_t][u_j]) = make_float2(uo[0], uo[1]);
-      *reinterpret_cast<float2*>(rec + Workspace::kU + u_t * kV + col0 + u_j) = make_float2(uo[0], uo[1]);
     }
     __syncthreads();
-    {  // Kh^T U over one half of the chunk
-      float2 acc[2][2] = {{splat(0.f), splat(0.f)}, {splat(0.f), splat(0.f)}};
-      const int t_lo = b_h * (kC / 2);
-#pragma unroll 8
-      for (int t = t_lo; t < t_lo + kC / 2; ++t) {
+    {  // Kh^T U over one split of the chunk
+      float2 acc[2][Cfg::kJW2 / 2];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int jj = 0; jj < Cfg::kJW2 / 2; ++jj) acc[a][jj] = splat(0.f);
+      const int t_lo = b_h * (kC / Cfg::kCS);
+#pragma unroll 4
+      for (int t = t_lo; t < t_lo + kC / Cfg::kCS; ++t) {
         const float2 kh = *reinterpret_cast<const float2*>(&b.kh[t][b_i]);
-        const float2 u0 = *reinterpret_cast<const float2*>(&sm.u[t][b_j]);
-        const float2 u1 = *reinterpret_cast<const float2*>(&sm.u[t][b_j + 2]);
-        acc[0][0] = ffma2(splat(kh.x), u0, acc[0][0]);
-        acc[0][1] = ffma2(splat(kh.x), u1, acc[0][1]);
-        acc[1][0] = ffma2(splat(kh.y), u0, acc[1][0]);
-        acc[1][1] = ffma2(splat(kh.y), u1, acc[1][1]);
+        float2 uv[Cfg::kJW2 / 2];
+#pragma unroll
+        for (int q4 = 0; q4 < Cfg::kJW2 / 4; ++q4) {
+          const float4 x = *reinterpret_cast<const float4*>(&sm.u[t][b_j + 4 * q4]);
+          uv[2 * q4] = make_float2(x.x, x.y);
+          uv[2 * q4 + 1] = make_float2(x.z, x.w);
+        }
+#pragma unroll
+        for (int jj = 0; jj < Cfg::kJW2 / 2; ++jj) {
+          acc[0][jj] = ffma2(splat(kh.x), uv[jj], acc[0][jj]);
+          acc[1][jj] = ffma2(splat(kh.y), uv[jj], acc[1][jj]);
+        }
       }
 #pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        sm.ps[b_h][b_j][b_i + a] = acc[a][0].x;
-        sm.ps[b_h][b_j + 1][b_i + a] = acc[a][0].y;
-        sm.ps[b_h][b_j + 2][b_i + a] = acc[a][1].x;
-        sm.ps[b_h][b_j + 3][b_i + a] = acc[a][1].y;
-      }
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int jj = 0; jj < Cfg::kJW2 / 2; ++jj) {
+          sm.ps[b_h][b_j + 2 * jj][b_i + a] = acc[a][jj].x;
+          sm.ps[b_h][b_j + 2 * jj + 1][b_i + a] = acc[a][jj].y;
+        }
     }
-    // S = D S + Kh^T U: thread (key row, 4 columns).  The decay is read before
-    // the barrier: after it no thread touches this chunk's stage buffer, which
-    // the next iteration's prefetch then refills.
-    const int s_i = tid / 2, s_j = (tid % 2) * 4;
+    // S = D S + Kh^T U.  The decay is read before the barrier: after it no
+    // thread touches this chunk's stage buffer, which the next iteration's
+    // prefetch then refills.
     const float d = b.dc[s_i];
     __syncthreads();
-    {
-      const float4 s0 = *reinterpret_cast<const float4*>(&sm.s[s_i][s_j]);
+#pragma unroll
+    for (int q4 = 0; q4 < Cfg::kSW / 4; ++q4) {
+      const int j = s_j + 4 * q4;
+      const float4 s0 = *reinterpret_cast<const float4*>(&sm.s[s_i][j]);
       float hs[4];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) hs[jj] = sm.ps[0][s_j + jj][s_i] + sm.ps[1][s_j + jj][s_i];
-      *reinterpret_cast<float4*>(&sm.s[s_i][s_j]) =
+      for (int jj = 0; jj < 4; ++jj) {
+        float acc = sm.ps[0][j + jj][s_i];
+#pragma unroll
+        for (int cs = 1; cs < Cfg::kCS; ++cs) acc += sm.ps[cs][j + jj][s_i];
+        hs[jj] = acc;
+      }
+      *reinterpret_cast<float4*>(&sm.s[s_i][j]) =
           make_float4(fmaf(d, s0.x, hs[0]), fmaf(d, s0.y, hs[1]), fmaf(d, s0.z, hs[2]), fmaf(d, s0.w, hs[3]));
     }
     // The next iteration's prefetch refills this chunk's stage buffer, which no
@@ -560,11 +606,20 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
     // writes of s before any read.
   }
   __syncthreads();
-  for (int c = tid; c < kK * (kBV / 4); c += kStateThreads) {
-    const int i = c / (kBV / 4), pc = c % (kBV / 4);
+  for (int c = tid; c < kK * (BV / 4); c += kStateThreads) {
+    const int i = c / (BV / 4), pc = c % (BV / 4);
     *reinterpret_cast<float4*>(blk + i * kV + col0 + pc * 4) = *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
   }
 }
+
+// The state kernel's value-tile width for N * HV heads: the narrowest tile
+// whose CTAs (one per SM: they hold 160-221 KB of shared memory) fit in one
+// wave of `sms` SMs, else the widest.
+__host__ __device__ constexpr int state_tile_width(int64_t heads, int sms) {
+  return heads * (kV / 8) <= sms ? 8 : (heads * (kV / 16) <= sms ? 16 : 32);
+}
+template <int BV>
+constexpr int kStateSmem = static_cast<int>(sizeof(typename StateCfg<BV>::Smem));
 
 // ---------------------------------------------------------------- kernel 3
 // The chunk outputs on the tensor cores (tcgen05, kind::f16), transposed so
@@ -842,7 +897,6 @@ __global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(cons
 }
 
 constexpr int kChunkSmem = static_cast<int>(sizeof(ChunkSmem));
-constexpr int kStateSmem = static_cast<int>(sizeof(StateSmem));
 constexpr int kOutSmem = static_cast<int>(sizeof(OutSmem));
 
 }  // namespace kdap
