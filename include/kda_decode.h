@@ -313,6 +313,21 @@ KDA_API kda_status kda_decode_host_pipelined(const kda_decode_args *args, const 
  */
 KDA_API int32_t kda_host_memory_is_mapped(const void *p, int64_t bytes);
 
+/*
+ * Device-side error word of the decode kernels on the current device.  The
+ * one-token gated kernels hand each value tile's outputs to the tile-0 CTA of
+ * the row's cluster, which waits for them with a bounded poll (seconds,
+ * against microseconds for the hand-over); if that wait ever gives up, the
+ * row's output is left unwritten (its state is stored) and this word is set
+ * to 1.
+ * Writes the word (0: no kernel gave up since the last clear) to *word;
+ * clear != 0 then resets it.  Synchronous: it waits for the device's work in
+ * flight.  Errors: KDA_ERR_INVALID_ARG for a NULL word, KDA_ERR_CUDA if the
+ * runtime refuses the read.  The library's own diagnostic; the pages describe
+ * none.
+ */
+KDA_API kda_status kda_decode_device_error(int32_t *word, int32_t clear);
+
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 

@@ -25,7 +25,7 @@ import threading
 import torch
 
 __all__ = ["kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_ex", "HostStep", "HostPipeline", "MappedStep",
-           "host_memory_is_mapped", "kda_prefill",
+           "host_memory_is_mapped", "device_error", "kda_prefill",
            "prefill_workspace_bytes", "KdaError", "library", "status_string",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_ALIAS",
            "KDA_ERR_MISALIGNED", "KDA_ERR_DEVICE", "KDA_ERR_CUDA", "KDA_ERR_SCRATCH_LIMIT", "KDA_STATE_FP32",
@@ -84,6 +84,7 @@ EXPORTED_SYMBOLS = {
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_host_memory_is_mapped": ([_P, _I], ctypes.c_int32),
     "kda_abi_version": ([], ctypes.c_int32),
+    "kda_decode_device_error": ([_P, ctypes.c_int32], ctypes.c_int),
     # include/kda_prefill.h
     "kda_prefill_workspace_bytes": ([_I] * 5, ctypes.c_int64),
     "kda_prefill": ([_P] * 9 + [_I] * 6 + [_F, _P], ctypes.c_int),
@@ -431,6 +432,17 @@ class HostPipeline:
             raise KdaError(rc, "kda_decode_host_pipelined")
         self._next = (i + 1) % len(self._steps)
         return st
+
+
+def device_error(clear: bool = False) -> int:
+    """The decode kernels' device-side error word on the current device (1 if a
+    kernel gave up a bounded wait since the last clear, else 0); ``clear``
+    resets it.  Waits for the device's work in flight."""
+    word = ctypes.c_int32(0)
+    status = library().kda_decode_device_error(ctypes.byref(word), 1 if clear else 0)
+    if status != KDA_OK:
+        raise KdaError(status, "kda_decode_device_error")
+    return int(word.value)
 
 
 def host_memory_is_mapped(t) -> bool:

@@ -20,11 +20,15 @@ namespace kda {
 extern template cudaError_t pick_decode_kernel<64>(const KernelChoice&, const void**, int*);
 extern template cudaError_t pick_decode_kernel<128>(const KernelChoice&, const void**, int*);
 extern template cudaError_t pick_decode_kernel<256>(const KernelChoice&, const void**, int*);
+extern template cudaError_t device_error_word<64>(int32_t*, bool);
+extern template cudaError_t device_error_word<128>(int32_t*, bool);
+extern template cudaError_t device_error_word<256>(int32_t*, bool);
 }  // namespace kda
 
 namespace {
 
 using namespace kda_host;
+
 
 // Host staging of kda_decode_host: the step's inputs are copied from host_in to
 // dev_in before the kernel, the output from out to host_out after it.  With a
@@ -398,6 +402,17 @@ const char* kda_status_string(kda_status status) {
   return "unknown status";
 }
 
-int32_t kda_abi_version(void) { return (1 << 16) | 8; }
+kda_status kda_decode_device_error(int32_t* word, int32_t clear) {
+  if (!word) return KDA_ERR_INVALID_ARG;
+  int32_t w64 = 0, w128 = 0, w256 = 0;
+  if (kda::device_error_word<64>(&w64, clear != 0) != cudaSuccess ||
+      kda::device_error_word<128>(&w128, clear != 0) != cudaSuccess ||
+      kda::device_error_word<256>(&w256, clear != 0) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  *word = w64 | w128 | w256;
+  return KDA_OK;
+}
+
+int32_t kda_abi_version(void) { return (1 << 16) | 9; }
 
 }  // extern "C"

@@ -4,4 +4,5 @@
 
 namespace kda {
 template cudaError_t pick_decode_kernel<128>(const KernelChoice&, const void**, int*);
+template cudaError_t device_error_word<128>(int32_t*, bool);
 }  // namespace kda

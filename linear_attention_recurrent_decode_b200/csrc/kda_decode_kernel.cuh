@@ -326,7 +326,7 @@ template <int RPT>
 struct TokenIn {
   uint32_t q[RPT / 2], k[RPT / 2];
   float g[RPT];
-  uint32_t v[2], z[2];
+  uint32_t v[2];
   float beta;
 };
 
@@ -350,6 +350,38 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(mbar)), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Wait for phase `parity` of the mbarrier with cluster-scope acquire (it also
+// sees what other CTAs of the cluster wrote before their release-arrives on
+// it), giving up after `limit` polls (false then): no kernel waits without
+// bound.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* mbar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_u32(mbar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+// Polls before a wait gives up: each try_wait suspends for a hardware-chosen
+// interval, so this is seconds, against microseconds for what is awaited.
+constexpr uint32_t kWaitPolls = 1u << 24;
+
+// Device-side error word of the kernels of one translation unit (one per key
+// size K): a kernel that gave up a bounded wait stores kDeviceErrorTimeout
+// here (read and cleared by the host through kda_decode_device_error).
+static __device__ int32_t g_device_error;
+constexpr int32_t kDeviceErrorTimeout = 1;
+
 // ---------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_map(uint32_t local_addr, uint32_t rank) {
   uint32_t r;
@@ -358,6 +390,15 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t local_addr, uint32_t ra
 }
 __device__ __forceinline__ void cluster_store_f32(uint32_t cluster_addr, float x) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(x) : "memory");
+}
+__device__ __forceinline__ void cluster_store_f32x4(uint32_t cluster_addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+// Arrive on an mbarrier in another CTA of the cluster, releasing this
+// thread's earlier writes (to that CTA's shared memory included) at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -511,9 +552,9 @@ struct TileIO {
 // Dynamic shared memory a kernel launch must give: the one-token kernel keeps a
 // [V][K] staging buffer there; the multi-token kernel overlays it on its own
 // static buffers.
-template <int K, typename ST, bool VK>
+template <int K, typename ST, int IN, bool VK>
 constexpr int kda_decode_kernel_dyn_smem = TileIO<ST, VK, K, K / 16>::kStageBytes;
-template <int K, typename ST, bool VK>
+template <int K, typename ST, int IN, bool VK>
 constexpr int kda_decode_chunked_kernel_dyn_smem = 0;
 
 // ---------------------------------------------------------------- token staging (T > 1 kernel)
@@ -675,38 +716,31 @@ __device__ __forceinline__ Reduced reduce_tile(const float2 (&pk)[2], const floa
   return r;
 }
 
-// Gated RMS norm of one output row across the V tiles of a cluster: lanes
-// 0..7 of warp 0 (the writers) hold the tile's 32 outputs in o; nrm is this
-// CTA's [kMaxClusterTiles] receive buffer for the per-tile sums of o^2.
-// Every thread of every CTA in the cluster must call it (cluster barrier).
-// (Writers only) push this tile's sum of o^2 into slot `tile` of every peer's
-// receive buffer nrm.
-__device__ __forceinline__ void push_sumsq(const float2 (&o)[2], float* nrm, int tile, int tiles, int lane) {
+// Gated RMS norm of one output row across the V tiles of a cluster.  Lanes
+// 0..7 of warp 0 of each CTA (the writers) hold the tile's 32 outputs.  The
+// writers of every tile hand those and their sum of squares to the CTA of
+// tile 0 (cluster rank 0) and are done: only that CTA waits for the slowest
+// tile, the others retire as soon as their own state is stored.  Its warp 0
+// then normalises the whole row: y = o / rms(o) * w * sigmoid(z).
+// Sum of o^2 over a writer's 4 outputs, reduced across the 8 writers.
+__device__ __forceinline__ float tile_sumsq(const float2 (&o)[2]) {
   float ss = o[0].x * o[0].x + o[0].y * o[0].y + o[1].x * o[1].x + o[1].y * o[1].y;
 #pragma unroll
   for (int m = 1; m < kColQuads; m <<= 1) ss += __shfl_xor_sync(0x000000ffu, ss, m);
-  if (lane < tiles) cluster_store_f32(cluster_map(smem_u32(&nrm[tile]), static_cast<uint32_t>(lane)), ss);
+  return ss;
 }
-// (Writers only, after the cluster barrier) y = o / rms(o) * w * sigmoid(z).
-__device__ __forceinline__ void apply_norm(float (&y)[4], const float2 (&o)[2], const float2 (&wgt)[2],
-                                           const uint32_t (&z)[2], const float* nrm, int tiles, int64_t V,
-                                           float eps) {
-  float tot = 0.f;
-  for (int r = 0; r < tiles; ++r) tot += nrm[r];
-  const float inv = rsqrtf(tot / static_cast<float>(V) + eps);
+// Per lane of warp 0 in tile 0: columns 4 lane + 128 j (j < passes) of the row.
+__device__ __forceinline__ void norm_store(__nv_bfloat16* out, const float* mail_o, float inv, const uint32_t (&z)[2],
+                                          const uint32_t (&w)[2], int64_t c, int64_t V, bool masked) {
+  const float4 x = *reinterpret_cast<const float4*>(mail_o + c);
+  const float ov[4] = {x.x, x.y, x.z, x.w};
   const float zz[4] = {bf16lo(z[0]), bf16hi(z[0]), bf16lo(z[1]), bf16hi(z[1])};
-  const float ov[4] = {o[0].x, o[0].y, o[1].x, o[1].y};
-  const float wv[4] = {wgt[0].x, wgt[0].y, wgt[1].x, wgt[1].y};
+  const float wv[4] = {bf16lo(w[0]), bf16hi(w[0]), bf16lo(w[1]), bf16hi(w[1])};
+  float y[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) y[j] = ov[j] * inv * wv[j] * (1.0f / (1.0f + __expf(-zz[j])));
-}
-__device__ __forceinline__ void gated_norm(float (&y)[4], const float2 (&o)[2], const float2 (&wgt)[2],
-                                           const uint32_t (&z)[2], float* nrm, int tile, int tiles,
-                                           int64_t V, float eps, bool writer, int lane) {
-  if (writer) push_sumsq(o, nrm, tile, tiles, lane);
-  cluster_arrive_release();
-  cluster_wait_acquire();
-  if (writer) apply_norm(y, o, wgt, z, nrm, tiles, V, eps);
+  if (masked) st_bf16x4_masked(out + c, y, c, V);
+  else *reinterpret_cast<uint2*>(out + c) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
 }
 
 template <int K, int VS, bool GATED, typename ST, int IN, bool VK>
@@ -719,7 +753,13 @@ kda_decode_kernel(const ParamsOf<IN> p) {
 
   __shared__ __align__(16) float2 red[kWarps][2][kColQuads * 2];  // [warp][k|q][column pairs]
   __shared__ float red_qk[kWarps];
-  __shared__ float nrm[kMaxClusterTiles];  // gated: per-tile sum of o^2
+  // gated, in tile 0's CTA: every tile's 32 outputs and sum of o^2, and the
+  // barrier the other tiles' writers arrive on once they have written theirs
+  __shared__ __align__(16) float mail_o[GATED ? kMaxClusterTiles : 1][kBV];
+  __shared__ float mail_ss[GATED ? kMaxClusterTiles : 1];
+  __shared__ uint64_t mail_bar;
+  __shared__ __align__(16) __nv_bfloat16 mail_z[GATED ? kMaxClusterTiles * kBV : 8];  // tile 0: gate row
+  __shared__ __align__(16) __nv_bfloat16 mail_w[GATED ? kMaxClusterTiles * kBV : 8];  // tile 0: norm weight
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -773,13 +813,21 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   }
   if constexpr (GEN) {
     ld_bf16x4_masked(cur.v, p.v + in_off<IN, kRowV>(p, row, n, h, V) + col, col, V);
-    if constexpr (GATED) ld_bf16x4_masked(cur.z, p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + col, col, V);
   } else {
     const uint2 vv_raw = __ldg(reinterpret_cast<const uint2*>(p.v + (IN == kInDense ? row * V : in_off<IN, kRowV>(p, row, n, h, V)) + col));
     cur.v[0] = vv_raw.x; cur.v[1] = vv_raw.y;
-    if constexpr (GATED) {
-      const uint2 zz = __ldg(reinterpret_cast<const uint2*>(p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + col));
-      cur.z[0] = zz.x; cur.z[1] = zz.y;
+  }
+  // Gated: warp 0 of tile 0 normalises the whole row, so it copies the gate
+  // and norm weight of every column into shared memory with the inputs (the
+  // general form, whose rows need not be aligned, reads them at the end).
+  if constexpr (GATED && !GEN) {
+    if (tile == 0 && warp == 0) {
+      const __nv_bfloat16* const zrow = p.gate + in_off<IN, kRowZ>(p, row, n, h, V);
+      for (int c = lane; c < V / 8; c += 32) {
+        cp_async16(smem_u32(&mail_z[8 * c]), zrow + 8 * c);
+        cp_async16(smem_u32(&mail_w[8 * c]), p.norm_weight + 8 * c);
+      }
+      cp_async_commit();
     }
   }
   if constexpr (RAW) {
@@ -817,19 +865,11 @@ kda_decode_kernel(const ParamsOf<IN> p) {
   if constexpr (GEN) MaskedTile<ST, RPT>::load(s, sp, V, r0, k_rt, col);
   else Tile::load(s, sp, V, stage, r0, cq);
 
-  if constexpr (GATED) cluster_arrive_relaxed();  // peers must be running before DSMEM writes
-
-  float2 wgt[2] = {f2(0.f), f2(0.f)};
   if constexpr (GATED) {
-    uint32_t w[2];
-    if constexpr (GEN) {
-      ld_bf16x4_masked(w, p.norm_weight + col, col, V);
-    } else {
-      const uint2 x = __ldg(reinterpret_cast<const uint2*>(p.norm_weight + col));
-      w[0] = x.x; w[1] = x.y;
-    }
-    wgt[0] = make_float2(bf16lo(w[0]), bf16hi(w[0]));
-    wgt[1] = make_float2(bf16lo(w[1]), bf16hi(w[1]));
+    // Tile 0's mailbox barrier counts the other tiles' writers; the cluster
+    // barrier makes its initialisation visible before any of them arrives.
+    if (tile == 0 && threadIdx.x == 0 && tiles > 1) mbar_init(&mail_bar, kColQuads * (tiles - 1));
+    cluster_arrive_relaxed();
   }
 
   // decay and the partial reductions over this thread's rows
@@ -882,19 +922,63 @@ kda_decode_kernel(const ParamsOf<IN> p) {
     }
   }
 
+  if constexpr (GATED) {
+    // The writers hand this tile's outputs to tile 0 before the state stores:
+    // their release-arrive then has no stores of this thread to wait for.
+    cluster_wait_acquire();  // every CTA of the cluster runs; tile 0's mailbox is initialised
+    if (writer) {
+      const float ss = tile_sumsq(o);
+      if (tile == 0) {
+        *reinterpret_cast<float4*>(&mail_o[0][4 * cq]) = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);
+        if (lane == 0) mail_ss[0] = ss;
+      } else {
+        cluster_store_f32x4(cluster_map(smem_u32(&mail_o[tile][4 * cq]), 0), o[0].x, o[0].y, o[1].x, o[1].y);
+        if (lane == 0) cluster_store_f32(cluster_map(smem_u32(&mail_ss[tile]), 0), ss);
+        mbar_arrive_remote(cluster_map(smem_u32(&mail_bar), 0));
+      }
+    }
+  }
+
   allow_next_grid();
   if constexpr (GEN) MaskedTile<ST, RPT>::store(sp, s, V, r0, k_rt, col);
   else Tile::store(sp, s, V, stage, r0, cq);
 
   if constexpr (GATED) {
-    // The norm needs the whole head's o; the state does not, so it is
-    // already on its way out before the cluster exchange.
-    cluster_wait_acquire();  // pairs with the relaxed arrive after the state loads
-    float y[4];
-    gated_norm(y, o, wgt, cur.z, nrm, tile, tiles, V, p.eps, writer, lane);
-    if (writer) {
-      if constexpr (GEN) st_bf16x4_masked(p.out + row * V + col, y, col, V);
-      else *reinterpret_cast<uint2*>(p.out + row * V + col) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+    // Tile 0's warp 0 waits (bounded) for the other tiles, normalises the row
+    // and stores it; every other CTA is done.
+    if (tile == 0 && warp == 0) {
+      __syncwarp();  // this tile's writers' mailbox entries
+      bool ok = tiles == 1 || mbar_wait_cluster_bounded(&mail_bar, 0, kWaitPolls);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        // The row's output stays unwritten; the CTA still waits (bounded) for
+        // the writes into its mailbox before it exits.
+        if (lane == 0) atomicExch(&g_device_error, kDeviceErrorTimeout);
+        mbar_wait_cluster_bounded(&mail_bar, 0, kWaitPolls);
+        return;
+      }
+      float tot = 0.f;
+      for (int r = 0; r < tiles; ++r) tot += mail_ss[r];
+      const float inv = rsqrtf(tot / static_cast<float>(V) + p.eps);
+      if constexpr (!GEN) cp_async_wait<0>();
+      __syncwarp();  // the gate and weight copies of every lane
+      constexpr int kNormPasses = VS ? (VS + 127) / 128 : kMaxClusterTiles * kBV / 128;
+#pragma unroll
+      for (int j = 0; j < kNormPasses; ++j) {
+        const int64_t c = 4 * lane + 128 * j;
+        if (c >= static_cast<int64_t>(tiles) * kBV) continue;
+        uint32_t z[2], w[2];
+        if constexpr (GEN) {
+          ld_bf16x4_masked(z, p.gate + in_off<IN, kRowZ>(p, row, n, h, V) + c, c, V);
+          ld_bf16x4_masked(w, p.norm_weight + c, c, V);
+        } else {
+          const uint2 zz = *reinterpret_cast<const uint2*>(&mail_z[c]);
+          const uint2 ww = *reinterpret_cast<const uint2*>(&mail_w[c]);
+          z[0] = zz.x; z[1] = zz.y;
+          w[0] = ww.x; w[1] = ww.y;
+        }
+        norm_store(p.out + row * V, &mail_o[0][0], inv, z, w, c, V, GEN);
+      }
     }
   }
 }

@@ -77,6 +77,18 @@ cudaError_t allow_dynamic_smem(int bytes) {
 }
 
 
+// The device error word of K's translation unit (g_device_error is static:
+// one per unit, written only by that unit's kernels); clear resets it.
+template <int K>
+cudaError_t device_error_word(int32_t* word, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_device_error, sizeof(int32_t));
+  if (e == cudaSuccess && clear) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+  }
+  return e;
+}
+
 template <int K>
 cudaError_t pick_decode_kernel(const KernelChoice& c, const void** func, int* smem_out) {
   cudaError_t err = cudaSuccess;
@@ -87,7 +99,7 @@ cudaError_t pick_decode_kernel(const KernelChoice& c, const void** func, int* sm
 #define KDA_PICK_ONE(KERNEL, KK, VV, GG, STT, RR, VKK)                                               \
   do {                                                                                                \
     constexpr auto kern = KERNEL<KK, VV, GG, STT, RR, VKK>;                                           \
-    constexpr int smem = KERNEL##_dyn_smem<KK, STT, VKK>;                                             \
+    constexpr int smem = KERNEL##_dyn_smem<KK, STT, RR, VKK>;                                         \
     *smem_out = smem;                                                                                 \
     err = smem ? allow_dynamic_smem<kern>(smem) : cudaSuccess;                                        \
     if (err == cudaSuccess && c.check_launch) err = launchable<kern>(gated ? c.tiles : 1, smem);      \

@@ -45,7 +45,7 @@ def test_header_declares_the_documented_entry_points():
     assert declared_functions() == {"kda_decode", "kda_decode_gated_rmsnorm", "kda_decode_bf16_state",
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
                                     "kda_decode_host", "kda_decode_host_pipelined", "kda_status_string",
-                                    "kda_abi_version", "kda_host_memory_is_mapped",
+                                    "kda_abi_version", "kda_host_memory_is_mapped", "kda_decode_device_error",
                                     "kda_prefill", "kda_prefill_workspace_bytes", "kda_prefill_no_alloc"}
 
 
@@ -66,7 +66,11 @@ def test_status_strings_and_version(lib):
     for s in range(1, 8):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(99) == "unknown status"
-    assert lib.kda_abi_version() == (1 << 16) | 8
+    assert lib.kda_abi_version() == (1 << 16) | 9
+
+
+def test_device_error_query_validates_its_argument(lib):
+    assert lib.kda_decode_device_error(None, 0) == kda.KDA_ERR_INVALID_ARG
 
 
 # ----------------------------------------------------------------- validation

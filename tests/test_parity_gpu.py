@@ -810,3 +810,20 @@ def test_mapped_host_step_equals_device_call(name, cuda_device):
     ref = kda.kda_decode_ex(d.q, d.k, d.v, d.state, d.slot_idx, scale=w.scale, **dextra)
     torch.cuda.synchronize()
     assert torch.equal(out_h, ref.cpu()) and torch.equal(pool, d.state)
+
+
+def test_no_kernel_gave_up_a_bounded_wait(cuda_device):
+    """The multi-token kernels' state-tile copy and the gated kernels' output
+    hand-over end in bounded waits; after a plain, a gated and a multi-token
+    call (and everything this file ran before) none of them gave up."""
+    kda.device_error(clear=False)
+    for name in ("n32_t4_hv8", "n32_t1_hv16_gated"):
+        w = workloads.config(name).to(cuda_device)
+        if w.gated:
+            kda.kda_decode_gated_rmsnorm(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx, w.gate, w.norm_weight,
+                                         eps=w.eps, scale=w.scale)
+        else:
+            kda.kda_decode(w.q, w.k, w.v, w.g, w.beta, w.state, w.slot_idx, scale=w.scale)
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    assert kda.device_error() == 0
