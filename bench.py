@@ -106,6 +106,51 @@ def profiled_traffic(workload: str):
     return None
 
 
+def fp32_alu_peak_tflops(sms: int, mhz: float = 1965.0) -> float:
+    """fp32 CUDA-core peak: SMs x 128 fp32 FMA lanes (4 sub-partitions x 32)
+    x 2 flop per FMA x the SM clock (B200's clocks.max.sm, 1965 MHz)."""
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def prefill_state_flops(w) -> int:
+    """Algorithmic flops of the prefill's state recurrence (stage 1) for one
+    call: per chunk of Tc tokens and (n, h), U = Ut - W S0 (2 Tc K V), the
+    decay D S0 (K V), S = D S0 + Kh^T U (2 K Tc V) and the subtraction (Tc V)."""
+    nchunks = (w.T + 63) // 64
+    return w.N * w.HV * (4 * w.T * w.K * w.V + nchunks * w.K * w.V + w.T * w.V)
+
+
+def time_prefill_state_stage(kda, reps, outs, stream, steps):
+    """µs per launch of the prefill's state recurrence (kda_prefill_stage 1, the
+    longest of the call's three kernels): CUDA events on the launching stream
+    around eager launches that rotate over the replicas, each replica's
+    workspace first filled by one whole call."""
+    import torch
+
+    fns = []
+    with torch.cuda.stream(stream):
+        for d, o in zip(reps, outs):
+            ws = torch.empty(kda.prefill_workspace_bytes(d.N, d.T, d.HV, d.K, d.V), dtype=torch.uint8,
+                             device=d.q.device)
+            kda.kda_prefill(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx, out=o, scale=d.scale, workspace=ws,
+                            stream=stream)
+            fns.append(lambda d=d, o=o, ws=ws: kda.kda_prefill(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx,
+                                                               out=o, scale=d.scale, workspace=ws, stream=stream,
+                                                               stage=1))
+        for f in fns[:3]:
+            f()
+    n = max(2 * len(fns), min(steps, 200))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for i in range(n):
+            fns[i % len(fns)]()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1e3 / n, n
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -395,6 +440,12 @@ def run_ours(args):
     torch.cuda.synchronize()
     eager_us = reduce_max(ea.elapsed_time(eb), dev) * 1e3 / n_eager
 
+    # prefill: the state recurrence alone (its roofline; see prefill_state_flops)
+    stage = None
+    if args.config.startswith("prefill_"):
+        stage_us, stage_n = time_prefill_state_stage(kda, reps, outs, stream, args.steps)
+        stage = (reduce_max(stage_us, dev), stage_n)
+
     # end to end through the public API: pinned host inputs in, output back out
     n_e2e = min(args.steps, args.e2e_steps)
     if args.config.startswith("prefill_"):
@@ -419,6 +470,25 @@ def run_ours(args):
         cpu = {"value": t_cpu * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n_calls} full calls of {args.config} (fp64 C loop, threads over (n,h))"}
     clocks = sampler.summary() if sampler else None
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": bytes_per_call,
+                "traffic": profiled_traffic(args.config)}
+    if stage is not None:
+        # The prefill's longest kernel is its fp32 state recurrence on the CUDA
+        # cores: flops against the fp32 ALU peak (the call's HBM view kept beside).
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        alu_peak = fp32_alu_peak_tflops(sms)
+        flops = prefill_state_flops(base)
+        tf = flops / (stage[0] * 1e-6) / 1e12
+        roofline = {"bound": "alu", "kernel": "kda_prefill_state_kernel (stage 1: the state recurrence)",
+                    "achieved": round(tf, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(tf / alu_peak, 4),
+                    "peak_source": f"derived: {sms} SMs x 128 fp32 FMA lanes x 2 flop x 1965 MHz",
+                    "algorithmic_flops_per_launch": flops, "launch_us": round(stage[0], 2),
+                    "launches_timed": stage[1], "traffic": None,
+                    "call_hbm": {"achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                                 "frac": round(achieved / peak, 4), "algorithmic_bytes_per_call": bytes_per_call}}
     line = {
         "metric": METRIC, "value": round(us_per_call_job, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -435,10 +505,7 @@ def run_ours(args):
                    "region_us_per_call": [round(x * 1e3 / args.steps, 4) for x in region_ms],
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "gbs": round(achieved, 1),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": bytes_per_call,
-                     "traffic": profiled_traffic(args.config)},
+        "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "eager": {"value": round(eager_us, 3), "unit": UNIT, "steps": n_eager,

@@ -81,6 +81,25 @@ KDA_API kda_status kda_prefill(const void *q, const void *k, const void *v, cons
                                kda_stream_t stream);
 
 /*
+ * One of kda_prefill's three kernels: stage 0 prepares every chunk (its solve
+ * and decayed factors into the workspace), stage 1 runs the state recurrence
+ * across the chunks (the final state into each active row's slot, each
+ * chunk's start state and corrections into the workspace), stage 2 writes the
+ * chunk outputs.  kda_prefill is stages 0, 1 and 2 in that order on one
+ * stream.  Same arguments, validation and errors as kda_prefill, plus
+ * KDA_ERR_INVALID_ARG for a stage outside 0..2; each stage reads what the
+ * previous one left in the workspace, so a caller keeps their order on the
+ * stream (stage 1 starts from the slot's state: run it once per prefill).
+ * For callers that time the stages or put other work between them; the pages
+ * name the chunk form's parts but no such entry point.
+ */
+KDA_API kda_status kda_prefill_stage(int32_t stage, const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta, float *state_pool,
+                                     const int32_t *slot_idx, void *out, void *workspace,
+                                     int64_t workspace_bytes, int64_t N, int64_t T, int64_t HV, int64_t K,
+                                     int64_t V, float scale, kda_stream_t stream);
+
+/*
  * The same chunked prefill for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point; it is this library's own.
  *

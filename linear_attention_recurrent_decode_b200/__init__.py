@@ -89,6 +89,7 @@ EXPORTED_SYMBOLS = {
     "kda_prefill_workspace_bytes": ([_I] * 5, ctypes.c_int64),
     "kda_prefill": ([_P] * 9 + [_I] * 6 + [_F, _P], ctypes.c_int),
     "kda_prefill_no_alloc": ([_P] * 8 + [_I] * 5 + [_F, _P], ctypes.c_int),
+    "kda_prefill_stage": ([ctypes.c_int32] + [_P] * 9 + [_I] * 6 + [_F, _P], ctypes.c_int),
 }
 
 _lock = threading.Lock()
@@ -547,12 +548,15 @@ def prefill_workspace_bytes(N: int, T: int, HV: int, K: int = 128, V: int = 128)
 
 
 def kda_prefill(q, k, v, g, beta, state_pool, slot_idx, out=None, scale: float | None = None, workspace=None,
-                stream=None):
+                stream=None, stage: int | None = None):
     """Chunked prefill (``kda_prefill`` of the C ABI): the decode recurrence over
     all T tokens of each sequence, taken in chunks of 64 tokens; updates
     ``state_pool`` (fp32 [num_slots, HV, K, V]) in place and returns ``out``
     (bf16 [N, T, HV, V]).  ``workspace``: a device uint8 tensor of at least
-    :func:`prefill_workspace_bytes` bytes (allocated here if not given)."""
+    :func:`prefill_workspace_bytes` bytes (allocated here if not given).
+    ``stage`` 0, 1 or 2 runs only that kernel (``kda_prefill_stage``: chunk
+    preparation, state recurrence, chunk outputs; a caller keeps their order
+    and passes the same workspace to all three)."""
     N, T, HV, K, V, out = _common(q, k, v, g, beta, state_pool, slot_idx, out)
     if state_pool.dtype != torch.float32:
         raise TypeError("kda_prefill takes an fp32 state pool")
@@ -562,9 +566,13 @@ def kda_prefill(q, k, v, g, beta, state_pool, slot_idx, out=None, scale: float |
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(workspace, "workspace", torch.uint8, None, torch.cuda.current_device())
-    st = library().kda_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(),
-                               state_pool.data_ptr(), slot_idx.data_ptr(), out.data_ptr(), workspace.data_ptr(),
-                               workspace.numel(), N, T, HV, K, V, float(scale), _stream_handle(stream))
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), beta.data_ptr(), state_pool.data_ptr(),
+            slot_idx.data_ptr(), out.data_ptr(), workspace.data_ptr(), workspace.numel(), N, T, HV, K, V,
+            float(scale), _stream_handle(stream))
+    if stage is None:
+        st = library().kda_prefill(*args)
+    else:
+        st = library().kda_prefill_stage(int(stage), *args)
     if st != KDA_OK:
-        raise KdaError(st, "kda_prefill")
+        raise KdaError(st, "kda_prefill" if stage is None else "kda_prefill_stage")
     return out

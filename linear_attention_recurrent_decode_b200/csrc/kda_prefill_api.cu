@@ -61,6 +61,13 @@ int sm_count() {
   return v;
 }
 
+// Validation and the launches of the stages in [first, last] (0: chunk
+// preparation, 1: state recurrence, 2: chunk outputs), in order.
+kda_status prefill_stages(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          float* state_pool, const int32_t* slot_idx, void* out, void* workspace,
+                          int64_t workspace_bytes, int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
+                          float scale, kda_stream_t stream, int first, int last);
+
 }  // namespace
 
 extern "C" {
@@ -78,6 +85,27 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
                        float* state_pool, const int32_t* slot_idx, void* out, void* workspace,
                        int64_t workspace_bytes, int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
                        float scale, kda_stream_t stream) {
+  return prefill_stages(q, k, v, g, beta, state_pool, slot_idx, out, workspace, workspace_bytes, N, T, HV, K, V,
+                        scale, stream, 0, 2);
+}
+
+kda_status kda_prefill_stage(int32_t stage, const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, float* state_pool, const int32_t* slot_idx, void* out,
+                             void* workspace, int64_t workspace_bytes, int64_t N, int64_t T, int64_t HV, int64_t K,
+                             int64_t V, float scale, kda_stream_t stream) {
+  if (stage < 0 || stage > 2) return KDA_ERR_INVALID_ARG;
+  return prefill_stages(q, k, v, g, beta, state_pool, slot_idx, out, workspace, workspace_bytes, N, T, HV, K, V,
+                        scale, stream, stage, stage);
+}
+
+}  // extern "C"
+
+namespace {
+
+kda_status prefill_stages(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          float* state_pool, const int32_t* slot_idx, void* out, void* workspace,
+                          int64_t workspace_bytes, int64_t N, int64_t T, int64_t HV, int64_t K, int64_t V,
+                          float scale, kda_stream_t stream, int first, int last) {
   if (N < 0 || T < 0 || HV < 0 || K < 0 || V < 0 || workspace_bytes < 0) return KDA_ERR_INVALID_ARG;
   if (HV < 1 || K != kp::kK || V != kp::kV) return KDA_ERR_UNSUPPORTED;
   if (N == 0 || T == 0) return KDA_OK;  // nothing to do; no pointer is touched
@@ -138,18 +166,23 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
   };
   const int bv = kp::state_tile_width(N * HV, sm_count());
   const int64_t grid_tiles = N * HV * (kp::kV / bv);
-  cudaError_t e_state = cudaSuccess;
-  if (run(kp::kda_prefill_chunk_kernel, grid_chunks, kp::kChunkThreads, kp::kChunkSmem) != cudaSuccess)
+  if (first <= 0 && 0 <= last &&
+      run(kp::kda_prefill_chunk_kernel, grid_chunks, kp::kChunkThreads, kp::kChunkSmem) != cudaSuccess)
     return KDA_ERR_CUDA;
-  if (bv == 8) e_state = run(kp::kda_prefill_state_kernel<8>, grid_tiles, kp::kStateThreads, kp::kStateSmem<8>);
-  else if (bv == 16) e_state = run(kp::kda_prefill_state_kernel<16>, grid_tiles, kp::kStateThreads, kp::kStateSmem<16>);
-  else e_state = run(kp::kda_prefill_state_kernel<32>, grid_tiles, kp::kStateThreads, kp::kStateSmem<32>);
-  if (e_state != cudaSuccess || run(kp::kda_prefill_output_kernel, grid_chunks, kp::kOutThreads, kp::kOutSmem) != cudaSuccess)
+  if (first <= 1 && 1 <= last) {
+    cudaError_t e_state;
+    if (bv == 8) e_state = run(kp::kda_prefill_state_kernel<8>, grid_tiles, kp::kStateThreads, kp::kStateSmem<8>);
+    else if (bv == 16) e_state = run(kp::kda_prefill_state_kernel<16>, grid_tiles, kp::kStateThreads, kp::kStateSmem<16>);
+    else e_state = run(kp::kda_prefill_state_kernel<32>, grid_tiles, kp::kStateThreads, kp::kStateSmem<32>);
+    if (e_state != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  if (first <= 2 && 2 <= last &&
+      run(kp::kda_prefill_output_kernel, grid_chunks, kp::kOutThreads, kp::kOutSmem) != cudaSuccess)
     return KDA_ERR_CUDA;
   return KDA_OK;
 }
 
-}  // extern "C"
+}  // namespace
 
 // ---------------------------------------------------------------- kda_prefill_no_alloc
 // Scratch for callers that cannot allocate (see include/kda_prefill.h): a

@@ -81,11 +81,13 @@ struct Workspace {
   static constexpr int64_t kWt = 0;                   // W^T  [K][C]
   static constexpr int64_t kKh = kWt + kK * kC;       // Kh   [C][K]
   static constexpr int64_t kUt = kKh + kC * kK;       // Ut   [C][V]   (the V part of the solve)
-  static constexpr int64_t kQ = kUt + kC * kV;        // Qt   [C][K]   (decayed queries)
-  static constexpr int64_t kP = kQ + kC * kK;         // P    [C][C]   (zero for s > t)
-  static constexpr int64_t kDc = kP + kC * kC;        // exp(Gamma_C) [K]
-  static constexpr int64_t kS0 = kDc + kK;            // chunk-start state [K][V]
-  static constexpr int64_t kU = kS0 + kK * kV;        // U [C][V]
+  // The output operands, as bf16 hi and lo planes in the canonical K-major
+  // layout (see put_pair): rows x K-dimension of each MMA operand.
+  static constexpr int64_t kQ = kUt + kC * kV;        // Qt   [C rows][K]  (decayed queries)
+  static constexpr int64_t kP = kQ + kC * kK;         // P    [C rows][C]  (zero for s > t)
+  static constexpr int64_t kDc = kP + kC * kC;        // exp(Gamma_C) [K]  (fp32)
+  static constexpr int64_t kS0 = kDc + kK;            // S0^T [V rows][K]  (chunk-start state)
+  static constexpr int64_t kU = kS0 + kK * kV;        // U^T  [V rows][C]
   static constexpr int64_t kFloats = kU + kC * kV;    // per record
   static __host__ __device__ int64_t record(int64_t unit, int64_t chunk, int32_t nchunks) {
     return kHeaderFloats + (unit * nchunks + chunk) * kFloats;
@@ -95,6 +97,44 @@ struct Workspace {
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// ---------------------------------------------------------------- output-operand tiles
+// The output kernel's four MMA operands (S0^T, Qt, U^T, P) are written by the
+// kernels that compute them straight into their workspace regions in the
+// tensor cores' shared-memory layout, each as a bf16 hi plane followed by a
+// bf16 lo plane (x = hi + lo, 16 significant bits; the same bytes as fp32),
+// so that the output kernel moves them into shared memory with bulk copies.
+// Offset, in bytes, of element (row r, k) of a K-major bf16 tile with kd
+// elements along K (canonical layout, no swizzle).
+__host__ __device__ constexpr uint32_t kmajor_off(int r, int k, int kd) {
+  return static_cast<uint32_t>((r / 8) * (kd / 8) * 128 + (k / 8) * 128 + (r % 8) * 16 + (k % 8) * 2);
+}
+// The hi and lo bf16 halves of eight fp32 values, packed for one 16-byte store each.
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+    h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[i] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Element (r, c) of an fp32 operand tile as its bf16 pair: hi = bf16(x) into
+// the hi plane at the canonical offset, lo = bf16(x - hi) at the same offset
+// of the lo plane, `plane_bytes` after it (the same split as split8).
+__device__ __forceinline__ void put_pair(unsigned char* hi_plane, int plane_bytes, int r, int c, int kd, float x) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
+  const uint32_t off = kmajor_off(r, c, kd);
+  *reinterpret_cast<__nv_bfloat16*>(hi_plane + off) = h;
+  *reinterpret_cast<__nv_bfloat16*>(hi_plane + plane_bytes + off) = l;
+}
+
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
@@ -214,7 +254,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   // exponentials per element (exp(+-(Gamma_t - Gamma_r))) and the channel's
   // exp(Gamma_r), exp(Gamma_C - Gamma_r).
   float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
-  float* const Pm = rec + Workspace::kP;  // P[t][s]
+  unsigned char* const q_pl = reinterpret_cast<unsigned char*>(rec + Workspace::kQ);  // Qt planes
+  unsigned char* const p_pl = reinterpret_cast<unsigned char*>(rec + Workspace::kP);  // P planes
+  constexpr int kQPlane = kC * kK * 2, kPPlane = kC * kC * 2;
   if (tid < kK) rec[Workspace::kDc + tid] = exp_of(gam_end);
   constexpr int kPer = kC * kK / kChunkThreads;  // elements per thread
   if (!exact) {
@@ -235,7 +277,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       fb[j] = kv * down;
       sm.kt[t][i] = fa[j] * sm.e_ref[i];                                // k exp(Gamma_t)
       rec[Workspace::kKh + t * kK + i] = fb[j] * sm.e_end_ref[i];       // k exp(Gamma_C - Gamma_t)
-      rec[Workspace::kQ + t * kK + i] = fq[j] * sm.e_ref[i];            // q exp(Gamma_t)
+      put_pair(q_pl, kQPlane, t, i, kK, fq[j] * sm.e_ref[i]);            // q exp(Gamma_t)
     }
     __syncthreads();
     // The solve needs v, which the factors overwrite: move it into the Gamma
@@ -290,7 +332,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
         for (int b = 0; b < 4; ++b) {
           const int s = sb * 4 + b;
           sm.L[t][s] = (s < t) ? sm.beta[t] * mv[b] : 0.f;
-          Pm[t * kC + s] = (s <= t) ? pv[b] : 0.f;
+          put_pair(p_pl, kPPlane, t, s, kC, (s <= t) ? pv[b] : 0.f);
         }
       }
     } else {  // the 120 tiles above the diagonal: zeros
@@ -306,7 +348,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           sm.L[tb * 4 + a][sb * 4 + b] = 0.f;
-          Pm[(tb * 4 + a) * kC + sb * 4 + b] = 0.f;
+          put_pair(p_pl, kPPlane, tb * 4 + a, sb * 4 + b, kC, 0.f);
         }
     }
   } else {
@@ -319,7 +361,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       const float dt = exp_of(gt);
       sm.kt[t][i] = kv * dt;                                                   // k exp(Gamma_t)
       rec[Workspace::kKh + t * kK + i] = kv * exp_of(sm.gam[kC - 1][i] - gt);  // k exp(Gamma_C - Gamma_t)
-      rec[Workspace::kQ + t * kK + i] = __bfloat162float(raw.q[t][i]) * dt;    // q exp(Gamma_t)
+      put_pair(q_pl, kQPlane, t, i, kK, __bfloat162float(raw.q[t][i]) * dt);   // q exp(Gamma_t)
     }
     for (int e = tid; e < kC * kC; e += kChunkThreads) {
       const int t = e / kC, s = e % kC;
@@ -332,7 +374,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
         }
       }
       sm.L[t][s] = (s < t) ? sm.beta[t] * mv : 0.f;
-      Pm[t * kC + s] = (s <= t) ? pv : 0.f;
+      put_pair(p_pl, kPPlane, t, s, kC, (s <= t) ? pv : 0.f);
     }
     __syncthreads();
     float* const vf = reinterpret_cast<float*>(&sm.gam[0][0]);
@@ -504,11 +546,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
     const typename Cfg::Buf& b = sm.buf[cb];
     float* const rec = p.ws + Workspace::record(unit, c, p.nchunks);
 
-    // chunk-start state to the workspace (the output kernel reads it)
-    for (int e = tid; e < kK * (BV / 4); e += kStateThreads) {
-      const int i = e / (BV / 4), pc = e % (BV / 4);
-      *reinterpret_cast<float4*>(rec + Workspace::kS0 + i * kV + col0 + pc * 4) =
-          *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
+    // chunk-start state to the workspace as the output MMA's S0^T operand
+    // (rows: this tile's value columns; 8 key rows per 16-byte store)
+    unsigned char* const s0_pl = reinterpret_cast<unsigned char*>(rec + Workspace::kS0);
+    for (int e = tid; e < BV * (kK / 8); e += kStateThreads) {
+      const int jl = e % BV, ig = e / BV;
+      float x[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) x[r] = sm.s[ig * 8 + r][jl];
+      uint4 hi, lo;
+      split8(x, hi, lo);
+      const uint32_t off = kmajor_off(col0 + jl, ig * 8, kK);
+      *reinterpret_cast<uint4*>(s0_pl + off) = hi;
+      *reinterpret_cast<uint4*>(s0_pl + kK * kV * 2 + off) = lo;
     }
 
     {  // W S over one quarter of K
@@ -544,12 +594,24 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
       for (int jj = 0; jj < Cfg::kUW; ++jj) {
         const int j = u_j + jj;
         const float ws = (sm.pw[0][j][u_t] + sm.pw[1][j][u_t]) + (sm.pw[2][j][u_t] + sm.pw[3][j][u_t]);
-        const float uo = b.ut[u_t][j] - ws;
-        sm.u[u_t][j] = uo;
-        rec[Workspace::kU + u_t * kV + col0 + j] = uo;
+        sm.u[u_t][j] = b.ut[u_t][j] - ws;
       }
     }
     __syncthreads();
+    {  // U to the workspace as the output MMA's U^T operand (8 tokens per 16-byte store)
+      unsigned char* const u_pl = reinterpret_cast<unsigned char*>(rec + Workspace::kU);
+      for (int e = tid; e < BV * (kC / 8); e += kStateThreads) {
+        const int jl = e % BV, tg = e / BV;
+        float x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) x[r] = sm.u[tg * 8 + r][jl];
+        uint4 hi, lo;
+        split8(x, hi, lo);
+        const uint32_t off = kmajor_off(col0 + jl, tg * 8, kC);
+        *reinterpret_cast<uint4*>(u_pl + off) = hi;
+        *reinterpret_cast<uint4*>(u_pl + kC * kV * 2 + off) = lo;
+      }
+    }
     {  // Kh^T U over one split of the chunk
       float2 acc[2][Cfg::kJW2 / 2];
 #pragma unroll
@@ -668,6 +730,16 @@ __device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(mbar)), "r"(count) : "memory");
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(mbar)), "r"(bytes) : "memory");
+}
+// Bulk copy (TMA unit) of `bytes` contiguous bytes, global -> this CTA's shared
+// memory (both 16-byte aligned, bytes a multiple of 16), completing on `mbar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(mbar))
+               : "memory");
+}
 // Wait for phase `parity` of the mbarrier, giving up after `limit` polls
 // (returns false then): the kernels never wait without bound.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* mbar, uint32_t parity, uint32_t limit) {
@@ -704,26 +776,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Offset, in bytes, of element (row r, k) of a K-major bf16 tile with kd
-// elements along K (canonical layout, no swizzle).
-__host__ __device__ constexpr uint32_t kmajor_off(int r, int k, int kd) {
-  return static_cast<uint32_t>((r / 8) * (kd / 8) * 128 + (k / 8) * 128 + (r % 8) * 16 + (k % 8) * 2);
-}
-// The hi and lo bf16 halves of eight fp32 values, packed for one 16-byte store each.
-__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-    const float2 hf = __bfloat1622float2(hh);
-    const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
-    h[i] = *reinterpret_cast<const uint32_t*>(&hh);
-    l[i] = *reinterpret_cast<const uint32_t*>(&ll);
-  }
-  hi = make_uint4(h[0], h[1], h[2], h[3]);
-  lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
 }  // namespace tc
 
 constexpr int kOutThreads = 256;
@@ -738,7 +790,8 @@ struct OutSmem {
   alignas(1024) unsigned char a2l[kV * kC * 2];
   alignas(1024) unsigned char b2h[kC * kC * 2];  // P     [C rows][C]
   alignas(1024) unsigned char b2l[kC * kC * 2];
-  uint64_t mbar;
+  uint64_t mbar_in;  // the operand copies
+  uint64_t mbar;     // the MMAs
   uint32_t tmem;
 };
 
@@ -762,93 +815,39 @@ __global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(cons
     return;
   }
   if (warp == 0) tc::tmem_alloc(&sm.tmem, kOutTmemCols);
-  if (tid == 0) tc::mbar_init(&sm.mbar, 1);
-
-  // ---- operand tiles: fp32 from the workspace, split to bf16 hi/lo.  Each
-  // phase issues all of a thread's (read-only) loads before any split or
-  // store, so the 144 KB a CTA reads are in flight together.
-  const float* const rec = p.ws + Workspace::record(unit, chunk, p.nchunks);
-  {  // A1 = S0^T: items (value row j, key group of 8), loads coalesced over j
-    constexpr int kItems = kV * (kK / 8) / kOutThreads;  // 8
-    float x[kItems][8];
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-      const int e = tid + it * kOutThreads, jj = e % kV, ig = e / kV;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) x[it][r] = __ldg(rec + Workspace::kS0 + (ig * 8 + r) * kV + jj);
-    }
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-      const int e = tid + it * kOutThreads, jj = e % kV, ig = e / kV;
-      uint4 hi, lo;
-      tc::split8(x[it], hi, lo);
-      *reinterpret_cast<uint4*>(sm.a1h + tc::kmajor_off(jj, ig * 8, kK)) = hi;
-      *reinterpret_cast<uint4*>(sm.a1l + tc::kmajor_off(jj, ig * 8, kK)) = lo;
-    }
+  if (tid == 0) {
+    tc::mbar_init(&sm.mbar_in, 1);
+    tc::mbar_init(&sm.mbar, 1);
   }
-  {  // A2 = U^T (items (j, token group of 8)) and B2 = P (items (t, token group of 8))
-    constexpr int kItemsA = kV * (kC / 8) / kOutThreads;  // 4
-    constexpr int kItemsB = kC * (kC / 8) / kOutThreads;  // 2
-    float x[kItemsA][8];
-    float4 y[kItemsB][2];
-#pragma unroll
-    for (int it = 0; it < kItemsA; ++it) {
-      const int e = tid + it * kOutThreads, jj = e % kV, sg = e / kV;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) x[it][r] = __ldg(rec + Workspace::kU + (sg * 8 + r) * kV + jj);
-    }
-#pragma unroll
-    for (int it = 0; it < kItemsB; ++it) {
-      const int e = tid + it * kOutThreads, t = e / (kC / 8), sg = e % (kC / 8);
-      y[it][0] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8));
-      y[it][1] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kP + t * kC + sg * 8 + 4));
-    }
-#pragma unroll
-    for (int it = 0; it < kItemsA; ++it) {
-      const int e = tid + it * kOutThreads, jj = e % kV, sg = e / kV;
-      uint4 hi, lo;
-      tc::split8(x[it], hi, lo);
-      *reinterpret_cast<uint4*>(sm.a2h + tc::kmajor_off(jj, sg * 8, kC)) = hi;
-      *reinterpret_cast<uint4*>(sm.a2l + tc::kmajor_off(jj, sg * 8, kC)) = lo;
-    }
-#pragma unroll
-    for (int it = 0; it < kItemsB; ++it) {
-      const int e = tid + it * kOutThreads, t = e / (kC / 8), sg = e % (kC / 8);
-      const float v8[8] = {y[it][0].x, y[it][0].y, y[it][0].z, y[it][0].w,
-                           y[it][1].x, y[it][1].y, y[it][1].z, y[it][1].w};
-      uint4 hi, lo;
-      tc::split8(v8, hi, lo);
-      *reinterpret_cast<uint4*>(sm.b2h + tc::kmajor_off(t, sg * 8, kC)) = hi;
-      *reinterpret_cast<uint4*>(sm.b2l + tc::kmajor_off(t, sg * 8, kC)) = lo;
-    }
-  }
-  {  // B1 = Qt: items (token row t, key group of 8), one 32-byte read each
-    constexpr int kItems = kC * (kK / 8) / kOutThreads;  // 4
-    float4 y[kItems][2];
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-      const int e = tid + it * kOutThreads, t = e / (kK / 8), ig = e % (kK / 8);
-      y[it][0] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8));
-      y[it][1] = __ldg(reinterpret_cast<const float4*>(rec + Workspace::kQ + t * kK + ig * 8 + 4));
-    }
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-      const int e = tid + it * kOutThreads, t = e / (kK / 8), ig = e % (kK / 8);
-      const float v8[8] = {y[it][0].x, y[it][0].y, y[it][0].z, y[it][0].w,
-                           y[it][1].x, y[it][1].y, y[it][1].z, y[it][1].w};
-      uint4 hi, lo;
-      tc::split8(v8, hi, lo);
-      *reinterpret_cast<uint4*>(sm.b1h + tc::kmajor_off(t, ig * 8, kK)) = hi;
-      *reinterpret_cast<uint4*>(sm.b1l + tc::kmajor_off(t, ig * 8, kK)) = lo;
-    }
-  }
-  tc::fence_proxy_async();  // the tiles, written by threads, are read by the tensor cores
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+
+  // ---- operand tiles: the producers left them in this layout, as bf16 hi and
+  // lo planes; eight bulk copies bring them in (144 KB).
+  const unsigned char* const rec =
+      reinterpret_cast<const unsigned char*>(p.ws + Workspace::record(unit, chunk, p.nchunks));
+  if (tid == 0) {
+    constexpr uint32_t kA1 = kV * kK * 2, kB1 = kC * kK * 2, kA2 = kV * kC * 2, kB2 = kC * kC * 2;
+    tc::mbar_arrive_expect_tx(&sm.mbar_in, 2 * (kA1 + kB1 + kA2 + kB2));
+    const unsigned char* const s0 = rec + Workspace::kS0 * 4;
+    const unsigned char* const qt = rec + Workspace::kQ * 4;
+    const unsigned char* const ut = rec + Workspace::kU * 4;
+    const unsigned char* const pp = rec + Workspace::kP * 4;
+    tc::bulk_load(sm.a1h, s0, kA1, &sm.mbar_in);
+    tc::bulk_load(sm.a1l, s0 + kA1, kA1, &sm.mbar_in);
+    tc::bulk_load(sm.b1h, qt, kB1, &sm.mbar_in);
+    tc::bulk_load(sm.b1l, qt + kB1, kB1, &sm.mbar_in);
+    tc::bulk_load(sm.a2h, ut, kA2, &sm.mbar_in);
+    tc::bulk_load(sm.a2l, ut + kA2, kA2, &sm.mbar_in);
+    tc::bulk_load(sm.b2h, pp, kB2, &sm.mbar_in);
+    tc::bulk_load(sm.b2l, pp + kB2, kB2, &sm.mbar_in);
+  }
+  // about 2^26 polls: seconds, against microseconds for the copies and MMAs
+  const bool in_ok = __syncthreads_and(tc::mbar_wait_bounded(&sm.mbar_in, 0, 1u << 26));
   const uint32_t tmem = sm.tmem;
 
-  if (tid == 0) {
+  if (tid == 0 && in_ok) {
     constexpr uint32_t idesc = tc::idesc_bf16(128, kC);
     const uint32_t a1h = smem_addr(sm.a1h), a1l = smem_addr(sm.a1l), b1h = smem_addr(sm.b1h),
                    b1l = smem_addr(sm.b1l), a2h = smem_addr(sm.a2h), a2l = smem_addr(sm.a2l),
@@ -874,8 +873,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(cons
     }
     tc::commit(&sm.mbar);
   }
-  // about 2^26 polls: seconds, against microseconds for the MMAs
-  const bool ok = tc::mbar_wait_bounded(&sm.mbar, 0, 1u << 26);
+  const bool ok = in_ok && tc::mbar_wait_bounded(&sm.mbar, 0, 1u << 26);
   tc::fence_after_sync();
   if (ok) {
     // lane j of this warp's 32-lane slice; columns (tokens) of this warp's half
@@ -890,6 +888,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) kda_prefill_output_kernel(cons
     }
   } else if (tid == 0) {
     atomicExch(reinterpret_cast<int*>(p.ws), 1);  // the workspace header's error word
+    if (!in_ok) tc::mbar_wait_bounded(&sm.mbar_in, 0, 1u << 26);  // copies still in flight
   }
   tc::fence_before_sync();
   __syncthreads();

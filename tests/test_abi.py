@@ -46,7 +46,8 @@ def test_header_declares_the_documented_entry_points():
                                     "kda_decode_gated_rmsnorm_bf16_state", "kda_decode_ex",
                                     "kda_decode_host", "kda_decode_host_pipelined", "kda_status_string",
                                     "kda_abi_version", "kda_host_memory_is_mapped", "kda_decode_device_error",
-                                    "kda_prefill", "kda_prefill_workspace_bytes", "kda_prefill_no_alloc"}
+                                    "kda_prefill", "kda_prefill_workspace_bytes", "kda_prefill_no_alloc",
+                                    "kda_prefill_stage"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -324,6 +325,17 @@ def test_prefill_validation(lib):
     assert call(ws=BASE + 9 * step + 64) == E.KDA_ERR_ALIAS   # workspace over out
     assert call(ws=BASE + 5 * step - 1024) == E.KDA_ERR_ALIAS # workspace runs into the pool
     assert call(g=BASE + 5 * step + 4096) == E.KDA_ERR_ALIAS  # an input inside slot 0
+
+    def stage(s, **kw):
+        return lib.kda_prefill_stage(s, BASE, BASE + step, BASE + 2 * step, BASE + 3 * step, BASE + 4 * step,
+                                     BASE + 5 * step, BASE + 8 * step, BASE + 9 * step, BASE + 12 * step, need,
+                                     kw.get("n", N), T, HV, kw.get("K", 128), 128, 0.1, None)
+
+    for s in (0, 1, 2):                                      # one kernel each, validated like the whole call
+        assert stage(s) == E.KDA_ERR_DEVICE
+        assert stage(s, K=64) == E.KDA_ERR_UNSUPPORTED
+    assert stage(3) == E.KDA_ERR_INVALID_ARG
+    assert stage(-1) == E.KDA_ERR_INVALID_ARG
 
 
 @no_gpu

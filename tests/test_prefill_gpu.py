@@ -112,6 +112,26 @@ def test_prefill_back_to_back_calls_continue_the_state(cuda_device):
         check_state(d.state[s].cpu().numpy(), ref_state[s])
 
 
+def test_prefill_stages_in_order_equal_one_call(cuda_device):
+    """kda_prefill_stage 0, 1, 2 on one stream compute exactly what kda_prefill
+    does (the same kernels with the same launch shapes): bit-identical outputs
+    and final states."""
+    w = workloads.make(N=3, T=150, HV=4, num_slots=5, seed=371, inactive=1)
+    a, b = w.to(cuda_device), w.to(cuda_device)
+    ws = torch.empty(kda.prefill_workspace_bytes(3, 150, 4), dtype=torch.uint8, device=cuda_device)
+    o_all = kda.kda_prefill(a.q, a.k, a.v, a.g, a.beta, a.state, a.slot_idx, scale=w.scale, workspace=ws)
+    ws2 = torch.empty_like(ws)
+    o_st = torch.empty_like(o_all)
+    for stage in (0, 1, 2):
+        kda.kda_prefill(b.q, b.k, b.v, b.g, b.beta, b.state, b.slot_idx, out=o_st, scale=w.scale, workspace=ws2,
+                        stage=stage)
+    torch.cuda.synchronize()
+    assert torch.equal(o_all, o_st)
+    assert torch.equal(a.state, b.state)
+    with pytest.raises(kda.KdaError):
+        kda.kda_prefill(b.q, b.k, b.v, b.g, b.beta, b.state, b.slot_idx, out=o_st, workspace=ws2, stage=3)
+
+
 def test_prefill_rejections(cuda_device):
     w = workloads.make(N=2, T=70, HV=2, num_slots=3, seed=361)
     d = w.to(cuda_device)
