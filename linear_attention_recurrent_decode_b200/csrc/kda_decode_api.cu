@@ -5,8 +5,9 @@
 // (queried once per device, as the FlashInfer #4562 review of `CheckTarget`
 // asks for a latency-sensitive decode path), and one kernel launch on the
 // caller's stream (kda_decode_host adds the copies in and out around it).
-// Nothing here allocates, synchronises or falls back to another
-// implementation.
+// Nothing here allocates or falls back to another implementation, and no
+// step entry point synchronises (kda_decode_device_error, a diagnostic, reads
+// the kernels' error word synchronously).
 #include <atomic>
 #include <cstddef>
 #include <cstdint>

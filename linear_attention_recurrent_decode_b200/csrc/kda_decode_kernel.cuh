@@ -40,9 +40,11 @@
 // and each state element is read and written once per chunk.
 //
 // The gated variant launches the V/32 tiles of one (n, h) as a thread-block
-// cluster: each CTA pushes its partial sum of o^2 into every peer's shared
-// memory (DSMEM) and a cluster barrier completes the RMS over V; the norm,
-// weight and sigmoid gate are applied before the bf16 store.
+// cluster.  One token: every tile hands its outputs and their sum of squares
+// to the tile-0 CTA through distributed shared memory and an mbarrier, and
+// that CTA alone applies the RMS over V, the norm weight and the sigmoid gate
+// before the bf16 store.  Several tokens: each CTA pushes its per-token sums of
+// o^2 into every peer and one cluster barrier per chunk completes the RMS.
 //
 // Inputs may be row-strided views (q, k, v as slices of one packed buffer),
 // and the serving form takes a raw bf16 gate and beta activated in the kernel

@@ -33,14 +33,17 @@ cudaError_t prepare_kernels() {
   cudaError_t e = cudaFuncSetAttribute(kp::kda_prefill_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kp::kChunkSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kp::kStateSmem<8>);
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<8, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<8, 256>);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kp::kStateSmem<16>);
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<16, 256>);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kp::kStateSmem<32>);
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<32, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<32, 256>);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kp::kda_prefill_state_kernel<64, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kp::kStateSmem<64, 512>);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kp::kda_prefill_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kp::kOutSmem);
@@ -171,9 +174,10 @@ kda_status prefill_stages(const void* q, const void* k, const void* v, const flo
     return KDA_ERR_CUDA;
   if (first <= 1 && 1 <= last) {
     cudaError_t e_state;
-    if (bv == 8) e_state = run(kp::kda_prefill_state_kernel<8>, grid_tiles, kp::kStateThreads, kp::kStateSmem<8>);
-    else if (bv == 16) e_state = run(kp::kda_prefill_state_kernel<16>, grid_tiles, kp::kStateThreads, kp::kStateSmem<16>);
-    else e_state = run(kp::kda_prefill_state_kernel<32>, grid_tiles, kp::kStateThreads, kp::kStateSmem<32>);
+    if (bv == 8) e_state = run(kp::kda_prefill_state_kernel<8, 256>, grid_tiles, 256, kp::kStateSmem<8, 256>);
+    else if (bv == 16) e_state = run(kp::kda_prefill_state_kernel<16, 256>, grid_tiles, 256, kp::kStateSmem<16, 256>);
+    else if (bv == 32) e_state = run(kp::kda_prefill_state_kernel<32, 256>, grid_tiles, 256, kp::kStateSmem<32, 256>);
+    else e_state = run(kp::kda_prefill_state_kernel<64, 512>, grid_tiles, 512, kp::kStateSmem<64, 512>);
     if (e_state != cudaSuccess) return KDA_ERR_CUDA;
   }
   if (first <= 2 && 2 <= last &&

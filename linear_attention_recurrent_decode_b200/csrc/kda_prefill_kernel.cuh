@@ -448,62 +448,78 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
 }
 
 // ---------------------------------------------------------------- kernel 2
-// One CTA per (n, h, BV-column value tile) walks the chunks in order with its
-// K x BV state tile in shared memory; the next chunk's W^T, Kh, Ut and
-// exp(Gamma_C) are staged with cp.async while the current one is processed.
-// Both products split their reduction over the CTA (W S over quarters of K,
-// Kh^T U over halves of the chunk for narrow tiles), use packed fp32x2 FMAs,
-// and sum the partials in a fixed order.  Every CTA reads the chunk's 64 KB
-// of W^T and Kh whatever its width, so the launch takes the widest tile that
-// still keeps one CTA on every SM it can: BV = 8 for a few heads (one 8192-
-// token prompt at 8 heads: 128 CTAs), 16 or 32 for batches of prompts.
-constexpr int kStateThreads = 256;
+// One CTA of NT threads per (n, h, BV-column value tile) walks the chunks in
+// order with its K x BV state tile in shared memory.  Per chunk:
+// U = Ut - W S0 (W S split over quarters of K) and S = D S0 + Kh^T U (Kh^T U
+// split over parts of the chunk for narrow tiles), packed fp32x2 FMAs, the
+// partials summed in a fixed order.
+// Staging: the next chunk's operands are copied (cp.async) while the current
+// one is processed.  Narrow tiles (8, 16 columns) double-buffer all of them.
+// Wide tiles keep one buffer each for W^T and Kh (64 KB together), refilled
+// for the next chunk as soon as the product that reads it is done (W^T after
+// W S, Kh after Kh^T U) -- their longer chunk steps leave each copy time to
+// land -- which is what lets a 64-column tile's buffers fit one SM.  The two
+// products' partial sums share their bytes (one is dead while the other is in
+// use).  Every CTA reads the
+// chunk's 64 KB of W^T and Kh whatever its width, so the launch takes the
+// narrowest tile whose CTAs fit one per SM in one wave, else 64-column tiles
+// of 512 threads (see state_tile_width).
 constexpr int kCU = kC + 4;  // padded rows of the transposed partial buffers
 
-template <int BV>
+template <int BV, int NT>
 struct StateCfg {
-  static_assert(BV == 8 || BV == 16 || BV == 32, "value tile of 8, 16 or 32 columns");
-  static constexpr int kJW = BV / 4;                 // W S: columns per thread (4 column groups)
-  static constexpr int kCS = BV == 32 ? 1 : 2;       // Kh^T U: splits of the chunk
-  static constexpr int kJW2 = BV == 8 ? 4 : 8;       // Kh^T U: columns per thread
-  static constexpr int kNG2 = BV / kJW2;             // Kh^T U: column groups
-  static_assert(64 * kNG2 * kCS == kStateThreads, "Kh^T U covers the tile once");
-  static constexpr int kUW = BV / 4;                 // U: columns per thread
-  static constexpr int kSW = BV / 2;                 // S update: columns per thread
-  struct Buf {
-    float wt[kK][kC];   // W^T
-    float kh[kC][kK];   // Kh
-    float ut[kC][BV];   // this tile's columns of Ut
-    float dc[kK];       // exp(Gamma_C)
+  static_assert((NT == 256 && (BV == 8 || BV == 16 || BV == 32)) || (NT == 512 && (BV == 32 || BV == 64)),
+                "tile widths 8, 16, 32 (256 threads) and 32, 64 (512 threads)");
+  static constexpr int kJW = 64 * BV / NT;   // W S: columns per thread (thread: K quarter, 4 tokens)
+  static constexpr int kNJ = BV / kJW;       //       column groups
+  static constexpr int kJW2 = BV == 8 ? 4 : 8;  // Kh^T U: columns per thread (thread: 2 key rows)
+  static constexpr int kNG2 = BV / kJW2;        //         column groups
+  static constexpr int kCS = NT / (64 * kNG2);  //         parts of the chunk
+  static_assert(64 * kNG2 * kCS == NT && kC % kCS == 0, "Kh^T U covers the tile once");
+  static constexpr int kUW = 64 * BV / NT;   // U: columns per thread (thread: one token)
+  static constexpr int kRT = NT / kK;        // S update: threads per key row
+  static constexpr int kSW = BV / kRT;       //           columns per thread
+  static_assert(kJW % 2 == 0 && kSW % 4 == 0, "packed pairs and float4 rows");
+  static constexpr int kPart = 4 * BV * kCU > kCS * BV * (kK + 4) ? 4 * BV * kCU : kCS * BV * (kK + 4);
+  static constexpr bool kDB = BV <= 16;      // W^T and Kh double-buffered
+  static constexpr int kNB = kDB ? 2 : 1;
+  struct UBuf {
+    float ut[kC][BV];  // this tile's columns of Ut
+    float dc[kK];      // exp(Gamma_C)
   };
   struct Smem {
-    Buf buf[2];
-    float s[kK][BV];              // state tile
-    float pw[4][BV][kCU];         // (W S) partial sums per quarter of K, [j][t]
-    float u[kC][BV + 4];          // U of the current chunk, [t][j]
-    float ps[kCS][BV][kK + 4];    // (Kh^T U) partial sums per split of the chunk, [j][i]
+    float wt[kNB][kK][kC];  // W^T of the current chunk (and of the next: see kDB)
+    float kh[kNB][kC][kK];  // Kh, likewise
+    UBuf ub[2];
+    float s[kK][BV];        // state tile
+    float u[kC][BV + 4];    // U of the current chunk, [t][j]
+    float part[kPart];      // (W S) partials [4][BV][kCU], then (Kh^T U) partials [kCS][BV][kK + 4]
   };
 };
 
-template <int BV>
-__device__ __forceinline__ void stage_chunk(typename StateCfg<BV>::Buf& b, const float* rec, int col0, int tid) {
-  for (int c = tid; c < (kK * kC) / 4; c += kStateThreads) {
-    cp_async16(&b.wt[0][0] + 4 * c, rec + Workspace::kWt + 4 * c);
-    cp_async16(&b.kh[0][0] + 4 * c, rec + Workspace::kKh + 4 * c);
-  }
-  for (int c = tid; c < kC * (BV / 4); c += kStateThreads) {
+template <int NT>
+__device__ __forceinline__ void stage_wt(float (&wt)[kK][kC], const float* rec, int tid) {
+  for (int c = tid; c < (kK * kC) / 4; c += NT) cp_async16(&wt[0][0] + 4 * c, rec + Workspace::kWt + 4 * c);
+}
+template <int NT>
+__device__ __forceinline__ void stage_kh(float (&kh)[kC][kK], const float* rec, int tid) {
+  for (int c = tid; c < (kC * kK) / 4; c += NT) cp_async16(&kh[0][0] + 4 * c, rec + Workspace::kKh + 4 * c);
+}
+template <int BV, int NT>
+__device__ __forceinline__ void stage_ub(typename StateCfg<BV, NT>::UBuf& b, const float* rec, int col0, int tid) {
+  for (int c = tid; c < kC * (BV / 4); c += NT) {
     const int t = c / (BV / 4), pc = c % (BV / 4);
     cp_async16(&b.ut[t][pc * 4], rec + Workspace::kUt + t * kV + col0 + pc * 4);
   }
-  for (int c = tid; c < kK / 4; c += kStateThreads) cp_async16(&b.dc[4 * c], rec + Workspace::kDc + 4 * c);
+  for (int c = tid; c < kK / 4; c += NT) cp_async16(&b.dc[4 * c], rec + Workspace::kDc + 4 * c);
 }
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 splat(float x) { return make_float2(x, x); }
 
-template <int BV>
-__global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(const Params p) {
-  using Cfg = StateCfg<BV>;
+template <int BV, int NT>
+__global__ void __launch_bounds__(NT, 1) kda_prefill_state_kernel(const Params p) {
+  using Cfg = StateCfg<BV, NT>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   typename Cfg::Smem& sm = *reinterpret_cast<typename Cfg::Smem*>(smem_raw);
   constexpr int kTiles = kV / BV;
@@ -517,39 +533,61 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
   if (slot < 0) return;
 
   float* const blk = p.state + (static_cast<int64_t>(slot) * p.HV + h) * kK * kV;
-  for (int c = tid; c < kK * (BV / 4); c += kStateThreads) {  // initial state tile
+  for (int c = tid; c < kK * (BV / 4); c += NT) {  // initial state tile
     const int i = c / (BV / 4), pc = c % (BV / 4);
     cp_async16(&sm.s[i][pc * 4], blk + i * kV + col0 + pc * 4);
   }
-  stage_chunk<BV>(sm.buf[0], p.ws + Workspace::record(unit, 0, p.nchunks), col0, tid);
+  {
+    const float* const rec0 = p.ws + Workspace::record(unit, 0, p.nchunks);
+    stage_wt<NT>(sm.wt[0], rec0, tid);
+    stage_kh<NT>(sm.kh[0], rec0, tid);
+    stage_ub<BV, NT>(sm.ub[0], rec0, col0, tid);
+  }
   cp_async_commit();
 
   // W S: thread (quarter of K, 4 tokens, kJW columns)
-  const int a_t = (tid % 16) * 4, a_j = ((tid / 16) % 4) * Cfg::kJW, a_q = tid / 64;
+  const int a_t = (tid % 16) * 4, a_j = ((tid / 16) % Cfg::kNJ) * Cfg::kJW, a_q = tid / (16 * Cfg::kNJ);
   // U: thread (token, kUW columns)
   const int u_t = tid % 64, u_j = (tid / 64) * Cfg::kUW;
-  // Kh^T U: thread (2 key rows, kJW2 columns, split of the chunk)
+  // Kh^T U: thread (2 key rows, kJW2 columns, part of the chunk)
   const int b_i = (tid % 64) * 2, b_j = ((tid / 64) % Cfg::kNG2) * Cfg::kJW2, b_h = tid / (64 * Cfg::kNG2);
   // S update: thread (key row, kSW columns)
-  const int s_i = tid / 2, s_j = (tid % 2) * Cfg::kSW;
+  const int s_i = tid / Cfg::kRT, s_j = (tid % Cfg::kRT) * Cfg::kSW;
+  float (*const pw)[BV][kCU] = reinterpret_cast<float (*)[BV][kCU]>(sm.part);
+  float (*const ps)[BV][kK + 4] = reinterpret_cast<float (*)[BV][kK + 4]>(sm.part);
 
   for (int32_t c = 0; c < p.nchunks; ++c) {
     const int cb = c & 1;
-    if (c + 1 < p.nchunks) {
-      stage_chunk<BV>(sm.buf[cb ^ 1], p.ws + Workspace::record(unit, c + 1, p.nchunks), col0, tid);
+    const bool more = c + 1 < p.nchunks;
+    float* const rec = p.ws + Workspace::record(unit, c, p.nchunks);
+    const float* const rec_next = p.ws + Workspace::record(unit, more ? c + 1 : c, p.nchunks);
+    constexpr bool kDB = Cfg::kDB;
+    const int wb = kDB ? cb : 0;  // this chunk's W^T and Kh buffers
+    if (more) {
+      stage_ub<BV, NT>(sm.ub[cb ^ 1], rec_next, col0, tid);
+      if constexpr (kDB) {
+        stage_wt<NT>(sm.wt[cb ^ 1], rec_next, tid);
+        stage_kh<NT>(sm.kh[cb ^ 1], rec_next, tid);
+      }
       cp_async_commit();
-      cp_async_wait<1>();
+    }
+    // This chunk's operands: with double buffers all of them, the next chunk's
+    // copies in flight; with single ones W^T, Ut and exp(Gamma_C) (all of
+    // chunk 0 at the start), this chunk's Kh and the next Ut in flight.
+    if (kDB || c == 0) {
+      if (more) cp_async_wait<1>(); else cp_async_wait<0>();
     } else {
-      cp_async_wait<0>();
+      if (more) cp_async_wait<2>(); else cp_async_wait<1>();
     }
     __syncthreads();
-    const typename Cfg::Buf& b = sm.buf[cb];
-    float* const rec = p.ws + Workspace::record(unit, c, p.nchunks);
+    const typename Cfg::UBuf& ub = sm.ub[cb];
+    const float (&wt)[kK][kC] = sm.wt[wb];
+    const float (&kh)[kC][kK] = sm.kh[wb];
 
     // chunk-start state to the workspace as the output MMA's S0^T operand
     // (rows: this tile's value columns; 8 key rows per 16-byte store)
     unsigned char* const s0_pl = reinterpret_cast<unsigned char*>(rec + Workspace::kS0);
-    for (int e = tid; e < BV * (kK / 8); e += kStateThreads) {
+    for (int e = tid; e < BV * (kK / 8); e += NT) {
       const int jl = e % BV, ig = e / BV;
       float x[8];
 #pragma unroll
@@ -570,10 +608,18 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
       const int i_lo = a_q * (kK / 4);
 #pragma unroll 4
       for (int i = i_lo; i < i_lo + kK / 4; ++i) {
-        const float4 w = *reinterpret_cast<const float4*>(&b.wt[i][a_t]);
+        const float4 w = *reinterpret_cast<const float4*>(&wt[i][a_t]);
         float2 sv[Cfg::kJW / 2];
+        if constexpr (Cfg::kJW % 4 == 0) {
 #pragma unroll
-        for (int jj = 0; jj < Cfg::kJW / 2; ++jj) sv[jj] = *reinterpret_cast<const float2*>(&sm.s[i][a_j + 2 * jj]);
+          for (int q4 = 0; q4 < Cfg::kJW / 4; ++q4) {
+            const float4 x = *reinterpret_cast<const float4*>(&sm.s[i][a_j + 4 * q4]);
+            sv[2 * q4] = make_float2(x.x, x.y);
+            sv[2 * q4 + 1] = make_float2(x.z, x.w);
+          }
+        } else {
+          sv[0] = *reinterpret_cast<const float2*>(&sm.s[i][a_j]);
+        }
         const float wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int a = 0; a < 4; ++a)
@@ -582,25 +628,34 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
       }
 #pragma unroll
       for (int jj = 0; jj < Cfg::kJW / 2; ++jj) {
-        *reinterpret_cast<float4*>(&sm.pw[a_q][a_j + 2 * jj][a_t]) =
+        *reinterpret_cast<float4*>(&pw[a_q][a_j + 2 * jj][a_t]) =
             make_float4(acc[0][jj].x, acc[1][jj].x, acc[2][jj].x, acc[3][jj].x);
-        *reinterpret_cast<float4*>(&sm.pw[a_q][a_j + 2 * jj + 1][a_t]) =
+        *reinterpret_cast<float4*>(&pw[a_q][a_j + 2 * jj + 1][a_t]) =
             make_float4(acc[0][jj].y, acc[1][jj].y, acc[2][jj].y, acc[3][jj].y);
       }
     }
-    __syncthreads();
+    __syncthreads();  // the partials are complete; W^T is free for the next chunk's
+    if (!kDB && more) {
+      stage_wt<NT>(sm.wt[0], rec_next, tid);
+      cp_async_commit();
+    }
     {  // U = Ut - W S, the quarters summed in a fixed order
 #pragma unroll
       for (int jj = 0; jj < Cfg::kUW; ++jj) {
         const int j = u_j + jj;
-        const float ws = (sm.pw[0][j][u_t] + sm.pw[1][j][u_t]) + (sm.pw[2][j][u_t] + sm.pw[3][j][u_t]);
-        sm.u[u_t][j] = b.ut[u_t][j] - ws;
+        const float ws = (pw[0][j][u_t] + pw[1][j][u_t]) + (pw[2][j][u_t] + pw[3][j][u_t]);
+        sm.u[u_t][j] = ub.ut[u_t][j] - ws;
       }
     }
-    __syncthreads();
+    // This chunk's Kh (chunk 0's came with the first group); the copies
+    // committed after it (the next Ut and W^T) stay in flight.
+    if (!kDB && c > 0) {
+      if (more) cp_async_wait<2>(); else cp_async_wait<0>();
+    }
+    __syncthreads();  // U is complete; the W S partials are dead
     {  // U to the workspace as the output MMA's U^T operand (8 tokens per 16-byte store)
       unsigned char* const u_pl = reinterpret_cast<unsigned char*>(rec + Workspace::kU);
-      for (int e = tid; e < BV * (kC / 8); e += kStateThreads) {
+      for (int e = tid; e < BV * (kC / 8); e += NT) {
         const int jl = e % BV, tg = e / BV;
         float x[8];
 #pragma unroll
@@ -612,7 +667,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
         *reinterpret_cast<uint4*>(u_pl + kC * kV * 2 + off) = lo;
       }
     }
-    {  // Kh^T U over one split of the chunk
+    {  // Kh^T U over one part of the chunk
       float2 acc[2][Cfg::kJW2 / 2];
 #pragma unroll
       for (int a = 0; a < 2; ++a)
@@ -621,7 +676,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
       const int t_lo = b_h * (kC / Cfg::kCS);
 #pragma unroll 4
       for (int t = t_lo; t < t_lo + kC / Cfg::kCS; ++t) {
-        const float2 kh = *reinterpret_cast<const float2*>(&b.kh[t][b_i]);
+        const float2 kv = *reinterpret_cast<const float2*>(&kh[t][b_i]);
         float2 uv[Cfg::kJW2 / 2];
 #pragma unroll
         for (int q4 = 0; q4 < Cfg::kJW2 / 4; ++q4) {
@@ -631,23 +686,26 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
         }
 #pragma unroll
         for (int jj = 0; jj < Cfg::kJW2 / 2; ++jj) {
-          acc[0][jj] = ffma2(splat(kh.x), uv[jj], acc[0][jj]);
-          acc[1][jj] = ffma2(splat(kh.y), uv[jj], acc[1][jj]);
+          acc[0][jj] = ffma2(splat(kv.x), uv[jj], acc[0][jj]);
+          acc[1][jj] = ffma2(splat(kv.y), uv[jj], acc[1][jj]);
         }
       }
 #pragma unroll
       for (int a = 0; a < 2; ++a)
 #pragma unroll
         for (int jj = 0; jj < Cfg::kJW2 / 2; ++jj) {
-          sm.ps[b_h][b_j + 2 * jj][b_i + a] = acc[a][jj].x;
-          sm.ps[b_h][b_j + 2 * jj + 1][b_i + a] = acc[a][jj].y;
+          ps[b_h][b_j + 2 * jj][b_i + a] = acc[a][jj].x;
+          ps[b_h][b_j + 2 * jj + 1][b_i + a] = acc[a][jj].y;
         }
     }
     // S = D S + Kh^T U.  The decay is read before the barrier: after it no
-    // thread touches this chunk's stage buffer, which the next iteration's
-    // prefetch then refills.
-    const float d = b.dc[s_i];
-    __syncthreads();
+    // thread reads this chunk's Ut buffer, which the next iteration refills.
+    const float d = ub.dc[s_i];
+    __syncthreads();  // the partials are complete; Kh is free for the next chunk's
+    if (!kDB && more) {
+      stage_kh<NT>(sm.kh[0], rec_next, tid);
+      cp_async_commit();
+    }
 #pragma unroll
     for (int q4 = 0; q4 < Cfg::kSW / 4; ++q4) {
       const int j = s_j + 4 * q4;
@@ -655,33 +713,34 @@ __global__ void __launch_bounds__(kStateThreads, 1) kda_prefill_state_kernel(con
       float hs[4];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
-        float acc = sm.ps[0][j + jj][s_i];
+        float acc = ps[0][j + jj][s_i];
 #pragma unroll
-        for (int cs = 1; cs < Cfg::kCS; ++cs) acc += sm.ps[cs][j + jj][s_i];
+        for (int cs = 1; cs < Cfg::kCS; ++cs) acc += ps[cs][j + jj][s_i];
         hs[jj] = acc;
       }
       *reinterpret_cast<float4*>(&sm.s[s_i][j]) =
           make_float4(fmaf(d, s0.x, hs[0]), fmaf(d, s0.y, hs[1]), fmaf(d, s0.z, hs[2]), fmaf(d, s0.w, hs[3]));
     }
-    // The next iteration's prefetch refills this chunk's stage buffer, which no
-    // thread reads after the barrier above; its first barrier orders these
-    // writes of s before any read.
+    // The next iteration's first barrier orders these writes of s before any
+    // read, and the partial buffer's reuse by its W S after this update.
   }
   __syncthreads();
-  for (int c = tid; c < kK * (BV / 4); c += kStateThreads) {
+  for (int c = tid; c < kK * (BV / 4); c += NT) {
     const int i = c / (BV / 4), pc = c % (BV / 4);
     *reinterpret_cast<float4*>(blk + i * kV + col0 + pc * 4) = *reinterpret_cast<const float4*>(&sm.s[i][pc * 4]);
   }
 }
 
 // The state kernel's value-tile width for N * HV heads: the narrowest tile
-// whose CTAs (one per SM: they hold 160-221 KB of shared memory) fit in one
-// wave of `sms` SMs, else the widest.
+// whose CTAs (one per SM) fit in one wave of `sms` SMs, else 64 columns (512
+// threads a CTA), which needs the fewest waves.
 __host__ __device__ constexpr int state_tile_width(int64_t heads, int sms) {
-  return heads * (kV / 8) <= sms ? 8 : (heads * (kV / 16) <= sms ? 16 : 32);
+  return heads * (kV / 8) <= sms ? 8 : (heads * (kV / 16) <= sms ? 16 : (heads * (kV / 32) <= sms ? 32 : 64));
 }
-template <int BV>
-constexpr int kStateSmem = static_cast<int>(sizeof(typename StateCfg<BV>::Smem));
+// Threads of the state kernel for a tile width.
+__host__ __device__ constexpr int state_threads(int bv) { return bv >= 64 ? 512 : 256; }
+template <int BV, int NT>
+constexpr int kStateSmem = static_cast<int>(sizeof(typename StateCfg<BV, NT>::Smem));
 
 // ---------------------------------------------------------------- kernel 3
 // The chunk outputs on the tensor cores (tcgen05, kind::f16), transposed so

@@ -53,7 +53,8 @@ def assert_prefill_parity(w, o, pool, before):
     (2, 257, 4, 0, "uniform"),     # five chunks, mild decays (exp(g) in [0.5, 1))
     (4, 200, 1, 2, "softplus"),    # two inactive rows
     (3, 130, 4, 1, "softplus"),    # 12 heads: the state chain's 16-column tiles
-    (5, 96, 8, 1, "uniform"),      # 40 heads: 32-column tiles
+    (4, 100, 6, 0, "softplus"),    # 24 heads: 32-column tiles
+    (5, 96, 8, 1, "uniform"),      # 40 heads: 64-column tiles of 512 threads
 ])
 def test_prefill_shapes(N, T, HV, inactive, decay, cuda_device):
     w = workloads.make(N=N, T=T, HV=HV, num_slots=N + 2, seed=300 + T + N, inactive=inactive, decay=decay)
