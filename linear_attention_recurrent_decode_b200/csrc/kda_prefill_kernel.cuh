@@ -207,10 +207,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       *reinterpret_cast<uint4*>(&raw.v[t][pc * 8]) = make_uint4(0, 0, 0, 0);
     }
   }
-  // g goes through the kt buffer (free until step 2): 32 pieces of 16 B per row
-  for (int c = tid; c < tc * (kK / 4); c += kChunkThreads) {
+  // g goes through the kt buffer (free until step 2): 32 pieces of 16 B per
+  // row; rows past the chunk's end are zeros (those tokens do not decay)
+  for (int c = tid; c < kC * (kK / 4); c += kChunkThreads) {
     const int t = c / (kK / 4), pc = c % (kK / 4);
-    cp_async16(&sm.kt[t][pc * 4], p.g + ((n * p.T + t0 + t) * p.HV + h) * kK + pc * 4);
+    if (t < tc) cp_async16(&sm.kt[t][pc * 4], p.g + ((n * p.T + t0 + t) * p.HV + h) * kK + pc * 4);
+    else *reinterpret_cast<float4*>(&sm.kt[t][pc * 4]) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   cp_async_commit();
   if (tid < kC) sm.beta[tid] = tid < tc ? __ldg(p.beta + (n * p.T + t0 + tid) * p.HV + h) : 0.f;
@@ -218,17 +220,25 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   cp_async_wait<0>();
   __syncthreads();
 
-  // Gamma per key channel (threads 0..127), summed in fp64; tokens past the
-  // chunk's end do not decay.  The reference token r is the chunk's middle.
+  // Gamma per key channel, summed in fp64 in token order: threads i and
+  // i + 128 each sum one half of the chunk, then the second half adds the
+  // first half's total.  The reference token r is the chunk's middle.
   constexpr int kRef = kC / 2 - 1;
-  if (tid < kK) {
-    const int i = tid;
+  {
+    const int i = tid % kK, t_lo = (tid / kK) * (kC / 2);
     double acc = 0.0;
-#pragma unroll 8
-    for (int t = 0; t < kC; ++t) {
-      if (t < tc) acc += static_cast<double>(sm.kt[t][i]);
+#pragma unroll
+    for (int t = t_lo; t < t_lo + kC / 2; ++t) {
+      acc += static_cast<double>(sm.kt[t][i]);
       sm.gam[t][i] = acc;
     }
+  }
+  __syncthreads();
+  if (tid >= kK) {
+    const int i = tid - kK;
+    const double first = sm.gam[kC / 2 - 1][i];
+#pragma unroll
+    for (int t = kC / 2; t < kC; ++t) sm.gam[t][i] += first;
   }
   __syncthreads();
   double gam_end = 0.0, gam_ref = 0.0;  // per channel (threads 0..127)
@@ -263,11 +273,16 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
     // The factors go through registers: the raw inputs they are made from live
     // in the buffers they are written to.
     float fa[kPer], fq[kPer], fb[kPer];
+    // each thread keeps one channel i (kChunkThreads is a multiple of K)
+    static_assert(kChunkThreads % kK == 0, "one key channel per thread");
+    const int ci = tid % kK;
+    const double g_ref = sm.gam[kRef][ci];
+    const float er = sm.e_ref[ci], eer = sm.e_end_ref[ci];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int e = tid + j * kChunkThreads;  // consecutive threads, consecutive channels
-      const int t = e / kK, i = e % kK;
-      const double d = sm.gam[t][i] - sm.gam[kRef][i];
+      const int t = e / kK, i = ci;
+      const double d = sm.gam[t][i] - g_ref;
       const float up = exp_of(d);      // exp(Gamma_t - Gamma_r), in [e^-80, e^80] on this path
       const float down = __frcp_rn(up);  // exp(Gamma_r - Gamma_t), correctly rounded reciprocal
       const float kv = __bfloat162float(raw.k[t][i]);
@@ -275,9 +290,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
       fa[j] = kv * up;
       fq[j] = qv * up;
       fb[j] = kv * down;
-      sm.kt[t][i] = fa[j] * sm.e_ref[i];                                // k exp(Gamma_t)
-      rec[Workspace::kKh + t * kK + i] = fb[j] * sm.e_end_ref[i];       // k exp(Gamma_C - Gamma_t)
-      put_pair(q_pl, kQPlane, t, i, kK, fq[j] * sm.e_ref[i]);            // q exp(Gamma_t)
+      sm.kt[t][i] = fa[j] * er;                                          // k exp(Gamma_t)
+      rec[Workspace::kKh + t * kK + i] = fb[j] * eer;                    // k exp(Gamma_C - Gamma_t)
+      put_pair(q_pl, kQPlane, t, i, kK, fq[j] * er);                     // q exp(Gamma_t)
     }
     __syncthreads();
     // The solve needs v, which the factors overwrite: move it into the Gamma
