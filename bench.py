@@ -451,7 +451,7 @@ def run_ours(args):
     if args.config.startswith("prefill_"):
         e2e = run_e2e_prefill(kda, base, dev, stream, n_e2e, world)
     else:
-        e2e = run_e2e(kda, base, dev, stream, n_e2e, world)
+        e2e = run_e2e(kda, base, dev, stream, n_e2e, world, args.e2e_sets)
     floor = None if args.no_floor else copy_floor(base, dev, stream, R, args.steps, args.preroll_ms / 1e3)
 
     if world > 1:
@@ -601,20 +601,20 @@ def _timed_steps(fn, steps, stream, lead_in, copy_stream=None):
     return e0.elapsed_time(e1)
 
 
-def run_e2e(kda, w, dev, stream, steps, world):
+def run_e2e(kda, w, dev, stream, steps, world, nsets=2):
     """µs per step with each step's inputs copied from pinned host memory and
     its output copied back, through the public API; the state pool stays
     resident on the GPU.  The value is the pipelined form (``HostPipeline``,
-    the C ABI's ``kda_decode_host_pipelined``): two staging sets used in turn,
-    each step's copy in on a second stream so that it overlaps the previous
-    step's kernel and copy out.  Also reported: the same steps one after
-    another on one stream (``HostStep``, ``kda_decode_host``), and the copy in
-    alone."""
+    the C ABI's ``kda_decode_host_pipelined``): ``nsets`` staging sets used in
+    turn, each step's copy in on a second stream so that it overlaps the
+    previous steps' kernels and copies out.  Also reported: the same steps one
+    after another on one stream (``HostStep``, ``kda_decode_host``), and the
+    copy in alone."""
     import torch
 
     pool = w.state.to(dev)
     copy_stream = torch.cuda.Stream(device=dev)
-    sets = [_host_step(kda, w, dev, stream, pool) for _ in range(2)]
+    sets = [_host_step(kda, w, dev, stream, pool) for _ in range(nsets)]
     pipe = kda.HostPipeline([s[0] for s in sets], copy_stream)
     h2d = sets[0][1].numel()  # the packed buffer each step copies (inputs and their 16-byte alignment)
     d2h = sets[0][3].numel() * sets[0][3].element_size()
@@ -625,7 +625,7 @@ def run_e2e(kda, w, dev, stream, steps, world):
     ms_eager = reduce_max(_timed_steps(pipe, steps, stream, lead_in=4, copy_stream=copy_stream), dev)
     # The same calls captured once into a CUDA graph (as a serving loop replays
     # its decode steps): each replay runs `per_graph` steps, copies included.
-    per_graph = 2 * max(1, min(steps, 64) // 2)
+    per_graph = nsets * max(1, min(steps, 64) // nsets)
     reps = max(1, -(-steps // per_graph))
     graph_note = None
     try:
@@ -656,7 +656,7 @@ def run_e2e(kda, w, dev, stream, steps, world):
             "h2d_copy_us": round(ms_copy * 1e3 / steps, 3),
             "how": "kda_decode_host_pipelined through HostPipeline, one call per step from Python: the copy of "
                    "the step's packed inputs from pinned host memory (on a copy stream, overlapping the previous "
-                   "step), the decode kernel and the copy of the output back to pinned host memory; two staging "
+                   f"step), the decode kernel and the copy of the output back to pinned host memory; {nsets} staging "
                    "sets in turn; the state pool stays resident on the GPU.  graph_us: the same calls captured "
                    f"{per_graph} at a time in a CUDA graph and replayed; serial_us: copy in, kernel and copy out "
                    "one after another on one stream (kda_decode_host); h2d_copy_us: the copy in alone",
@@ -780,6 +780,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--replicas", type=int, default=0, help="0 = enough to exceed 2x L2")
     ap.add_argument("--e2e-steps", type=int, default=5000)
+    ap.add_argument("--e2e-sets", type=int, default=2,
+                    help="staging sets the pipelined end-to-end steps use in turn (>= 1)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-floor", action="store_true", help="skip the in-place copy-floor reference")
