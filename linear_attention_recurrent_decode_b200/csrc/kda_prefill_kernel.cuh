@@ -177,7 +177,7 @@ struct ChunkRaw {
 };
 static_assert(sizeof(ChunkRaw) <= 3 * kK * kCP * sizeof(float), "raw inputs fit over the factor buffers");
 
-constexpr int kChunkThreads = 256;
+constexpr int kChunkThreads = 512;
 
 __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(const Params p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -220,41 +220,46 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   cp_async_wait<0>();
   __syncthreads();
 
-  // Gamma per key channel, summed in fp64 in token order: threads i and
-  // i + 128 each sum one half of the chunk, then the second half adds the
-  // first half's total.  The reference token r is the chunk's middle.
+  // Gamma per key channel, summed in fp64 in token order: four threads per
+  // channel each sum a quarter of the chunk, then each adds the totals of the
+  // quarters before its own.  The reference token r is the chunk's middle.
   constexpr int kRef = kC / 2 - 1;
+  static_assert(kChunkThreads % kK == 0 && kC % (kChunkThreads / kK) == 0, "whole quarters per channel");
+  constexpr int kQT = kC / (kChunkThreads / kK);  // tokens per thread
+  const int ci = tid % kK, cq = tid / kK;          // this thread's channel and part of the chunk
   {
-    const int i = tid % kK, t_lo = (tid / kK) * (kC / 2);
     double acc = 0.0;
 #pragma unroll
-    for (int t = t_lo; t < t_lo + kC / 2; ++t) {
-      acc += static_cast<double>(sm.kt[t][i]);
-      sm.gam[t][i] = acc;
+    for (int t = cq * kQT; t < (cq + 1) * kQT; ++t) {
+      acc += static_cast<double>(sm.kt[t][ci]);
+      sm.gam[t][ci] = acc;
     }
   }
   __syncthreads();
-  if (tid >= kK) {
-    const int i = tid - kK;
-    const double first = sm.gam[kC / 2 - 1][i];
+  {
+    double off = 0.0;
+    for (int q = 0; q < cq; ++q) off += sm.gam[(q + 1) * kQT - 1][ci];
+    __syncthreads();  // every part's total is read before any part adds its offset
+    if (cq > 0) {
 #pragma unroll
-    for (int t = kC / 2; t < kC; ++t) sm.gam[t][i] += first;
+      for (int t = cq * kQT; t < (cq + 1) * kQT; ++t) sm.gam[t][ci] += off;
+    }
   }
   __syncthreads();
-  double gam_end = 0.0, gam_ref = 0.0;  // per channel (threads 0..127)
-  if (tid < kK) {
-    gam_end = sm.gam[kC - 1][tid];
-    gam_ref = sm.gam[kRef][tid];
+  double gam_end = 0.0;  // per channel (the threads of the first part)
+  {
+    const double gam_ref = sm.gam[kRef][ci];
     double worst = 0.0;
-    for (int t = 0; t < kC; ++t) {
-      const double d = sm.gam[t][tid] - gam_ref;
-      worst = fmax(worst, fabs(d));
-    }
+#pragma unroll
+    for (int t = cq * kQT; t < (cq + 1) * kQT; ++t) worst = fmax(worst, fabs(sm.gam[t][ci] - gam_ref));
     // the factored path also forms exp(Gamma_r) and exp(Gamma_C - Gamma_r): keep
     // them normal fp32 numbers
     if (worst > kSafeExp || gam_ref < -kSafeExp) atomicOr(&sm.exact, 1);
-    sm.e_ref[tid] = exp_of(gam_ref);
-    sm.e_end_ref[tid] = exp_of(gam_end - gam_ref);
+    if (cq == 0) {
+      gam_end = sm.gam[kC - 1][ci];
+      sm.e_ref[ci] = exp_of(gam_ref);
+      sm.e_end_ref[ci] = exp_of(gam_end - gam_ref);
+    }
   }
   __syncthreads();
   const bool exact = sm.exact != 0;
@@ -273,9 +278,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
     // The factors go through registers: the raw inputs they are made from live
     // in the buffers they are written to.
     float fa[kPer], fq[kPer], fb[kPer];
-    // each thread keeps one channel i (kChunkThreads is a multiple of K)
-    static_assert(kChunkThreads % kK == 0, "one key channel per thread");
-    const int ci = tid % kK;
+    // each thread keeps its channel ci
     const double g_ref = sm.gam[kRef][ci];
     const float er = sm.e_ref[ci], eer = sm.e_end_ref[ci];
 #pragma unroll
@@ -311,7 +314,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
     __syncthreads();
     // ---- 3. M and P in 4 x 4 tiles of (t, s): the 136 tiles on or below the
     // diagonal go to the first 136 threads (whole warps past them skip the
-    // loop), the tiles above it are zeros written by the rest.
+    // loop), the 120 tiles above it are zeros written by the next 120 threads.
     constexpr int kTb = kC / 4;                           // tile rows (16)
     constexpr int kLower = kTb * (kTb + 1) / 2;          // 136
     int tb, sb;
@@ -350,7 +353,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
           put_pair(p_pl, kPPlane, t, s, kC, (s <= t) ? pv[b] : 0.f);
         }
       }
-    } else {  // the 120 tiles above the diagonal: zeros
+    } else if (tid < kLower + kTb * (kTb - 1) / 2) {  // the 120 tiles above the diagonal: zeros
       // k -> (r, c) with c < r in the strict lower triangle, mirrored to (tb, sb) = (c, r)
       const int k = tid - kLower;
       int r = static_cast<int>((sqrtf(8.f * k + 1.f) + 1.f) * 0.5f);
@@ -407,12 +410,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1) kda_prefill_chunk_kernel(con
   __syncthreads();
 
   // ---- 4. forward substitution: X[t] = beta_t R[t] - sum_{s<t} L[t][s] X[s],
-  // R = [Kt | V]; thread j owns column j (j < K: W, else Ut).  Blocks of 16
+  // R = [Kt | V]; thread j < K + V owns column j (j < K: W, else Ut).  Blocks of 16
   // tokens: the earlier blocks' contribution is a small product over solved
   // rows kept in shared memory (rolled over the blocks), the in-block
   // triangle is unrolled; the same arithmetic as a row-by-row solve with a
   // quarter of the code (the kernel was stalling on instruction fetch).
-  {
+  if (tid < kK + kV) {
     constexpr int kB = 16;                                   // tokens per block
     constexpr int kCols = kK + kV;                           // solve columns
     const int j = tid;
