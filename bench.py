@@ -120,11 +120,21 @@ def prefill_state_flops(w) -> int:
     return w.N * w.HV * (4 * w.T * w.K * w.V + nchunks * w.K * w.V + w.T * w.V)
 
 
-def time_prefill_state_stage(kda, reps, outs, stream, steps):
-    """µs per launch of the prefill's state recurrence (kda_prefill_stage 1, the
-    longest of the call's three kernels): CUDA events on the launching stream
-    around eager launches that rotate over the replicas, each replica's
-    workspace first filled by one whole call."""
+def prefill_output_flops(w) -> int:
+    """Algorithmic flops of the prefill's chunk outputs (stage 2, the tensor-core
+    kernel) for one call: per chunk of Tc tokens and (n, h), Qt S0 (2 Tc K V)
+    and P U (2 Tc Tc V, P lower-triangular but multiplied whole) -- each
+    product counted once, although the kernel runs three bf16 MMAs per product
+    (hi.hi, hi.lo, lo.hi of the split fp32 operands)."""
+    nchunks = (w.T + 63) // 64
+    return w.N * w.HV * nchunks * (2 * 64 * w.K * w.V + 2 * 64 * 64 * w.V)
+
+
+def time_prefill_state_stage(kda, reps, outs, stream, steps, stage=1):
+    """µs per launch of one prefill stage (kda_prefill_stage; 1 = the state
+    recurrence, the longest of the call's three kernels): CUDA events on the
+    launching stream around eager launches that rotate over the replicas, each
+    replica's workspace first filled by one whole call."""
     import torch
 
     fns = []
@@ -136,7 +146,7 @@ def time_prefill_state_stage(kda, reps, outs, stream, steps):
                             stream=stream)
             fns.append(lambda d=d, o=o, ws=ws: kda.kda_prefill(d.q, d.k, d.v, d.g, d.beta, d.state, d.slot_idx,
                                                                out=o, scale=d.scale, workspace=ws, stream=stream,
-                                                               stage=1))
+                                                               stage=stage))
         for f in fns[:3]:
             f()
     n = max(2 * len(fns), min(steps, 200))
@@ -149,6 +159,18 @@ def time_prefill_state_stage(kda, reps, outs, stream, steps):
         b.record(stream)
     torch.cuda.synchronize()
     return a.elapsed_time(b) * 1e3 / n, n
+
+
+def measured_bf16_peak():
+    """Dense bf16 tensor peak in TFLOP/s: the measured burst figure (a kernel
+    timed on its own), else the recipe's earlier measurement on this machine."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
 
 
 def measured_peaks():
@@ -444,7 +466,8 @@ def run_ours(args):
     stage = None
     if args.config.startswith("prefill_"):
         stage_us, stage_n = time_prefill_state_stage(kda, reps, outs, stream, args.steps)
-        stage = (reduce_max(stage_us, dev), stage_n)
+        out_us, _ = time_prefill_state_stage(kda, reps, outs, stream, args.steps, stage=2)
+        stage = (reduce_max(stage_us, dev), stage_n, reduce_max(out_us, dev))
 
     # end to end through the public API: pinned host inputs in, output back out
     n_e2e = min(args.steps, args.e2e_steps)
@@ -489,6 +512,15 @@ def run_ours(args):
                     "launches_timed": stage[1], "traffic": None,
                     "call_hbm": {"achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                                  "frac": round(achieved / peak, 4), "algorithmic_bytes_per_call": bytes_per_call}}
+        bf16_peak, bf16_kind = measured_bf16_peak()
+        oflops = prefill_output_flops(base)
+        otf = oflops / (stage[2] * 1e-6) / 1e12
+        roofline["tensor_kernel"] = {
+            "kernel": "kda_prefill_output_kernel (stage 2: chunk outputs, tcgen05 bf16 MMAs)",
+            "bound": "tensor", "achieved": round(otf, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+            "frac": round(otf / bf16_peak, 4), "peak_source": bf16_kind, "algorithmic_flops_per_launch": oflops,
+            "launch_us": round(stage[2], 2),
+            "note": "each fp32 product counted once; the kernel issues three bf16 MMAs per product"}
     line = {
         "metric": METRIC, "value": round(us_per_call_job, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
