@@ -36,3 +36,25 @@ def test_warmup_below_three_is_refused():
 
     with pytest.raises(SystemExit):
         bench.main(["--impl", "reference", "--steps", "2", "--warmup", "1"])
+
+
+def test_prefill_roofline_counts():
+    """The prefill line's algorithmic flop counts, against a count made here
+    chunk by chunk from the chunk form's products (a ragged last chunk counts
+    its own tokens for the state recurrence and a whole chunk for the output
+    kernel, which multiplies whole 64-row tiles), and the fp32 ALU peak's
+    derivation (148 SMs x 128 lanes x 2 flops x 1965 MHz = 74.4 TFLOP/s)."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class W:
+        N, T, HV, K, V = 3, 150, 2, 128, 128
+
+    w = W()
+    chunks = [64, 64, 22]
+    state = sum(2 * tc * w.K * w.V + w.K * w.V + 2 * w.K * tc * w.V + tc * w.V for tc in chunks)
+    assert bench.prefill_state_flops(w) == w.N * w.HV * state
+    out = sum(2 * 64 * w.K * w.V + 2 * 64 * 64 * w.V for _ in chunks)
+    assert bench.prefill_output_flops(w) == w.N * w.HV * out
+    assert abs(bench.fp32_alu_peak_tflops(148) - 74.4) < 0.05
+    assert abs(bench.fp32_alu_peak_tflops(148, 1000.0) - 37.888) < 1e-9
